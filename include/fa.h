@@ -1,0 +1,113 @@
+/*
+ * fa.h - C ABI of libfa.so: exact fused attention (FlashAttention forward and backward)
+ * for NVIDIA B200 (sm_100a).
+ *
+ * What is computed.  For every (batch b, head h) pair, with Q, K, V the N x d matrices of
+ * that head:
+ *     S = scale * Q K^T                 (scaled scores; "xinc.fun archive 235", section 6
+ *                                        标准注意力为什么慢)
+ *     P = softmax(S) row-wise,  O = P V (exact attention; same section, and "Flash
+ *                                        Attention" on special-jiahao.github.io, section
+ *                                        Standard Attention)
+ * computed tile by tile with a running row max, denominator and unnormalised accumulator
+ * (the online softmax of "xinc.fun archive 235", section 7, a whole key block per step), so
+ * that S and P never reach device memory.  The forward also saves, per query row, the
+ * natural-log log-sum-exp of the scaled scores, LSE_i = ln sum_j exp(S_ij).  The backward
+ * recomputes S and P tile by tile from Q, K and LSE (same section: "recompute local scores
+ * from the saved inputs and a few statistics") and returns
+ *     dV = P^T dO,  dP = dO V^T,  D_i = rowsum(dO o O) = rowsum(P o dP),
+ *     dS = P o (dP - D_i),  dQ = scale * dS K,  dK = scale * dS^T Q.
+ * With causal != 0, key j is visible to query i only when j <= i (square self-attention).
+ *
+ * Layout.  Q, K, V, O, dO, dQ, dK, dV are bf16 tensors [B, H, N, d], contiguous
+ * (row-major: d fastest, then N, then H, then B).  LSE is fp32 [B, H, N], contiguous.
+ * Supported: d in {64, 128} for the forward, d == 128 for the backward; N >= 0;
+ * B * H * N * d < 2^62.  B, H or N equal to 0 is an empty problem: the call returns FA_OK
+ * without launching anything.
+ *
+ * Ownership and memory.  Every pointer is a device pointer owned by the caller; the
+ * library allocates no device memory per call.  Tensors handed to a TMA unit must start on
+ * a 16-byte boundary (q, k, v, o, dO, dq, dk, dv); lse, dQ-workspace need 4-byte alignment.
+ * Outputs are fully overwritten (the backward's dq, dk, dv are not accumulated into).
+ * The only state kept by the library: per-device kernel attributes, set on first use, and
+ * one device status word (see fa_get_device_status).
+ *
+ * Streams and errors.  stream is a cudaStream_t passed as void* (NULL = legacy default
+ * stream).  Calls are asynchronous on that stream.  Argument errors are detected on the
+ * host before any launch and returned synchronously: FA_ERR_INVALID_ARG (null pointer,
+ * negative size, misalignment, non-finite or non-positive scale, causal not 0/1, workspace
+ * too small, size overflow) or FA_ERR_UNSUPPORTED (head dimension, or a device that is not
+ * sm_100).  A failed launch returns FA_ERR_CUDA.  Every wait inside a kernel is bounded;
+ * a wait that runs out sets a bit in the device status word and the kernel exits early
+ * (its outputs are then undefined); fa_get_device_status reports that as FA_ERR_TIMEOUT.
+ * No C++ exception crosses this interface.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,
+  FA_ERR_UNSUPPORTED = 2,
+  FA_ERR_CUDA = 3,
+  FA_ERR_TIMEOUT = 4
+} fa_status_t;
+
+/*
+ * Forward pass ("xinc.fun archive 235", sections 6-7).
+ *   q, k, v : in,  bf16 [B,H,N,d]
+ *   o       : out, bf16 [B,H,N,d]   O = softmax(scale * Q K^T [masked]) V, rounded to bf16
+ *   lse     : out, fp32 [B,H,N]     natural-log log-sum-exp of each row of the scaled,
+ *                                   masked scores (-inf for a row with no visible key)
+ *   scale   : finite, > 0 (1/sqrt(d) for standard attention)
+ *   causal  : 0 or 1
+ */
+fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int B, int H, int N, int d, float scale, int causal, void* stream);
+
+/*
+ * Bytes of device workspace that fa_bwd needs: the fp32 row term D [B*H*N] (rounded up to
+ * 256 bytes) followed by the fp32 dQ accumulator [B*H*N*d].  Returns 0 for an empty or
+ * invalid shape.
+ */
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * Backward pass (recomputation, "xinc.fun archive 235", section 7; formulas above).
+ *   q, k, v, o, dO : in,  bf16 [B,H,N,d]  (o is the forward's output)
+ *   lse            : in,  fp32 [B,H,N]    (the forward's lse)
+ *   dq, dk, dv     : out, bf16 [B,H,N,d]
+ *   workspace      : device scratch of at least fa_bwd_workspace_bytes(B,H,N,d) bytes,
+ *                    256-byte aligned; its contents on entry do not matter and on exit
+ *                    are unspecified.  Concurrent calls need distinct workspaces.
+ */
+fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o,
+                   const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                   void* workspace, size_t workspace_bytes,
+                   int B, int H, int N, int d, float scale, int causal, void* stream);
+
+/*
+ * Synchronises `stream`, reads and clears the device status word of the current device.
+ * Returns FA_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call,
+ * FA_ERR_CUDA if the synchronisation itself failed, FA_OK otherwise.
+ */
+fa_status_t fa_get_device_status(void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* fa_status_string(fa_status_t s);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

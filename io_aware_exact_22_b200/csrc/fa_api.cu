@@ -1,0 +1,202 @@
+// fa_api.cu - the C ABI of libfa.so (declared in include/fa.h): argument validation,
+// TMA tensor-map encoding and kernel launches.  No exception crosses this boundary and no
+// device memory is allocated here.
+#include "fa.h"
+#include "fa_internal.cuh"
+#include "sm100_ptx.cuh"
+
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+namespace fa {
+
+__device__ uint32_t g_fa_status = 0;
+
+uint32_t* device_status_word() {
+  static uint32_t* cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_fa_status) != cudaSuccess) return nullptr;
+  if (dev >= 0 && dev < 64) cached[dev] = static_cast<uint32_t*>(p);
+  return static_cast<uint32_t*>(p);
+}
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Per-device check that the current device is an sm_100 part (cached for up to 64 devices).
+fa_status_t check_device() {
+  static int cached[64];  // 0 unknown, 1 ok, 2 unsupported
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev] == 1 ? FA_OK : FA_ERR_UNSUPPORTED;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return FA_ERR_CUDA;
+  const bool ok = (major == 10 && minor == 0);
+  if (dev >= 0 && dev < 64) cached[dev] = ok ? 1 : 2;
+  return ok ? FA_OK : FA_ERR_UNSUPPORTED;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Shared shape/scalar validation.  Returns FA_OK and sets *empty when there is nothing to do.
+fa_status_t check_shape(int B, int H, int N, int d, float scale, int causal, bool* empty) {
+  *empty = false;
+  if (B < 0 || H < 0 || N < 0) return FA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const long long bh = (long long)B * H;
+  if (bh > INT_MAX) return FA_ERR_INVALID_ARG;
+  if (bh == 0 || N == 0) {
+    *empty = true;
+    return FA_OK;
+  }
+  // element count must stay far from overflow in every index computation
+  if ((long double)bh * N * d >= (long double)(1ull << 62)) return FA_ERR_INVALID_ARG;
+  // one CTA per (head, 256 query rows) in the forward, per (head, 128 keys) in the backward
+  if (bh * ((N + 127) / 128) > INT_MAX) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+size_t dvec_bytes(long long rows) { return ((size_t)rows * 4 + 255) & ~(size_t)255; }
+
+}  // namespace
+
+bool make_tmap_bf16(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+const char* fa_status_string(fa_status_t s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+  }
+  return "FA_ERR_UNKNOWN";
+}
+
+int fa_version(void) { return 100; }
+
+fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                   int N, int d, float scale, int causal, void* stream) {
+  bool empty = false;
+  fa_status_t st = check_shape(B, H, N, d, scale, causal, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return FA_ERR_INVALID_ARG;
+  if ((st = check_device()) != FA_OK) return st;
+  const int BH = B * H;
+  CUtensorMap tq, tk, tv, to;
+  if (!make_tmap_bf16(&tq, q, BH, N, d, 128) || !make_tmap_bf16(&tk, k, BH, N, d, 128) ||
+      !make_tmap_bf16(&tv, v, BH, N, d, 128) || !make_tmap_bf16(&to, o, BH, N, d, 32))
+    return FA_ERR_CUDA;
+  FwdArgs a;
+  if (!(a.status = device_status_word())) return FA_ERR_CUDA;
+  a.lse = lse;
+  a.N = N;
+  a.BH = BH;
+  a.nqb = (N + 255) / 256;
+  a.causal = causal;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  if ((long long)a.BH * a.nqb > INT_MAX) return FA_ERR_INVALID_ARG;
+  return launch_fwd(d, tq, tk, tv, to, a, (cudaStream_t)stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
+  const long long rows = (long long)B * H * N;
+  return dvec_bytes(rows) + (size_t)rows * d * 4;
+}
+
+fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                   const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                   size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
+                   void* stream) {
+  bool empty = false;
+  fa_status_t st = check_shape(B, H, N, d, scale, causal, &empty);
+  if (st != FA_OK || empty) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dO, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) ||
+      !aligned(workspace, 256))
+    return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  if ((st = check_device()) != FA_OK) return st;
+  const int BH = B * H;
+  const long long rows = (long long)BH * N;
+  float* dvec = reinterpret_cast<float*>(workspace);
+  float* dq_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + dvec_bytes(rows));
+  cudaStream_t s = (cudaStream_t)stream;
+  CUtensorMap tq, tk, tv, tdo, tdk, tdv;
+  if (!make_tmap_bf16(&tq, q, BH, N, d, 128) || !make_tmap_bf16(&tk, k, BH, N, d, 128) ||
+      !make_tmap_bf16(&tv, v, BH, N, d, 128) || !make_tmap_bf16(&tdo, dO, BH, N, d, 128) ||
+      !make_tmap_bf16(&tdk, dk, BH, N, d, 32) || !make_tmap_bf16(&tdv, dv, BH, N, d, 32))
+    return FA_ERR_CUDA;
+  BwdArgs a;
+  if (!(a.status = device_status_word())) return FA_ERR_CUDA;
+  a.lse = lse;
+  a.dvec = dvec;
+  a.dq_acc = dq_acc;
+  a.N = N;
+  a.BH = BH;
+  a.causal = causal;
+  a.scale = scale;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  if (launch_bwd_pre(o, dO, dvec, dq_acc, rows, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  cudaError_t e = launch_bwd_main(d, tq, tk, tv, tdo, tdk, tdv, a, s);
+  if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return FA_ERR_CUDA;
+  if (launch_bwd_post(dq_acc, dq, rows * d, scale, s) != cudaSuccess) return FA_ERR_CUDA;
+  return FA_OK;
+}
+
+fa_status_t fa_get_device_status(void* stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return FA_ERR_CUDA;
+  uint32_t h = 0;
+  const uint32_t zero = 0;
+  if (cudaMemcpyFromSymbol(&h, g_fa_status, sizeof(h)) != cudaSuccess) return FA_ERR_CUDA;
+  if (h != 0 && cudaMemcpyToSymbol(g_fa_status, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
+  return h ? FA_ERR_TIMEOUT : FA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,354 @@
+// fa_fwd.cu - fused exact-attention forward for sm_100a (tcgen05 + TMEM + TMA).
+//
+// Method: the online softmax of "xinc.fun archive 235", section 7 (running max m, denominator
+// l and unnormalised accumulator z per query row, o = z / l at the end), one key block of 128
+// keys per step, so that the scores S = scale * Q K^T (section 6) and probabilities P never
+// leave the SM.  The running max is kept as a reference value that only moves when a block's
+// max exceeds it by more than 2^8 (in base-2 units); z and l are relative to that reference,
+// which cancels in z / l (see the two-block merge identities of "Flash Attention",
+// special-jiahao.github.io, section 增量求解 softmax), and every exponent stays <= 2^8.
+//
+// One CTA owns 256 query rows of one (batch, head) as two 128-row tiles and streams the K/V
+// blocks through a shared-memory ring.  Roles (320 threads):
+//   warps 0-3  softmax warpgroup for query tile 0   (one thread per query row)
+//   warps 4-7  softmax warpgroup for query tile 1
+//   warp  8    MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j on the tensor core
+//   warp  9    TMA producer (one thread): Q tiles once, then K_j, V_j into the ring
+// TMEM (512 columns x 128 lanes, fp32): S_0 [0,128), S_1 [128,256), O_0 [256,256+d),
+// O_1 [256+d, 256+2d).  P_t (bf16, two per column) overwrites the first 64 columns of S_t.
+// While softmax warpgroup 0 works on S_0, the tensor core runs tile 1's MMAs and vice versa.
+#include "fa_internal.cuh"
+#include "sm100_ptx.cuh"
+
+#include <cmath>
+
+namespace fa {
+
+using namespace ptx;
+
+template <int D>
+struct FwdCfg {
+  static constexpr int NBOX = D / 64;              // 64-column (128-byte) swizzle boxes per row
+  static constexpr int TILE = 128 * D * 2;         // bytes of one 128-row bf16 tile
+  static constexpr int NS = (D == 128) ? 4 : 8;    // K/V ring stages (one K or one V each)
+  static constexpr int Q_OFF = 0;
+  static constexpr int KV_OFF = 2 * TILE;
+  static constexpr int BAR_OFF = KV_OFF + NS * TILE;
+  // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_full
+  static constexpr int NBAR = 1 + 2 * NS + 2 + 2 + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int SMEM = MISC_OFF + 16 + 1024;  // + slack to align the base to 1024
+  static constexpr int THREADS = 320;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t IDESC_QK = idesc_bf16(128, 128, false, false);
+  static constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                  const FwdArgs a) {
+  using C = FwdCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  uint8_t* gb = smem_raw + (sb - raw);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item: (head bh, block of 256 query rows); heavier causal blocks first
+  const int bh = blockIdx.x / a.nqb;
+  const int qb = a.nqb - 1 - (blockIdx.x % a.nqb);
+  const int q0 = qb * 256;
+  const int Tk = (a.N + 127) >> 7;
+  const bool has1 = (q0 + 128) < a.N;
+  const int n0 = a.causal ? min(Tk, 2 * qb + 1) : Tk;
+  const int n1 = has1 ? (a.causal ? min(Tk, 2 * qb + 2) : Tk) : 0;
+  const int nmax = max(n0, n1);
+
+  const uint32_t bar = sb + C::BAR_OFF;
+  const uint32_t q_full = bar;
+  auto kv_full = [&](int s) { return bar + 8u * (1 + s); };
+  auto kv_empty = [&](int s) { return bar + 8u * (1 + C::NS + s); };
+  auto s_full = [&](int t) { return bar + 8u * (1 + 2 * C::NS + t); };
+  auto p_full = [&](int t) { return bar + 8u * (3 + 2 * C::NS + t); };
+  const uint32_t o_full = bar + 8u * (5 + 2 * C::NS);
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gb + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + C::MISC_OFF + 4);
+  const WaitCtx wc{abort_flag, a.status};
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(s_full(t), 1);
+      mbar_init(p_full(t), 128);
+    }
+    mbar_init(o_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(sb + C::MISC_OFF, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 9) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && !*abort_flag) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      const uint64_t keep = policy_evict_last();
+      const int nq = has1 ? 2 : 1;
+      mbar_arrive_expect_tx(q_full, nq * C::TILE);
+      for (int t = 0; t < nq; ++t)
+        for (int b = 0; b < C::NBOX; ++b)
+          tma_load_3d(sb + C::Q_OFF + t * C::TILE + b * 16384, &tmQ, q_full, 64 * b, q0 + 128 * t, bh);
+      int it = 0;
+      bool ok = true;
+      for (int j = 0; j < nmax && ok; ++j) {
+        for (int kv = 0; kv < 2; ++kv, ++it) {
+          const int s = it % C::NS;
+          const uint32_t ph = (it / C::NS) & 1;
+          if (!mbar_wait(kv_empty(s), ph ^ 1, wc)) { ok = false; break; }
+          mbar_arrive_expect_tx(kv_full(s), C::TILE);
+          const CUtensorMap* m = kv ? &tmV : &tmK;
+          for (int b = 0; b < C::NBOX; ++b)
+            tma_load_3d_hint(sb + C::KV_OFF + s * C::TILE + b * 16384, m, kv_full(s), 64 * b, 128 * j,
+                             bh, keep);
+        }
+      }
+      if (!ok) {  // let copies already issued land before the CTA exits
+        mbar_wait_drain(q_full, 0);
+        for (int back = 1; back <= C::NS && it - back >= 0; ++back) {
+          const int i2 = it - back;
+          mbar_wait_drain(kv_full(i2 % C::NS), (i2 / C::NS) & 1);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && !*abort_flag) {
+      const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
+      const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
+      const int nt[2] = {n0, n1};
+      auto issue_qk = [&](uint32_t dst, uint32_t qaddr, uint32_t kaddr) {
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+          mma_ss(dst, sdesc_sw128(qaddr + off, 16, 1024), sdesc_sw128(kaddr + off, 16, 1024),
+                 C::IDESC_QK, k > 0);
+        }
+      };
+      auto issue_pv = [&](uint32_t dst, uint32_t ptm, uint32_t vaddr, bool acc) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mma_ts(dst, ptm + 8 * k, sdesc_sw128(vaddr + k * 2048, 16384, 1024), C::IDESC_PV,
+                 (acc || k > 0) ? 1u : 0u);
+      };
+      auto stage_addr = [&](int it) { return sb + C::KV_OFF + (it % C::NS) * C::TILE; };
+      auto stage_par = [&](int it) { return (uint32_t)((it / C::NS) & 1); };
+      bool ok = mbar_wait(q_full, 0, wc);
+      if (ok) ok = mbar_wait(kv_full(0), 0, wc);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t)
+          if (nt[t] > 0) {
+            issue_qk(tS[t], sb + C::Q_OFF + t * C::TILE, stage_addr(0));
+            mma_commit(s_full(t));
+          }
+        mma_commit(kv_empty(0));
+      }
+      for (int j = 0; j < nmax && ok; ++j) {
+        const int itK = 2 * (j + 1), itV = 2 * j + 1;  // ring positions of K_{j+1} and V_j
+        if (!(ok = mbar_wait(kv_full(itV % C::NS), stage_par(itV), wc))) break;
+        tc_fence_after();
+        bool k_ready = false;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j >= nt[t]) continue;
+          if (!(ok = mbar_wait(p_full(t), j & 1, wc))) break;
+          tc_fence_after();
+          issue_pv(tO[t], tS[t], stage_addr(itV), j > 0);
+          if (j + 1 < nt[t]) {
+            if (!k_ready) {
+              if (!(ok = mbar_wait(kv_full(itK % C::NS), stage_par(itK), wc))) break;
+              tc_fence_after();
+              k_ready = true;
+            }
+            issue_qk(tS[t], sb + C::Q_OFF + t * C::TILE, stage_addr(itK));
+            mma_commit(s_full(t));
+          }
+        }
+        if (!ok) break;
+        mma_commit(kv_empty(itV % C::NS));
+        if (k_ready) mma_commit(kv_empty(itK % C::NS));
+      }
+      mma_commit(o_full);
+      if (!ok) mbar_wait_drain(o_full, 0);  // every issued MMA has completed before TMEM is freed
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int t = warp >> 2;
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;  // row within the query tile == TMEM lane
+    const int ntile = t ? n1 : n0;
+    const int qrow = q0 + 128 * t + r;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tSrow = tmem + lane_off + 128u * t;
+    const uint32_t tOrow = tmem + lane_off + 256u + (uint32_t)(D * t);
+    const float cs = a.scale_log2;
+    float m_ref = -INFINITY;  // reference max, base-2 scaled units
+    float l = 0.f;
+    bool ok = !*abort_flag;
+
+    for (int j = 0; j < ntile && ok; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full(t), j & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[128];
+      tmem_ld32(tSrow + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tSrow + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tSrow + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+      tmem_ld32(tSrow + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+      tmem_wait_ld();
+      reg_fence(sr);
+      float x[128];
+#pragma unroll
+      for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
+      if (j == ntile - 1) {  // the only block that can hold the diagonal or the ragged tail
+        int lim = a.N - 1 - 128 * j;
+        if (a.causal) lim = min(lim, qrow - 128 * j);
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c > lim) x[c] = -INFINITY;
+      }
+      float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
+#pragma unroll
+      for (int c = 4; c < 128; c += 4) {
+        mx0 = fmaxf(mx0, x[c]);
+        mx1 = fmaxf(mx1, x[c + 1]);
+        mx2 = fmaxf(mx2, x[c + 2]);
+        mx3 = fmaxf(mx3, x[c + 3]);
+      }
+      const float mblk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * cs;
+      const bool move = mblk > m_ref + 8.0f;
+      float alpha = 1.f;
+      if (move) {
+        alpha = ex2(m_ref - mblk);  // 0 when m_ref is still -inf
+        m_ref = mblk;
+      }
+      if (__any_sync(0xffffffffu, move && j > 0)) {
+        // O_t holds sum_{j' < j} of P V relative to the old reference: rescale by alpha.
+#pragma unroll 1
+        for (int cc = 0; cc < D; cc += 32) {
+          uint32_t o[32];
+          tmem_ld32(tOrow + cc, o);
+          tmem_wait_ld();
+          reg_fence(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tOrow + cc, o);
+        }
+      }
+      l *= alpha;
+      const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      float rs0 = 0.f, rs1 = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 128; c += 2) {
+        const float p0 = ex2(fmaf(x[c], cs, mneg));
+        const float p1 = ex2(fmaf(x[c + 1], cs, mneg));
+        rs0 += p0;
+        rs1 += p1;
+        pk[c >> 1] = pack_bf16(p0, p1);
+      }
+      l += rs0 + rs1;
+      tmem_st32(tSrow + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(tSrow + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full(t));
+    }
+
+    if (ntile > 0 && ok) {
+      // ---------------------------------------------------------- epilogue
+      ok = __all_sync(0xffffffffu, mbar_wait(o_full, 0, wc));
+      if (ok) {
+        tc_fence_after();
+        const float inv = (l > 0.f) ? 1.f / l : 0.f;
+        uint8_t* stage = gb + C::Q_OFF + t * C::TILE;  // Q_t is dead once o_full has fired
+#pragma unroll
+        for (int b = 0; b < C::NBOX; ++b) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t o[32];
+            tmem_ld32(tOrow + 64 * b + 32 * h, o);
+            tmem_wait_ld();
+            reg_fence(o);
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              uint4 v;
+              v.x = pack_bf16(__uint_as_float(o[8 * cc + 0]) * inv, __uint_as_float(o[8 * cc + 1]) * inv);
+              v.y = pack_bf16(__uint_as_float(o[8 * cc + 2]) * inv, __uint_as_float(o[8 * cc + 3]) * inv);
+              v.z = pack_bf16(__uint_as_float(o[8 * cc + 4]) * inv, __uint_as_float(o[8 * cc + 5]) * inv);
+              v.w = pack_bf16(__uint_as_float(o[8 * cc + 6]) * inv, __uint_as_float(o[8 * cc + 7]) * inv);
+              const int chunk = h * 4 + cc;  // 16-byte chunk within the 128-byte row
+              *reinterpret_cast<uint4*>(stage + b * 16384 + r * 128 + ((chunk ^ (r & 7)) << 4)) = v;
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        const int row0 = q0 + 128 * t + 32 * wq;
+        if (lane == 0 && row0 < a.N) {
+          for (int b = 0; b < C::NBOX; ++b)
+            tma_store_3d(&tmO, sb + C::Q_OFF + t * C::TILE + b * 16384 + wq * 4096, 64 * b, row0, bh);
+          bulk_commit();
+          bulk_wait_read0();
+        }
+        __syncwarp();
+        if (qrow < a.N)
+          a.lse[(size_t)bh * a.N + qrow] =
+              (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int D>
+static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                const CUtensorMap& to, const FwdArgs& a, cudaStream_t stream) {
+  using C = FwdCfg<D>;
+  static_assert(C::SMEM <= 232448, "shared memory budget");
+  cudaError_t e = cudaFuncSetAttribute(fa_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const long long grid = (long long)a.BH * a.nqb;
+  fa_fwd_kernel<D><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, to, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& to, const FwdArgs& a, cudaStream_t stream) {
+  if (d == 64) return launch_fwd_t<64>(tq, tk, tv, to, a, stream);
+  return launch_fwd_t<128>(tq, tk, tv, to, a, stream);
+}
+
+}  // namespace fa

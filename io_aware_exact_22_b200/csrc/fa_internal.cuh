@@ -1,0 +1,50 @@
+// fa_internal.cuh - declarations shared by the host side of libfa.so (not part of the ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace fa {
+
+struct FwdArgs {
+  uint32_t* status;  // device status word
+  float* lse;        // [BH, N] fp32
+  int N;             // sequence length
+  int BH;            // batch * heads
+  int nqb;           // query blocks of 256 rows per head
+  int causal;        // 0 / 1
+  float scale_log2;  // scale * log2(e)
+};
+
+struct BwdArgs {
+  uint32_t* status;  // device status word
+  const float* lse;  // [BH, N] fp32, natural log
+  const float* dvec; // [BH, N] fp32, D_i = rowsum(dO o O)
+  float* dq_acc;     // [BH, N, d] fp32 accumulator (zeroed by the pre-kernel)
+  int N;
+  int BH;
+  int causal;
+  float scale;       // softmax scale
+  float scale_log2;  // scale * log2(e)
+};
+
+// Device address of this library's status word on the current device (nullptr on error).
+uint32_t* device_status_word();
+
+// Tensor maps for a bf16 [BH, N, d] tensor, 128-byte swizzle, box = 64 columns x `rows`.
+bool make_tmap_bf16(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_rows);
+
+cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& to, const FwdArgs& a, cudaStream_t stream);
+
+cudaError_t launch_bwd_pre(const void* o, const void* dO, float* dvec, float* dq_acc,
+                           long long rows, int d, cudaStream_t stream);
+cudaError_t launch_bwd_main(int d, const CUtensorMap& tq, const CUtensorMap& tk,
+                            const CUtensorMap& tv, const CUtensorMap& tdo,
+                            const CUtensorMap& tdk, const CUtensorMap& tdv, const BwdArgs& a,
+                            cudaStream_t stream);
+cudaError_t launch_bwd_post(const float* dq_acc, void* dq, long long elems, float scale,
+                            cudaStream_t stream);
+
+}  // namespace fa

@@ -1,0 +1,145 @@
+"""ctypes binding over libfa.so (C ABI in include/fa.h).
+
+The functions ``fa_fwd``, ``fa_bwd``, ``fa_bwd_workspace_bytes``, ``fa_get_device_status``,
+``fa_status_string`` and ``fa_version`` carry the C names and only marshal arguments: torch
+tensors supply device pointers and the current CUDA stream, and every step of the attention
+path runs in the library's kernels.  ``forward`` / ``backward`` additionally allocate the
+output tensors with torch (memory plumbing only).
+
+Loading fails loudly (``RuntimeError``) when the shared library is missing: there is no
+fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.environ.get("FA_LIB_PATH", os.path.join(_HERE, "libfa.so"))
+
+STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_CUDA",
+          4: "FA_ERR_TIMEOUT"}
+EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_device_status",
+           "fa_status_string", "fa_version")
+
+_lib = None
+
+
+class FAError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what} failed: {STATUS.get(code, code)}")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfa.so once; raise RuntimeError if it is not built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libfa.so not found at {LIB_PATH}; build it with "
+                               "`python -m io_aware_exact_22_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+        L.fa_fwd.restype = i
+        L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, vp]
+        L.fa_bwd.restype = i
+        L.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
+        L.fa_bwd_workspace_bytes.restype = sz
+        L.fa_get_device_status.argtypes = [vp]
+        L.fa_get_device_status.restype = i
+        L.fa_status_string.argtypes = [i]
+        L.fa_status_string.restype = ctypes.c_char_p
+        L.fa_version.argtypes = []
+        L.fa_version.restype = i
+        _lib = L
+    return _lib
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# ------------------------------------------------------------------ C-named wrappers
+def fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, stream=None) -> int:
+    return lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                        float(scale), int(causal), _stream(stream))
+
+
+def fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes, B, H, N, d, scale,
+           causal, stream=None) -> int:
+    return lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq),
+                        _ptr(dk), _ptr(dv), _ptr(workspace), int(workspace_bytes), B, H, N, d,
+                        float(scale), int(causal), _stream(stream))
+
+
+def fa_bwd_workspace_bytes(B, H, N, d) -> int:
+    return lib().fa_bwd_workspace_bytes(B, H, N, d)
+
+
+def fa_get_device_status(stream=None) -> int:
+    return lib().fa_get_device_status(_stream(stream))
+
+
+def fa_status_string(code: int) -> str:
+    return lib().fa_status_string(code).decode()
+
+
+def fa_version() -> int:
+    return lib().fa_version()
+
+
+# ------------------------------------------------------------------ tensor conveniences
+def _check(t, name):
+    if not (t.is_cuda and t.dtype == torch.bfloat16 and t.dim() == 4 and t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor [B,H,N,d]")
+
+
+def forward(q, k, v, causal: bool, scale: float | None = None, out=None, lse=None):
+    """O, LSE = attention(q, k, v) through fa_fwd.  Inputs: contiguous bf16 [B,H,N,d] on CUDA."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n)
+    B, H, N, d = q.shape
+    scale = d ** -0.5 if scale is None else scale
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+    rc = fa_fwd(q, k, v, out, lse, B, H, N, d, scale, causal)
+    if rc:
+        raise FAError(rc, "fa_fwd")
+    return out, lse
+
+
+def backward(q, k, v, o, do, lse, causal: bool, scale: float | None = None, workspace=None,
+             dq=None, dk=None, dv=None):
+    """dQ, dK, dV through fa_bwd (workspace allocated with torch when not given)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "dO")):
+        _check(t, n)
+    B, H, N, d = q.shape
+    scale = d ** -0.5 if scale is None else scale
+    nbytes = fa_bwd_workspace_bytes(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 256), device=q.device, dtype=torch.uint8)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    rc = fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, workspace.numel(), B, H, N, d, scale,
+                causal)
+    if rc:
+        raise FAError(rc, "fa_bwd")
+    return dq, dk, dv
