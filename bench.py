@@ -1,0 +1,387 @@
+"""Attention benchmark on B200: one step = the whole hot path (fused forward, then backward
+with recomputation) over one batch of synthetic input, through libfa.so's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload 4]
+                    [--no-cpu-baseline] [--no-e2e]
+
+Default workload: the long-sequence causal shape B=1, H=32, N=16384, d=128, bf16, q,k ~ N(0,3),
+v, dO ~ N(0,1), scale 1/sqrt(128).  Metric: attention TFLOPS, with 4*B*H*N^2*d for the forward,
+2.5x that for the backward, halved for causal.  Prints ONE JSON line (rank 0).
+
+Multi-GPU (launched under torch.distributed.run): every rank runs its own copy of the workload
+(independent heads; attention has no exchange step), timing is the max over ranks and
+`value` totals the work of all ranks (weak scaling).
+
+`--impl reference` times the fp64 CPU oracle (plain standard attention that materialises S
+and P) on the host cores, one bounded sample of the workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from io_aware_exact_22_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "attention TFLOPS (fwd/bwd, causal halved) and % of B200 BF16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def step_workload(wid: int):
+    w = WORKLOADS[wid]
+    # the step is forward + backward at this shape; dO ~ N(0,1) is drawn after q, k, v
+    return w
+
+
+# ---------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        loaded = [x for x in sm if x > 0.5 * max(sm)] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows),
+                "power_w_max": max((float(r[3]) for r in rows
+                                    if r[3].replace(".", "").isdigit()), default=None)}
+
+
+# ---------------------------------------------------------------------- traffic
+def kernel_traffic(name: str, src_file: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    ent = t.get(name)
+    if not ent:
+        return None
+    with open(os.path.join(ROOT, src_file), "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    return ent.get("bytes_per_launch") if ent.get("source_sha") == sha else None
+
+
+# ---------------------------------------------------------------------- GPU arm
+def run_gpu(args):
+    from io_aware_exact_22_b200 import fa
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    w = step_workload(args.workload)
+    B, H, N, d = w.shape
+    q, k, v = make_inputs(w, with_grad=False)
+    g = torch.Generator("cpu").manual_seed(w.seed + 1)
+    do = torch.randn(w.shape, generator=g).to(torch.bfloat16)
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o = torch.empty_like(qd)
+    lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    ws_bytes = fa.fa_bwd_workspace_bytes(B, H, N, d)
+    ws = torch.empty(ws_bytes, device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    scale = w.scale
+
+    def step():
+        rc = fa.fa_fwd(qd, kd, vd, o, lse, B, H, N, d, scale, w.causal, sp)
+        rc |= fa.fa_bwd(qd, kd, vd, o, dod, lse, dq, dk, dv, ws, ws_bytes, B, H, N, d, scale,
+                        w.causal, sp)
+        if rc:
+            raise RuntimeError(f"fa call failed: {rc}")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if fa.fa_get_device_status(sp) != 0:
+        raise RuntimeError("device-side timeout during warm-up")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    n_ev = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_ev)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        rc = fa.fa_fwd(qd, kd, vd, o, lse, B, H, N, d, scale, w.causal, sp)
+        ev[i][1].record(stream)
+        rc |= fa.fa_bwd(qd, kd, vd, o, dod, lse, dq, dk, dv, ws, ws_bytes, B, H, N, d, scale,
+                        w.causal, sp)
+        ev[i][2].record(stream)
+        if rc:
+            raise RuntimeError(f"fa call failed: {rc}")
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    status = fa.fa_get_device_status(sp)
+    total_ms = t0.elapsed_time(t1)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    if world > 1:
+        t = torch.tensor([total_ms, fwd_ms, bwd_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms, fwd_ms, bwd_ms = t.tolist()
+    ms_per_step = total_ms / args.steps
+    flops_step = w.fwd_flops() + w.bwd_flops()
+    value = flops_step * world / (ms_per_step * 1e-3) / 1e12
+
+    # ------------------------------------------------------------ end-to-end (host buffers)
+    e2e = None
+    if not args.no_e2e:
+        pin = [t.pin_memory() for t in (q, k, v, do)]
+        outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, dq, dk, dv)]
+        lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in pin)
+        d2h = sum(t.numel() * t.element_size() for t in outs) + lse_h.numel() * 4
+
+        def e2e_step():
+            for src, dst in zip(pin, (qd, kd, vd, dod)):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for src, dst in zip((o, dq, dk, dv), outs):
+                dst.copy_(src, non_blocking=True)
+            lse_h.copy_(lse, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        k_e2e = max(3, min(args.steps, 10))
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            torch.distributed.barrier()
+        a0.record(stream)
+        for _ in range(k_e2e):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = a0.elapsed_time(a1) / k_e2e
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e_ms = t.item()
+        e2e = {"value": flops_step * world / (e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "steps": k_e2e, "api": "io_aware_exact_22_b200.fa.fa_fwd/fa_bwd from pinned host"}
+
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return None
+
+    peaks, peak_src = load_peaks()
+    peak = peaks["bf16_tflops"]
+    bwd_tflops = w.bwd_flops() / (bwd_ms * 1e-3) / 1e12
+    fwd_tflops = w.fwd_flops() / (fwd_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOPS",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
+                   "step": "fa_fwd + fa_bwd", "per_rank": "same workload on every rank",
+                   "l2": "inputs larger than L2 (q,k,v,o,dO 134 MB each vs 126 MB L2), no flush"},
+        "pct_of_peak": round(100 * value / world / peak, 2),
+        "fwd": {"ms": round(fwd_ms, 4), "tflops": round(fwd_tflops, 1),
+                "pct_of_peak": round(100 * fwd_tflops / peak, 2)},
+        "bwd": {"ms": round(bwd_ms, 4), "tflops": round(bwd_tflops, 1),
+                "pct_of_peak": round(100 * bwd_tflops / peak, 2)},
+        "roofline": {"kernel": "fa_bwd (main kernel + memory-bound pre/post, timed together)",
+                     "bound": "tensor", "achieved": round(bwd_tflops, 1), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(bwd_tflops / peak, 4),
+                     "traffic": kernel_traffic("fa_bwd_main_kernel",
+                                               "io_aware_exact_22_b200/csrc/fa_bwd.cu"),
+                     "peak_source": f"{peak_src} bf16_tflops (burst)",
+                     "algorithmic_flops_per_launch": w.bwd_flops()},
+        "roofline_fwd": {"kernel": "fa_fwd_kernel<128>", "bound": "tensor",
+                         "achieved": round(fwd_tflops, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(fwd_tflops / peak, 4),
+                         "traffic": kernel_traffic("fa_fwd_kernel",
+                                                   "io_aware_exact_22_b200/csrc/fa_fwd.cu"),
+                         "algorithmic_flops_per_launch": w.fwd_flops()},
+        "clocks": clk,
+        "gpu_launches": 4 * args.steps,
+        "device_status": status,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, q, k, v, do)
+    return line
+
+
+# ---------------------------------------------------------------------- CPU (oracle) arms
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def _oracle_sample(w, q, k, v, do, heads, rows):
+    """Oracle fwd + bwd on the given (b, h) heads, restricted to query `rows` (None = all)."""
+    import oracle
+    from io_aware_exact_22_b200.inputs import to_f64
+    t0 = time.perf_counter()
+    for b, h in heads:
+        qh, kh, vh, dh = (to_f64(t[b, h]) for t in (q, k, v, do))
+        oracle.attention_forward_head(qh, kh, vh, w.scale, w.causal, rows=rows)
+        oracle.attention_backward_head(qh, kh, vh, dh, w.scale, w.causal, rows=rows)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, q, k, v, do):
+    heads = [(0, 0), (0, 1)]
+    secs = _oracle_sample(w, q, k, v, do, heads, None)
+    frac = len(heads) / (w.B * w.H)
+    flops = (w.fwd_flops() + w.bwd_flops()) * frac
+    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOPS", "cores": _blas_threads(),
+            "kind": "oracle", "seconds": round(secs, 2),
+            "sample": f"oracle fwd+bwd on {len(heads)} of {w.B * w.H} heads (full N={w.N}), "
+                      "fp64 numpy, materialised S and P; metric FLOPs scaled by the head fraction"}
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    w = step_workload(args.workload)
+    q, k, v = make_inputs(w, with_grad=False)
+    g = torch.Generator("cpu").manual_seed(w.seed + 1)
+    do = torch.randn(w.shape, generator=g).to(torch.bfloat16)
+    R = 128
+    rows = np.linspace(0, w.N - 1, R).round().astype(np.int64)
+    frac = R / (w.B * w.H * w.N)
+    flops = (w.fwd_flops() + w.bwd_flops()) * frac
+    for _ in range(args.warmup):
+        _oracle_sample(w, q, k, v, do, [(0, 0)], rows)
+    secs = [_oracle_sample(w, q, k, v, do, [(0, 0)], rows) for _ in range(args.steps)]
+    ms = 1e3 * sum(secs) / len(secs)
+    value = flops / (ms * 1e-3) / 1e12
+    sample = (f"oracle fwd+bwd for {R} query rows spread over the sequence of head (0,0), "
+              "fp64 numpy; metric FLOPs scaled by the row fraction")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOPS",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                       "causal": w.causal, "step": "oracle fwd + bwd (bounded row sample)"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": _blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["fa", "reference"], default="fa")
+    ap.add_argument("--workload", type=int, default=4, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, _, _ = dist_env()
+    if world != args.gpus:
+        if args.gpus > 1 and world == 1:
+            ap.error("run multi-GPU through torch.distributed.run (one process per GPU)")
+    line = run_reference(args) if args.impl == "reference" else run_gpu(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -73,9 +73,9 @@ fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* 
                    int B, int H, int N, int d, float scale, int causal, void* stream);
 
 /*
- * Bytes of device workspace that fa_bwd needs: the fp32 row term D [B*H*N] (rounded up to
- * 256 bytes) followed by the fp32 dQ accumulator [B*H*N*d].  Returns 0 for an empty or
- * invalid shape.
+ * Bytes of device workspace that fa_bwd needs: per 64-row query tile, the fp32 base-2 LSE and
+ * row term D_i of its 64 rows (B*H*ceil(N/64)*128 floats, rounded up to 256 bytes), followed
+ * by the fp32 dQ accumulator [B*H*N*d].  Returns 0 for an empty or invalid shape.
  */
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 

@@ -79,7 +79,11 @@ fa_status_t check_shape(int B, int H, int N, int d, float scale, int causal, boo
   return FA_OK;
 }
 
-size_t dvec_bytes(long long rows) { return ((size_t)rows * 4 + 255) & ~(size_t)255; }
+// Per-query-tile statistics of the backward: [BH][ceil(N/64)][128] fp32, rounded to 256 bytes.
+size_t ld_bytes(long long bh, int N) {
+  const long long tiles = bh * ((N + 63) / 64);
+  return ((size_t)tiles * 128 * 4 + 255) & ~(size_t)255;
+}
 
 }  // namespace
 
@@ -144,7 +148,7 @@ fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* 
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
   const long long rows = (long long)B * H * N;
-  return dvec_bytes(rows) + (size_t)rows * d * 4;
+  return ld_bytes((long long)B * H, N) + (size_t)rows * d * 4;
 }
 
 fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
@@ -164,25 +168,25 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
   if ((st = check_device()) != FA_OK) return st;
   const int BH = B * H;
   const long long rows = (long long)BH * N;
-  float* dvec = reinterpret_cast<float*>(workspace);
-  float* dq_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + dvec_bytes(rows));
+  float* ld = reinterpret_cast<float*>(workspace);
+  float* dq_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + ld_bytes(BH, N));
   cudaStream_t s = (cudaStream_t)stream;
   CUtensorMap tq, tk, tv, tdo, tdk, tdv;
-  if (!make_tmap_bf16(&tq, q, BH, N, d, 128) || !make_tmap_bf16(&tk, k, BH, N, d, 128) ||
-      !make_tmap_bf16(&tv, v, BH, N, d, 128) || !make_tmap_bf16(&tdo, dO, BH, N, d, 128) ||
+  if (!make_tmap_bf16(&tq, q, BH, N, d, 64) || !make_tmap_bf16(&tk, k, BH, N, d, 128) ||
+      !make_tmap_bf16(&tv, v, BH, N, d, 128) || !make_tmap_bf16(&tdo, dO, BH, N, d, 64) ||
       !make_tmap_bf16(&tdk, dk, BH, N, d, 32) || !make_tmap_bf16(&tdv, dv, BH, N, d, 32))
     return FA_ERR_CUDA;
   BwdArgs a;
   if (!(a.status = device_status_word())) return FA_ERR_CUDA;
   a.lse = lse;
-  a.dvec = dvec;
+  a.ld = ld;
   a.dq_acc = dq_acc;
   a.N = N;
   a.BH = BH;
   a.causal = causal;
   a.scale = scale;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
-  if (launch_bwd_pre(o, dO, dvec, dq_acc, rows, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (launch_bwd_pre(o, dO, lse, ld, dq_acc, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
   cudaError_t e = launch_bwd_main(d, tq, tk, tv, tdo, tdk, tdv, a, s);
   if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
   if (e != cudaSuccess) return FA_ERR_CUDA;

@@ -1,19 +1,482 @@
-// fa_bwd.cu - backward of exact attention (recomputation; "xinc.fun archive 235", section 7).
+// fa_bwd.cu - backward of exact attention for sm_100a, by recomputation ("xinc.fun archive
+// 235", section 7: the backward recomputes the local scores from the saved inputs and a few
+// per-row statistics instead of reading an N x N matrix).
+//
+// With S = scale Q K^T, P = softmax(S) and the saved LSE_i = ln sum_j exp(S_ij):
+//   P_ij = exp(S_ij - LSE_i),  dV = P^T dO,  dP = dO V^T,  D_i = rowsum(dO o O),
+//   dS = P o (dP - D_i),  dQ = scale dS K,  dK = scale dS^T Q.
+//
+// Three kernels:
+//   K2 fa_bwd_pre   per query row: D_i and LSE_i * log2(e), stored per 64-row query tile as
+//                   [64 x LSE2 | 64 x D] (rows past N get LSE2 = +inf, D = 0, i.e. P = 0), and
+//                   zeroes the fp32 dQ accumulator.  Memory-bound.
+//   K3 fa_bwd_main  one CTA per (head, 128-key tile j); K_j and V_j stay in shared memory and
+//                   the 64-row query tiles i stream through a 3-stage TMA ring.  Per tile:
+//                     S^T  = K_j Q_i^T          (tcgen05, TMEM)
+//                     dP^T = V_j dO_i^T         (tcgen05, TMEM)
+//                     P^T  = exp2(S^T * scale*log2e - LSE2_i)          (registers)
+//                     dV  += P^T dO_i           (tcgen05, A = P^T from TMEM)
+//                     dS^T = P^T o (dP^T - D_i)                         (registers)
+//                     dK  += dS^T Q_i           (tcgen05, A = dS^T from TMEM)
+//                     dQ_i^T = K_j^T dS^T        (tcgen05, B = dS^T from shared memory)
+//                   and dQ_i^T is reduced into the fp32 accumulator with coalesced atomics.
+//                   Roles (320 threads): warps 0-3 compute P and dS (one thread per key row),
+//                   warps 4-7 drain dQ^T, warp 8 issues MMAs, warp 9 issues TMA loads.
+//                   TMEM columns: S^T [0,64), dP^T [64,128), dQ^T x2 [128,256),
+//                   dV [256,384), dK [384,512).
+//   K4 fa_bwd_post  dQ = scale * accumulator, rounded to bf16.
 #include "fa_internal.cuh"
 #include "sm100_ptx.cuh"
 
+#include <cuda_bf16.h>
+
+#include <cmath>
+
 namespace fa {
 
-cudaError_t launch_bwd_pre(const void*, const void*, float*, float*, long long, int, cudaStream_t) {
-  return cudaErrorNotSupported;
+using namespace ptx;
+
+namespace {
+constexpr float kLog2e = 1.4426950408889634074f;
 }
-cudaError_t launch_bwd_main(int, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                            const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                            const BwdArgs&, cudaStream_t) {
-  return cudaErrorNotSupported;
+
+// ------------------------------------------------------------------ K2
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
+                                                         const __nv_bfloat16* __restrict__ dO,
+                                                         const float* __restrict__ lse,
+                                                         float* __restrict__ ld,
+                                                         float* __restrict__ dq_acc, int BH, int N,
+                                                         int Tq) {
+  const int lane = threadIdx.x & 31;
+  const long long total = (long long)BH * Tq * 64;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < total; row += nw) {
+    const int bh = (int)(row / ((long long)Tq * 64));
+    const int qp = (int)(row % ((long long)Tq * 64));
+    float dsum = 0.f, l2 = INFINITY;
+    if (qp < N) {
+      const size_t base = ((size_t)bh * N + qp) * 128 + lane * 4;
+      const uint2 ov = *reinterpret_cast<const uint2*>(o + base);
+      const uint2 gv = *reinterpret_cast<const uint2*>(dO + base);
+      const float2 o01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ov.x));
+      const float2 o23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ov.y));
+      const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv.x));
+      const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv.y));
+      dsum = o01.x * g01.x + o01.y * g01.y + o23.x * g23.x + o23.y * g23.y;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
+      const float L = lse[(size_t)bh * N + qp];
+      l2 = (L == -INFINITY) ? INFINITY : L * kLog2e;  // a row with no visible key gets P = 0
+      *reinterpret_cast<float4*>(dq_acc + base) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (lane == 0) {
+      float* t = ld + ((size_t)bh * Tq + (qp >> 6)) * 128;
+      t[qp & 63] = l2;
+      t[64 + (qp & 63)] = dsum;
+    }
+  }
 }
-cudaError_t launch_bwd_post(const float*, void*, long long, float, cudaStream_t) {
-  return cudaErrorNotSupported;
+
+// ------------------------------------------------------------------ K4
+__global__ void __launch_bounds__(256) fa_bwd_post_kernel(const float4* __restrict__ acc,
+                                                          uint2* __restrict__ dq, long long n4,
+                                                          float scale) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (long long)gridDim.x * blockDim.x) {
+    const float4 a = acc[i];
+    uint2 r;
+    r.x = pack_bf16(a.x * scale, a.y * scale);
+    r.y = pack_bf16(a.z * scale, a.w * scale);
+    dq[i] = r;
+  }
+}
+
+// ------------------------------------------------------------------ K3
+struct BwdCfg {
+  static constexpr int D = 128;
+  static constexpr int BQ = 64;             // query rows per step
+  static constexpr int NSQ = 3;             // Q/dO ring stages
+  static constexpr int KT = 128 * D * 2;    // bytes of K_j (or V_j)
+  static constexpr int QT = BQ * D * 2;     // bytes of Q_i (or dO_i)
+  static constexpr int LDB = 512;           // LSE2 + D of one query tile
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = KT;
+  static constexpr int ST_OFF = 2 * KT;     // stage s: [Q_i | dO_i], 2*QT bytes
+  static constexpr int ST_BYTES = 2 * QT;
+  static constexpr int DS_OFF = ST_OFF + NSQ * ST_BYTES;  // dS^T, two buffers of 128 x 64 bf16
+  static constexpr int DS_BYTES = 128 * BQ * 2;
+  static constexpr int LD_OFF = DS_OFF + 2 * DS_BYTES;
+  static constexpr int BAR_OFF = LD_OFF + NSQ * LDB;
+  // kv_full, qd_full[3], qd_empty[3], s_full, dp_full, p_ready, ds_ready, dq_full[2],
+  // dq_free[2], ds_free[2], kv_done
+  static constexpr int NBAR = 1 + 2 * NSQ + 4 + 6 + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int SMEM = MISC_OFF + 16 + 1024;
+  static constexpr int THREADS = 320;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t T_S = 0, T_DP = 64, T_DQ = 128, T_DV = 256, T_DK = 384;
+  static constexpr uint32_t IDESC_S = idesc_bf16(128, BQ, false, false);   // S^T, dP^T
+  static constexpr uint32_t IDESC_KV = idesc_bf16(128, D, false, true);    // dV, dK
+  static constexpr uint32_t IDESC_Q = idesc_bf16(128, BQ, true, true);     // dQ^T
+};
+
+__global__ void __launch_bounds__(320, 1)
+    fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                       const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
+                       const BwdArgs a, const int Tk, const int Tq) {
+  using C = BwdCfg;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  uint8_t* gb = smem_raw + (sb - raw);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int bh = blockIdx.x / Tk;
+  const int j = blockIdx.x % Tk;               // key tile: keys [128 j, 128 j + 128)
+  const int i0 = a.causal ? 2 * j : 0;         // first query tile with a visible pair
+  const int count = max(0, Tq - i0);
+
+  const uint32_t bar = sb + C::BAR_OFF;
+  const uint32_t kv_full = bar;
+  auto qd_full = [&](int s) { return bar + 8u * (1 + s); };
+  auto qd_empty = [&](int s) { return bar + 8u * (1 + C::NSQ + s); };
+  const uint32_t s_full = bar + 8u * (1 + 2 * C::NSQ);
+  const uint32_t dp_full = s_full + 8;
+  const uint32_t p_ready = s_full + 16;
+  const uint32_t ds_ready = s_full + 24;
+  auto dq_full = [&](int b) { return s_full + 32 + 8u * b; };
+  auto dq_free = [&](int b) { return s_full + 48 + 8u * b; };
+  auto ds_free = [&](int b) { return s_full + 64 + 8u * b; };
+  const uint32_t kv_done = s_full + 80;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gb + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + C::MISC_OFF + 4);
+  const WaitCtx wc{abort_flag, a.status};
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < C::NSQ; ++s) {
+      mbar_init(qd_full(s), 1);
+      mbar_init(qd_empty(s), 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_ready, 128);
+    mbar_init(ds_ready, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(dq_full(b), 1);
+      mbar_init(dq_free(b), 128);
+      mbar_init(ds_free(b), 1);
+    }
+    mbar_init(kv_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(sb + C::MISC_OFF, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 9) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmdO);
+      const uint64_t keep = policy_evict_last();
+      mbar_arrive_expect_tx(kv_full, 2 * C::KT);
+      for (int b = 0; b < 2; ++b) {
+        tma_load_3d(sb + C::K_OFF + b * 16384, &tmK, kv_full, 64 * b, 128 * j, bh);
+        tma_load_3d(sb + C::V_OFF + b * 16384, &tmV, kv_full, 64 * b, 128 * j, bh);
+      }
+      int n = 0;
+      for (; n < count; ++n) {
+        const int s = n % C::NSQ;
+        const int i = i0 + n;
+        if (!mbar_wait(qd_empty(s), ((n / C::NSQ) & 1) ^ 1, wc)) break;
+        mbar_arrive_expect_tx(qd_full(s), 2 * C::QT + C::LDB);
+        const uint32_t st = sb + C::ST_OFF + s * C::ST_BYTES;
+        for (int b = 0; b < 2; ++b) {
+          tma_load_3d_hint(st + b * 8192, &tmQ, qd_full(s), 64 * b, C::BQ * i, bh, keep);
+          tma_load_3d_hint(st + C::QT + b * 8192, &tmdO, qd_full(s), 64 * b, C::BQ * i, bh, keep);
+        }
+        const float* src = a.ld + ((size_t)bh * Tq + i) * 128;
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                sb + C::LD_OFF + s * C::LDB),
+            "l"(reinterpret_cast<uint64_t>(src)), "r"(C::LDB), "r"(qd_full(s))
+            : "memory");
+      }
+      if (n < count) {  // aborted: let issued copies land before the CTA exits
+        mbar_wait_drain(kv_full, 0);
+        for (int back = 1; back <= C::NSQ && n - back >= 0; ++back)
+          mbar_wait_drain(qd_full((n - back) % C::NSQ), ((n - back) / C::NSQ) & 1);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(kv_full, 0, wc);
+      const uint32_t kA = sb + C::K_OFF, vA = sb + C::V_OFF;
+      for (int n = 0; n < count && ok; ++n) {
+        const int s = n % C::NSQ;
+        const int b = n & 1;
+        const uint32_t qA = sb + C::ST_OFF + s * C::ST_BYTES;
+        const uint32_t doA = qA + C::QT;
+        if (!(ok = mbar_wait(qd_full(s), (n / C::NSQ) & 1, wc))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {  // S^T = K_j Q_i^T  (K over d)
+          const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32, qo = (k >> 2) * 8192 + (k & 3) * 32;
+          mma_ss(tmem + C::T_S, sdesc_sw128(kA + ko, 16, 1024), sdesc_sw128(qA + qo, 16, 1024),
+                 C::IDESC_S, k > 0);
+        }
+        mma_commit(s_full);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {  // dP^T = V_j dO_i^T
+          const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32, qo = (k >> 2) * 8192 + (k & 3) * 32;
+          mma_ss(tmem + C::T_DP, sdesc_sw128(vA + ko, 16, 1024), sdesc_sw128(doA + qo, 16, 1024),
+                 C::IDESC_S, k > 0);
+        }
+        mma_commit(dp_full);
+        if (!(ok = mbar_wait(p_ready, n & 1, wc))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 4; ++k)  // dV += P^T dO_i  (K over the 64 queries)
+          mma_ts(tmem + C::T_DV, tmem + C::T_S + 8 * k, sdesc_sw128(doA + k * 2048, 8192, 1024),
+                 C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
+        if (!(ok = mbar_wait(ds_ready, n & 1, wc))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 4; ++k)  // dK += dS^T Q_i
+          mma_ts(tmem + C::T_DK, tmem + C::T_DP + 8 * k, sdesc_sw128(qA + k * 2048, 8192, 1024),
+                 C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
+        if (!(ok = mbar_wait(dq_free(b), ((n >> 1) & 1) ^ 1, wc))) break;
+        tc_fence_after();
+        const uint32_t dsA = sb + C::DS_OFF + b * C::DS_BYTES;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)  // dQ_i^T = K_j^T dS^T  (K over the 128 keys)
+          mma_ss(tmem + C::T_DQ + 64 * b, sdesc_sw128(kA + k * 2048, 16384, 1024),
+                 sdesc_sw128(dsA + k * 2048, 8192, 1024), C::IDESC_Q, k > 0);
+        mma_commit(dq_full(b));
+        mma_commit(ds_free(b));
+        mma_commit(qd_empty(s));
+      }
+      mma_commit(kv_done);
+      if (!ok) mbar_wait_drain(kv_done, 0);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ P and dS (one key row each)
+    const int r = warp * 32 + lane;
+    const int key = 128 * j + r;
+    const bool key_ok = key < a.N;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const float cs = a.scale_log2;
+    bool ok = true;
+    for (int n = 0; n < count && ok; ++n) {
+      const int s = n % C::NSQ;
+      const int i = i0 + n;
+      const int b = n & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(qd_full(s), (n / C::NSQ) & 1, wc) &&
+                                       mbar_wait(s_full, n & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[64];
+      tmem_ld32(tmem + lane_off + C::T_S, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tmem + lane_off + C::T_S + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_wait_ld();
+      reg_fence(sr);
+      const float* ldp = reinterpret_cast<const float*>(gb + C::LD_OFF + s * C::LDB);
+      // causal: query 64 i + c sees this key iff 64 i + c >= key
+      const int first_vis = a.causal ? (key - C::BQ * i) : -1;  // smallest visible column
+      float p[64];
+#pragma unroll
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 l2 = *reinterpret_cast<const float4*>(ldp + 4 * c4);
+        p[4 * c4 + 0] = ex2(fmaf(__uint_as_float(sr[4 * c4 + 0]), cs, -l2.x));
+        p[4 * c4 + 1] = ex2(fmaf(__uint_as_float(sr[4 * c4 + 1]), cs, -l2.y));
+        p[4 * c4 + 2] = ex2(fmaf(__uint_as_float(sr[4 * c4 + 2]), cs, -l2.z));
+        p[4 * c4 + 3] = ex2(fmaf(__uint_as_float(sr[4 * c4 + 3]), cs, -l2.w));
+      }
+      if (!key_ok) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) p[c] = 0.f;
+      } else if (first_vis > 0) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (c < first_vis) p[c] = 0.f;
+      }
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(p[2 * c], p[2 * c + 1]);
+      tmem_st32(tmem + lane_off + C::T_S, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_ready);
+
+      ok = __all_sync(0xffffffffu, mbar_wait(dp_full, n & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      tmem_ld32(tmem + lane_off + C::T_DP, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tmem + lane_off + C::T_DP + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_wait_ld();
+      reg_fence(sr);
+#pragma unroll
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 dd = *reinterpret_cast<const float4*>(ldp + 64 + 4 * c4);
+        p[4 * c4 + 0] *= __uint_as_float(sr[4 * c4 + 0]) - dd.x;
+        p[4 * c4 + 1] *= __uint_as_float(sr[4 * c4 + 1]) - dd.y;
+        p[4 * c4 + 2] *= __uint_as_float(sr[4 * c4 + 2]) - dd.z;
+        p[4 * c4 + 3] *= __uint_as_float(sr[4 * c4 + 3]) - dd.w;
+      }
+#pragma unroll
+      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(p[2 * c], p[2 * c + 1]);
+      tmem_st32(tmem + lane_off + C::T_DP, pk);
+      // dS^T row r into the shared buffer read by the dQ MMA (128-byte swizzled rows)
+      ok = __all_sync(0xffffffffu, mbar_wait(ds_free(b), ((n >> 1) & 1) ^ 1, wc));
+      if (!ok) break;
+      uint8_t* dsrow = gb + C::DS_OFF + b * C::DS_BYTES + r * 128;
+#pragma unroll
+      for (int c16 = 0; c16 < 8; ++c16)
+        *reinterpret_cast<uint4*>(dsrow + ((c16 ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
+      fence_proxy_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(ds_ready);
+    }
+    (void)i0;
+  } else {
+    // ------------------------------------------------------------ dQ^T drain (one d index each)
+    const int wq = warp & 3;
+    const int dd = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    bool ok = true;
+    for (int n = 0; n < count && ok; ++n) {
+      const int b = n & 1;
+      const int i = i0 + n;
+      ok = __all_sync(0xffffffffu, mbar_wait(dq_full(b), (n >> 1) & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t v[64];
+      tmem_ld32(tmem + lane_off + C::T_DQ + 64 * b, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_ld32(tmem + lane_off + C::T_DQ + 64 * b + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      tmem_wait_ld();
+      reg_fence(v);
+      tc_fence_before();
+      mbar_arrive(dq_free(b));
+      const int q0 = C::BQ * i;
+      const int nvalid = min(C::BQ, a.N - q0);
+      float* dst = a.dq_acc + ((size_t)bh * a.N + q0) * C::D + dd;
+#pragma unroll
+      for (int c = 0; c < 64; ++c)
+        if (c < nvalid) atomicAdd(dst + (size_t)c * C::D, __uint_as_float(v[c]));
+    }
+  }
+
+  // ---------------------------------------------------------------- epilogue: dK, dV
+  if (warp < 8) {
+    const bool is_dk = warp < 4;
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    bool ok = !*abort_flag;
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(kv_done, 0, wc));
+    if (ok) {
+      tc_fence_after();
+      const float mul = is_dk ? a.scale : 1.f;
+      const uint32_t src = tmem + lane_off + (is_dk ? C::T_DK : C::T_DV);
+      uint8_t* stage = gb + C::ST_OFF + (is_dk ? 0 : C::ST_BYTES);  // the Q/dO ring is idle now
+#pragma unroll
+      for (int bx = 0; bx < 2; ++bx) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t o[32];
+          tmem_ld32(src + 64 * bx + 32 * h, o);
+          tmem_wait_ld();
+          reg_fence(o);
+          if (count == 0) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = 0u;
+          }
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint4 w;
+            w.x = pack_bf16(__uint_as_float(o[8 * cc + 0]) * mul, __uint_as_float(o[8 * cc + 1]) * mul);
+            w.y = pack_bf16(__uint_as_float(o[8 * cc + 2]) * mul, __uint_as_float(o[8 * cc + 3]) * mul);
+            w.z = pack_bf16(__uint_as_float(o[8 * cc + 4]) * mul, __uint_as_float(o[8 * cc + 5]) * mul);
+            w.w = pack_bf16(__uint_as_float(o[8 * cc + 6]) * mul, __uint_as_float(o[8 * cc + 7]) * mul);
+            const int chunk = h * 4 + cc;
+            *reinterpret_cast<uint4*>(stage + bx * 16384 + r * 128 + ((chunk ^ (r & 7)) << 4)) = w;
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      const int row0 = 128 * j + 32 * wq;
+      if (lane == 0 && row0 < a.N) {
+        const uint32_t sbuf = sb + C::ST_OFF + (is_dk ? 0 : C::ST_BYTES);
+        for (int bx = 0; bx < 2; ++bx)
+          tma_store_3d(is_dk ? &tmdK : &tmdV, sbuf + bx * 16384 + wq * 4096, 64 * bx, row0, bh);
+        bulk_commit();
+        bulk_wait_read0();
+      }
+      __syncwarp();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ launchers
+static int grid_for(long long work, int per_block) {
+  long long g = (work + per_block - 1) / per_block;
+  const long long cap = 148LL * 16;
+  return (int)(g < 1 ? 1 : (g > cap ? cap : g));
+}
+
+cudaError_t launch_bwd_pre(const void* o, const void* dO, const float* lse, float* ld, float* dq_acc,
+                           int BH, int N, int d, cudaStream_t stream) {
+  if (d != 128) return cudaErrorNotSupported;
+  const int Tq = (N + 63) / 64;
+  const long long rows = (long long)BH * Tq * 64;
+  fa_bwd_pre_kernel<<<grid_for(rows, 8), 256, 0, stream>>>(
+      reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(dO), lse, ld,
+      dq_acc, BH, N, Tq);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_main(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
+                            const BwdArgs& a, cudaStream_t stream) {
+  if (d != 128) return cudaErrorNotSupported;
+  using C = BwdCfg;
+  static_assert(C::SMEM <= 232448, "shared memory budget");
+  cudaError_t e = cudaFuncSetAttribute(fa_bwd_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int Tk = (a.N + 127) / 128;
+  const int Tq = (a.N + 63) / 64;
+  const long long grid = (long long)a.BH * Tk;
+  fa_bwd_main_kernel<<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, tdo, tdk, tdv, a, Tk, Tq);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_post(const float* dq_acc, void* dq, long long elems, float scale, cudaStream_t stream) {
+  const long long n4 = elems / 4;
+  fa_bwd_post_kernel<<<grid_for(n4, 256), 256, 0, stream>>>(reinterpret_cast<const float4*>(dq_acc),
+                                                            reinterpret_cast<uint2*>(dq), n4, scale);
+  return cudaGetLastError();
 }
 
 }  // namespace fa

@@ -20,7 +20,8 @@ struct FwdArgs {
 struct BwdArgs {
   uint32_t* status;  // device status word
   const float* lse;  // [BH, N] fp32, natural log
-  const float* dvec; // [BH, N] fp32, D_i = rowsum(dO o O)
+  const float* ld;   // [BH, ceil(N/64), 128] fp32: per 64-row query tile, 64 x LSE*log2(e)
+                     // then 64 x D_i = rowsum(dO o O); rows past N hold +inf and 0
   float* dq_acc;     // [BH, N, d] fp32 accumulator (zeroed by the pre-kernel)
   int N;
   int BH;
@@ -38,8 +39,8 @@ bool make_tmap_bf16(CUtensorMap* m, const void* ptr, int BH, int N, int d, int b
 cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& to, const FwdArgs& a, cudaStream_t stream);
 
-cudaError_t launch_bwd_pre(const void* o, const void* dO, float* dvec, float* dq_acc,
-                           long long rows, int d, cudaStream_t stream);
+cudaError_t launch_bwd_pre(const void* o, const void* dO, const float* lse, float* ld, float* dq_acc,
+                           int BH, int N, int d, cudaStream_t stream);
 cudaError_t launch_bwd_main(int d, const CUtensorMap& tq, const CUtensorMap& tk,
                             const CUtensorMap& tv, const CUtensorMap& tdo,
                             const CUtensorMap& tdk, const CUtensorMap& tdv, const BwdArgs& a,

@@ -125,7 +125,8 @@ def attention_forward(q, k, v, scale: float, causal: bool):
     return o, lse
 
 
-def attention_backward_head(q, k, v, do, scale: float, causal: bool, row_chunk: int = 4096):
+def attention_backward_head(q, k, v, do, scale: float, causal: bool, row_chunk: int = 4096,
+                            rows: np.ndarray | None = None):
     """Gradients of O = softmax(scale * Q K^T) V for one head, by plain calculus of the
     materialised forward (the pages only say the backward recomputes the scores from the
     saved inputs and a few statistics, [xinc] section 7):
@@ -136,7 +137,9 @@ def attention_backward_head(q, k, v, do, scale: float, causal: bool, row_chunk: 
         dQ = scale * dS K
         dK = scale * dS^T Q
     Masked entries have P = 0 and so contribute nothing.  The sums over query rows in dV
-    and dK are split into chunks of ``row_chunk`` rows only to bound memory.
+    and dK are split into chunks of ``row_chunk`` rows only to bound memory.  ``rows``
+    restricts the computation to the given query rows: dQ and D are then filled for those
+    rows only and dK, dV hold those rows' contributions (used to time bounded samples).
     Returns (dQ, dK, dV, D).
     """
     q = _f64(q)
@@ -148,8 +151,9 @@ def attention_backward_head(q, k, v, do, scale: float, causal: bool, row_chunk: 
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
     dvec = np.zeros(N)
-    for c0 in range(0, N, row_chunk):
-        r = np.arange(c0, min(N, c0 + row_chunk))
+    all_rows = np.arange(N) if rows is None else np.asarray(rows)
+    for c0 in range(0, all_rows.shape[0], row_chunk):
+        r = all_rows[c0:c0 + row_chunk]
         s = scaled_scores(q, k, scale, causal, r)
         p, _, _ = softmax_rows(s)
         dv += p.T @ do[r]

@@ -31,10 +31,34 @@ def check_lse(l_gpu: np.ndarray, l_ref: np.ndarray):
     return err.max() if err.size else 0.0
 
 
-def check_grad(g_gpu: np.ndarray, g_ref: np.ndarray, what: str):
+# A reference gradient whose RMS is below this is zero up to fp64 rounding (e.g. dQ when a
+# row sees a single key: dS = P (dP - D) = 0); relative error is undefined there, and the
+# GPU result must instead be zero up to fp32 rounding.
+ZERO_RMS = 1e-9
+ZERO_MAX_ABS = 1e-4
+
+
+# Output rounding: a bf16 result is at best within half an ulp (2^-9 relative) of the exact
+# value, which exceeds the 5e-2 absolute budget once |value| > 25.6.  For shapes outside the
+# five benchmark workloads whose gradients grow that large (the long-sequence backward with
+# q, k ~ N(0, 3)), the bound is 5e-2 + 2^-8 |reference|: the absolute budget plus one bf16
+# ulp of the value.
+BF16_ULP_REL = 2.0 ** -8
+
+
+def check_grad(g_gpu: np.ndarray, g_ref: np.ndarray, what: str, rel_tol: float = GRAD_REL_L2,
+               ulp_slack: bool = False):
     assert np.isfinite(g_gpu).all(), f"{what}: non-finite values"
     err = np.abs(g_gpu - g_ref)
-    rel = np.linalg.norm(g_gpu - g_ref) / max(np.linalg.norm(g_ref), 1e-30)
-    assert err.max() <= GRAD_MAX_ABS, f"{what}: max-abs {err.max():.3e} > {GRAD_MAX_ABS}"
-    assert rel <= GRAD_REL_L2, f"{what}: rel-L2 {rel:.3e} > {GRAD_REL_L2}"
+    if ulp_slack:
+        excess = err - (GRAD_MAX_ABS + BF16_ULP_REL * np.abs(g_ref))
+        assert excess.max() <= 0, f"{what}: error exceeds 5e-2 + 2^-8|ref| by {excess.max():.3e}"
+    else:
+        assert err.max() <= GRAD_MAX_ABS, f"{what}: max-abs {err.max():.3e} > {GRAD_MAX_ABS}"
+    ref_norm = np.linalg.norm(g_ref)
+    if ref_norm <= ZERO_RMS * np.sqrt(g_ref.size):
+        assert err.max() <= ZERO_MAX_ABS, f"{what}: zero gradient, got max-abs {err.max():.3e}"
+        return err.max(), 0.0
+    rel = np.linalg.norm(g_gpu - g_ref) / ref_norm
+    assert rel <= rel_tol, f"{what}: rel-L2 {rel:.3e} > {rel_tol}"
     return err.max(), rel

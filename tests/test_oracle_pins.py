@@ -383,3 +383,14 @@ def test_planted_backward_mistakes_are_caught(which):
     g_auto = {"sign_of_row_term": tq, "unscaled_dk": tk, "transposed_dp": tv}[which].grad.numpy()
     np.testing.assert_allclose(g_ref, g_auto, atol=1e-12)
     assert np.abs(g_bad - g_auto).max() > 1e-6
+
+
+def test_backward_row_subsets_sum_to_the_whole():
+    n, d = 50, 6
+    q, k, v, do = _rand(n, d), _rand(n, d), _rand(n, d), _rand(n, d)
+    full = ref.attention_backward_head(q, k, v, do, 0.4, True)
+    a = ref.attention_backward_head(q, k, v, do, 0.4, True, rows=np.arange(0, 20))
+    b = ref.attention_backward_head(q, k, v, do, 0.4, True, rows=np.arange(20, 50))
+    np.testing.assert_allclose(a[0] + b[0], full[0], atol=1e-13)
+    np.testing.assert_allclose(a[1] + b[1], full[1], atol=1e-13)
+    np.testing.assert_allclose(a[2] + b[2], full[2], atol=1e-13)
