@@ -115,8 +115,9 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------- traffic
-def kernel_traffic(name: str, src_file: str):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
+def kernel_traffic(name: str):
+    """DRAM bytes per launch from the committed ncu summary, or None once the kernel's sources
+    have changed since the counters were taken."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
@@ -125,9 +126,11 @@ def kernel_traffic(name: str, src_file: str):
     ent = t.get(name)
     if not ent:
         return None
-    with open(os.path.join(ROOT, src_file), "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()[:16]
-    return ent.get("bytes_per_launch") if ent.get("source_sha") == sha else None
+    h = hashlib.sha256()
+    for rel in ent["files"]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return ent.get("bytes_per_launch") if ent.get("source_sha") == h.hexdigest()[:16] else None
 
 
 # ---------------------------------------------------------------------- GPU arm
@@ -277,15 +280,13 @@ def run_gpu(args):
         "roofline": {"kernel": "fa_bwd (main kernel + memory-bound pre/post, timed together)",
                      "bound": "tensor", "achieved": round(bwd_tflops, 1), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(bwd_tflops / peak, 4),
-                     "traffic": kernel_traffic("fa_bwd_main_kernel",
-                                               "io_aware_exact_22_b200/csrc/fa_bwd.cu"),
+                     "traffic": kernel_traffic("fa_bwd_main_kernel"),
                      "peak_source": f"{peak_src} bf16_tflops (burst)",
                      "algorithmic_flops_per_launch": w.bwd_flops()},
         "roofline_fwd": {"kernel": "fa_fwd_kernel<128>", "bound": "tensor",
                          "achieved": round(fwd_tflops, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(fwd_tflops / peak, 4),
-                         "traffic": kernel_traffic("fa_fwd_kernel",
-                                                   "io_aware_exact_22_b200/csrc/fa_fwd.cu"),
+                         "traffic": kernel_traffic("fa_fwd_kernel"),
                          "algorithmic_flops_per_launch": w.fwd_flops()},
         "clocks": clk,
         "gpu_launches": 4 * args.steps,
