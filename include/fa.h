@@ -94,6 +94,34 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o,
                    int B, int H, int N, int d, float scale, int causal, void* stream);
 
 /*
+ * Size of the scratch array that fa_bwd_noalloc uses in place of a workspace: 64 MiB, held in
+ * device memory on every GPU that has loaded the library, for as long as it stays loaded.
+ */
+#define FA_BWD_NOALLOC_MAX_SCRATCH_BYTES ((size_t)64 << 20)
+
+/*
+ * fa_bwd for callers that cannot allocate device memory.  (The pages have no counterpart: this
+ * is an interface convenience, not part of the method.)
+ *
+ * Who needs it: code that runs inside a host framework owning all device memory and offering
+ * its extensions no allocator, and hot paths whose rules forbid cudaMalloc (which can
+ * synchronise the device).  Arguments and results are those of fa_bwd minus the workspace;
+ * inputs and outputs are still the caller's buffers.  No memory is allocated by this call.
+ *
+ * Scratch: a fixed FA_BWD_NOALLOC_MAX_SCRATCH_BYTES array inside the library replaces the
+ * workspace.  Problems whose fa_bwd_workspace_bytes(B,H,N,d) exceeds that size are refused with
+ * FA_ERR_INVALID_ARG before any GPU work (at d = 128 this allows B*H*N up to about 129,000
+ * query rows).  The first call on each device looks up the array's device address (a CUDA
+ * runtime query) and caches it; make that first call before any stream capture on that device.
+ * Every call shares the one array: calls that overlap on the GPU (other streams, other host
+ * threads) race on it and must be serialised by the caller.  Each call rewrites the scratch it
+ * reads, so leftovers from an earlier call do not affect results.
+ */
+fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                           const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                           int B, int H, int N, int d, float scale, int causal, void* stream);
+
+/*
  * Synchronises `stream`, reads and clears the device status word of the current device.
  * Returns FA_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call,
  * FA_ERR_CUDA if the synchronisation itself failed, FA_OK otherwise.

@@ -22,7 +22,9 @@ LIB_PATH = os.environ.get("FA_LIB_PATH", os.path.join(_HERE, "libfa.so"))
 STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_CUDA",
           4: "FA_ERR_TIMEOUT"}
 EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_device_status",
-           "fa_status_string", "fa_version")
+           "fa_status_string", "fa_version", "fa_bwd_noalloc")
+# Size of the library's built-in scratch used by fa_bwd_noalloc (include/fa.h).
+NOALLOC_MAX_SCRATCH_BYTES = 64 << 20
 
 _lib = None
 
@@ -54,6 +56,8 @@ def lib() -> ctypes.CDLL:
         L.fa_status_string.restype = ctypes.c_char_p
         L.fa_version.argtypes = []
         L.fa_version.restype = i
+        L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+        L.fa_bwd_noalloc.restype = i
         _lib = L
     return _lib
 
@@ -85,6 +89,15 @@ def fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes, B, H, N,
     return lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq),
                         _ptr(dk), _ptr(dv), _ptr(workspace), int(workspace_bytes), B, H, N, d,
                         float(scale), int(causal), _stream(stream))
+
+
+def fa_bwd_noalloc(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal,
+                   stream=None) -> int:
+    """fa_bwd without a workspace: the library's fixed scratch array is used instead, for
+    callers that cannot allocate device memory.  Overlapping calls race on that array."""
+    return lib().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse),
+                                _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
+                                int(causal), _stream(stream))
 
 
 def fa_bwd_workspace_bytes(B, H, N, d) -> int:

@@ -1,0 +1,55 @@
+"""fa_bwd_noalloc: the backward for callers that cannot allocate device memory.
+
+Some callers cannot hand the library a workspace: code living inside a framework that owns
+all device memory and gives its extensions no allocator, or a hot path that must not call
+cudaMalloc.  fa_bwd_noalloc serves them with a scratch array built into the library.  This
+file checks, through the C ABI, that it returns what fa_bwd (with a caller workspace)
+returns, on two calls in a row (the second call runs on scratch the first one left behind),
+and that problems too large for the built-in scratch are refused.  It sits in its own file,
+collected last, so that a failure here never hides the other tests.
+"""
+import numpy as np
+import pytest
+import torch
+
+from io_aware_exact_22_b200 import fa
+from io_aware_exact_22_b200.inputs import custom, make_inputs
+from tests._helpers import check_grad, f64
+
+pytestmark = pytest.mark.gpu
+
+OK, INVALID = 0, 1
+
+
+def _inputs(w):
+    q, k, v, do = (t.cuda() for t in make_inputs(w))
+    o, lse = fa.forward(q, k, v, w.causal, w.scale)
+    return q, k, v, o, do, lse
+
+
+@pytest.mark.parametrize("B,H,N,causal", [(1, 3, 1000, True), (2, 2, 777, False)])
+def test_noalloc_matches_workspace_backward_twice(cuda_ok, B, H, N, causal):
+    w = custom(B, H, N, 128, causal, seed=31, backward=True)
+    q, k, v, o, do, lse = _inputs(w)
+    ref = fa.backward(q, k, v, o, do, lse, causal, w.scale)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        dq, dk, dv = (torch.full_like(q, float("nan")) for _ in range(3))
+        rc = fa.fa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, B, H, N, 128, w.scale, causal)
+        assert rc == OK, fa.fa_status_string(rc)
+        torch.cuda.synchronize()
+        assert fa.fa_get_device_status() == OK
+        for got, want, name in zip((dq, dk, dv), ref, ("dQ", "dK", "dV")):
+            check_grad(f64(got), f64(want), f"noalloc {name}")
+        # dK and dV are summed in a fixed order: identical to the workspace path
+        assert torch.equal(dk, ref[1]) and torch.equal(dv, ref[2])
+
+
+def test_noalloc_refuses_problems_beyond_its_scratch(cuda_ok):
+    N = 16384
+    H = 16  # 16 * 16384 query rows need about 130 MiB of scratch at d = 128
+    assert fa.fa_bwd_workspace_bytes(1, H, N, 128) > fa.NOALLOC_MAX_SCRATCH_BYTES
+    x = torch.empty(16, device="cuda", dtype=torch.bfloat16)
+    rc = fa.fa_bwd_noalloc(x, x, x, x, x, x, x, x, x, 1, H, N, 128, 0.088, 1)
+    assert rc == INVALID
+    assert fa.fa_bwd_workspace_bytes(1, 4, 4096, 128) <= fa.NOALLOC_MAX_SCRATCH_BYTES
