@@ -100,6 +100,19 @@ bool make_tmap_bf16(CUtensorMap* m, const void* ptr, int BH, int N, int d, int b
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_f32(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_inner, int box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)N * d * 4};
+  cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace fa
 
 using namespace fa;
@@ -171,10 +184,11 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
   float* ld = reinterpret_cast<float*>(workspace);
   float* dq_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + ld_bytes(BH, N));
   cudaStream_t s = (cudaStream_t)stream;
-  CUtensorMap tq, tk, tv, tdo, tdk, tdv;
+  CUtensorMap tq, tk, tv, tdo, tdk, tdv, tdq;
   if (!make_tmap_bf16(&tq, q, BH, N, d, 64) || !make_tmap_bf16(&tk, k, BH, N, d, 128) ||
       !make_tmap_bf16(&tv, v, BH, N, d, 128) || !make_tmap_bf16(&tdo, dO, BH, N, d, 64) ||
-      !make_tmap_bf16(&tdk, dk, BH, N, d, 32) || !make_tmap_bf16(&tdv, dv, BH, N, d, 32))
+      !make_tmap_bf16(&tdk, dk, BH, N, d, 32) || !make_tmap_bf16(&tdv, dv, BH, N, d, 32) ||
+      !make_tmap_f32(&tdq, dq_acc, BH, N, d, 32, 64))
     return FA_ERR_CUDA;
   BwdArgs a;
   if (!(a.status = device_status_word())) return FA_ERR_CUDA;
@@ -187,7 +201,7 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
   a.scale = scale;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   if (launch_bwd_pre(o, dO, lse, ld, dq_acc, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
-  cudaError_t e = launch_bwd_main(d, tq, tk, tv, tdo, tdk, tdv, a, s);
+  cudaError_t e = launch_bwd_main(d, tq, tk, tv, tdo, tdk, tdv, tdq, a, s);
   if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
   if (e != cudaSuccess) return FA_ERR_CUDA;
   if (launch_bwd_post(dq_acc, dq, rows * d, scale, s) != cudaSuccess) return FA_ERR_CUDA;

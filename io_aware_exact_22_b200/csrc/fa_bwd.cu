@@ -19,9 +19,7 @@
 //                     dS^T = P^T o (dP^T - D_i)                         (registers)
 //                     dK  += dS^T Q_i           (tcgen05, A = dS^T from TMEM)
 //                     dQ_i^T = K_j^T dS^T        (tcgen05, B = dS^T from shared memory)
-//                   and dQ_i^T is reduced into the fp32 accumulator with coalesced atomics.
-//                   Roles (320 threads): warps 0-3 compute P and dS (one thread per key row),
-//                   warps 4-7 drain dQ^T, warp 8 issues MMAs, warp 9 issues TMA loads.
+//                   and dQ_i^T is added into the fp32 accumulator by TMA reduce-add.
 //                   TMEM columns: S^T [0,64), dP^T [64,128), dQ^T x2 [128,256),
 //                   dV [256,384), dK [384,512).
 //   K4 fa_bwd_post  dQ = scale * accumulator, rounded to bf16.
@@ -105,26 +103,39 @@ struct BwdCfg {
   static constexpr int ST_BYTES = 2 * QT;
   static constexpr int DS_OFF = ST_OFF + NSQ * ST_BYTES;  // dS^T, two buffers of 128 x 64 bf16
   static constexpr int DS_BYTES = 128 * BQ * 2;
-  static constexpr int LD_OFF = DS_OFF + 2 * DS_BYTES;
+  static constexpr int DQS_OFF = DS_OFF + 2 * DS_BYTES;   // dQ staging: 4 warps x [64 q][32 d] fp32
+  static constexpr int DQS_WARP = BQ * 32 * 4;
+  static constexpr int LD_OFF = DQS_OFF + 4 * DQS_WARP;
   static constexpr int BAR_OFF = LD_OFF + NSQ * LDB;
   // kv_full, qd_full[3], qd_empty[3], s_full, dp_full, p_ready, ds_ready, dq_full[2],
   // dq_free[2], ds_free[2], kv_done
   static constexpr int NBAR = 1 + 2 * NSQ + 4 + 6 + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM = MISC_OFF + 16 + 1024;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 448;
   static constexpr uint32_t TMEM_COLS = 512;
+  // TMEM columns (a 512-column allocation always starts at column 0, lane 0)
   static constexpr uint32_t T_S = 0, T_DP = 64, T_DQ = 128, T_DV = 256, T_DK = 384;
   static constexpr uint32_t IDESC_S = idesc_bf16(128, BQ, false, false);   // S^T, dP^T
   static constexpr uint32_t IDESC_KV = idesc_bf16(128, D, false, true);    // dV, dK
   static constexpr uint32_t IDESC_Q = idesc_bf16(128, BQ, true, true);     // dQ^T
 };
 
-__global__ void __launch_bounds__(320, 1)
+// Roles (448 threads):
+//   warps 0-3   compute warpgroup 0: P^T and dS^T for query columns [0, 32)  (one key row each)
+//   warps 4-7   compute warpgroup 1: the same for query columns [32, 64)
+//   warps 8-11  dQ^T drain: TMEM -> shared staging -> TMA reduce-add into the fp32 accumulator
+//   warp 12     MMA issuer (whole warp, one elected lane issues)
+//   warp 13     TMA producer (whole warp, one elected lane issues)
+// Each compute warpgroup writes its packed P^T (and dS^T) inside its own S^T (dP^T) columns,
+// so neither overwrites scores the other has not read yet: P^T of query columns [32g, 32g+32)
+// sits at TMEM columns [32g, 32g+16), dS^T at [64+32g, 64+32g+16).
+__global__ void __launch_bounds__(448, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                        const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
-                       const BwdArgs a, const int Tk, const int Tq) {
+                       const __grid_constant__ CUtensorMap tmdQ, const BwdArgs a, const int Tk,
+                       const int Tq) {
   using C = BwdCfg;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -162,8 +173,8 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_ready, 128);
-    mbar_init(ds_ready, 128);
+    mbar_init(p_ready, 256);
+    mbar_init(ds_ready, 256);
     for (int b = 0; b < 2; ++b) {
       mbar_init(dq_full(b), 1);
       mbar_init(dq_free(b), 128);
@@ -173,43 +184,46 @@ __global__ void __launch_bounds__(320, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == 12) {
     tmem_alloc(sb + C::MISC_OFF, C::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  // All TMEM addresses below are compile-time column offsets from address 0.
+  if (*tmem_slot != 0u) {
+    if (threadIdx.x == 0) atomicOr(a.status, FA_DEV_TMEM_BASE);
+    *abort_flag = 1;
+  }
+  const uint32_t tmem = 0u;
 
-  if (warp == 9) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmdO);
+  if (warp == 13) {
+    // ------------------------------------------------------------ TMA producer (whole warp)
+    if (!*abort_flag) {
+      if (elect_one()) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmdO);
+      }
       const uint64_t keep = policy_evict_last();
-      mbar_arrive_expect_tx(kv_full, 2 * C::KT);
+      const uint64_t once = policy_evict_first();
+      mbar_arrive_expect_tx_e(kv_full, 2 * C::KT);
       for (int b = 0; b < 2; ++b) {
-        tma_load_3d(sb + C::K_OFF + b * 16384, &tmK, kv_full, 64 * b, 128 * j, bh);
-        tma_load_3d(sb + C::V_OFF + b * 16384, &tmV, kv_full, 64 * b, 128 * j, bh);
+        tma_load_3d_e(sb + C::K_OFF + b * 16384, &tmK, kv_full, 64 * b, 128 * j, bh, once);
+        tma_load_3d_e(sb + C::V_OFF + b * 16384, &tmV, kv_full, 64 * b, 128 * j, bh, once);
       }
       int n = 0;
       for (; n < count; ++n) {
         const int s = n % C::NSQ;
         const int i = i0 + n;
-        if (!mbar_wait(qd_empty(s), ((n / C::NSQ) & 1) ^ 1, wc)) break;
-        mbar_arrive_expect_tx(qd_full(s), 2 * C::QT + C::LDB);
+        if (!__all_sync(0xffffffffu, mbar_wait(qd_empty(s), ((n / C::NSQ) & 1) ^ 1, wc))) break;
+        mbar_arrive_expect_tx_e(qd_full(s), 2 * C::QT + C::LDB);
         const uint32_t st = sb + C::ST_OFF + s * C::ST_BYTES;
         for (int b = 0; b < 2; ++b) {
-          tma_load_3d_hint(st + b * 8192, &tmQ, qd_full(s), 64 * b, C::BQ * i, bh, keep);
-          tma_load_3d_hint(st + C::QT + b * 8192, &tmdO, qd_full(s), 64 * b, C::BQ * i, bh, keep);
+          tma_load_3d_e(st + b * 8192, &tmQ, qd_full(s), 64 * b, C::BQ * i, bh, keep);
+          tma_load_3d_e(st + C::QT + b * 8192, &tmdO, qd_full(s), 64 * b, C::BQ * i, bh, keep);
         }
-        const float* src = a.ld + ((size_t)bh * Tq + i) * 128;
-        asm volatile(
-            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                sb + C::LD_OFF + s * C::LDB),
-            "l"(reinterpret_cast<uint64_t>(src)), "r"(C::LDB), "r"(qd_full(s))
-            : "memory");
+        bulk_load_e(sb + C::LD_OFF + s * C::LDB, a.ld + ((size_t)bh * Tq + i) * 128, C::LDB, qd_full(s));
       }
       if (n < count) {  // aborted: let issued copies land before the CTA exits
         mbar_wait_drain(kv_full, 0);
@@ -218,67 +232,98 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 8) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      bool ok = mbar_wait(kv_full, 0, wc);
+  } else if (warp == 12) {
+    // ------------------------------------------------------------ MMA issuer (whole warp)
+    // Issue order, software-pipelined by one query tile so that the tensor core never waits
+    // for the compute warps in steady state:
+    //   S_0, dP_0 | dV_n, S_{n+1}, dK_n, dQ_n, dP_{n+1} | ...
+    // S_{n+1} overwrites the S^T/P^T columns only after dV_n (which reads P^T_n) and dP_{n+1}
+    // overwrites the dP^T/dS^T columns only after dK_n (which reads dS^T_n): tcgen05 MMAs
+    // issued by one thread execute in order.
+    if (!*abort_flag) {
+      bool ok = __all_sync(0xffffffffu, mbar_wait(kv_full, 0, wc));
       const uint32_t kA = sb + C::K_OFF, vA = sb + C::V_OFF;
+      auto q_addr = [&](int n) { return sb + C::ST_OFF + (n % C::NSQ) * C::ST_BYTES; };
+      auto issue_s = [&](int n) {  // S^T = K_j Q_i^T  (K over d)
+        const uint32_t qA = q_addr(n);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32, qo = (k >> 2) * 8192 + (k & 3) * 32;
+          mma_ss_e(tmem + C::T_S, sdesc_sw128(kA + ko, 16, 1024), sdesc_sw128(qA + qo, 16, 1024),
+                   C::IDESC_S, k > 0);
+        }
+        mma_commit_e(s_full);
+      };
+      auto issue_dp = [&](int n) {  // dP^T = V_j dO_i^T
+        const uint32_t doA = q_addr(n) + C::QT;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32, qo = (k >> 2) * 8192 + (k & 3) * 32;
+          mma_ss_e(tmem + C::T_DP, sdesc_sw128(vA + ko, 16, 1024), sdesc_sw128(doA + qo, 16, 1024),
+                   C::IDESC_S, k > 0);
+        }
+        mma_commit_e(dp_full);
+      };
+      if (ok && count > 0) {
+        if ((ok = __all_sync(0xffffffffu, mbar_wait(qd_full(0), 0, wc)))) {
+          tc_fence_after();
+          issue_s(0);
+          issue_dp(0);
+        }
+      }
       for (int n = 0; n < count && ok; ++n) {
         const int s = n % C::NSQ;
         const int b = n & 1;
-        const uint32_t qA = sb + C::ST_OFF + s * C::ST_BYTES;
+        const uint32_t qA = q_addr(n);
         const uint32_t doA = qA + C::QT;
-        if (!(ok = mbar_wait(qd_full(s), (n / C::NSQ) & 1, wc))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {  // S^T = K_j Q_i^T  (K over d)
-          const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32, qo = (k >> 2) * 8192 + (k & 3) * 32;
-          mma_ss(tmem + C::T_S, sdesc_sw128(kA + ko, 16, 1024), sdesc_sw128(qA + qo, 16, 1024),
-                 C::IDESC_S, k > 0);
-        }
-        mma_commit(s_full);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {  // dP^T = V_j dO_i^T
-          const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32, qo = (k >> 2) * 8192 + (k & 3) * 32;
-          mma_ss(tmem + C::T_DP, sdesc_sw128(vA + ko, 16, 1024), sdesc_sw128(doA + qo, 16, 1024),
-                 C::IDESC_S, k > 0);
-        }
-        mma_commit(dp_full);
-        if (!(ok = mbar_wait(p_ready, n & 1, wc))) break;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(p_ready, n & 1, wc)))) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 4; ++k)  // dV += P^T dO_i  (K over the 64 queries)
-          mma_ts(tmem + C::T_DV, tmem + C::T_S + 8 * k, sdesc_sw128(doA + k * 2048, 8192, 1024),
-                 C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
-        if (!(ok = mbar_wait(ds_ready, n & 1, wc))) break;
+          mma_ts_e(tmem + C::T_DV, tmem + C::T_S + 32 * (k >> 1) + 8 * (k & 1),
+                   sdesc_sw128(doA + k * 2048, 8192, 1024), C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
+        const bool more = n + 1 < count;
+        if (more) {
+          if (!(ok = __all_sync(0xffffffffu,
+                                mbar_wait(qd_full((n + 1) % C::NSQ), ((n + 1) / C::NSQ) & 1, wc))))
+            break;
+          tc_fence_after();
+          issue_s(n + 1);
+        }
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(ds_ready, n & 1, wc)))) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 4; ++k)  // dK += dS^T Q_i
-          mma_ts(tmem + C::T_DK, tmem + C::T_DP + 8 * k, sdesc_sw128(qA + k * 2048, 8192, 1024),
-                 C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
-        if (!(ok = mbar_wait(dq_free(b), ((n >> 1) & 1) ^ 1, wc))) break;
+          mma_ts_e(tmem + C::T_DK, tmem + C::T_DP + 32 * (k >> 1) + 8 * (k & 1),
+                   sdesc_sw128(qA + k * 2048, 8192, 1024), C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(dq_free(b), ((n >> 1) & 1) ^ 1, wc)))) break;
         tc_fence_after();
         const uint32_t dsA = sb + C::DS_OFF + b * C::DS_BYTES;
 #pragma unroll
         for (int k = 0; k < 8; ++k)  // dQ_i^T = K_j^T dS^T  (K over the 128 keys)
-          mma_ss(tmem + C::T_DQ + 64 * b, sdesc_sw128(kA + k * 2048, 16384, 1024),
-                 sdesc_sw128(dsA + k * 2048, 8192, 1024), C::IDESC_Q, k > 0);
-        mma_commit(dq_full(b));
-        mma_commit(ds_free(b));
-        mma_commit(qd_empty(s));
+          mma_ss_e(tmem + C::T_DQ + 64 * b, sdesc_sw128(kA + k * 2048, 16384, 1024),
+                   sdesc_sw128(dsA + k * 2048, 8192, 1024), C::IDESC_Q, k > 0);
+        mma_commit_e(dq_full(b));
+        mma_commit_e(ds_free(b));
+        mma_commit_e(qd_empty(s));
+        if (more) issue_dp(n + 1);
       }
-      mma_commit(kv_done);
+      mma_commit_e(kv_done);
       if (!ok) mbar_wait_drain(kv_done, 0);
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ P and dS (one key row each)
-    const int r = warp * 32 + lane;
+    const int g = warp >> 2;          // query columns [32 g, 32 g + 32)
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
     const int key = 128 * j + r;
     const bool key_ok = key < a.N;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::T_S + 32 * g;
+    const uint32_t tDP = tmem + lane_off + C::T_DP + 32 * g;
     const float cs = a.scale_log2;
-    bool ok = true;
+    bool ok = !*abort_flag;
     for (int n = 0; n < count && ok; ++n) {
       const int s = n % C::NSQ;
       const int i = i0 + n;
@@ -287,17 +332,16 @@ __global__ void __launch_bounds__(320, 1)
                                        mbar_wait(s_full, n & 1, wc));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld32(tmem + lane_off + C::T_S, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tmem + lane_off + C::T_S + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      uint32_t sr[32];
+      tmem_ld32(tS, sr);
+      const float* ldp = reinterpret_cast<const float*>(gb + C::LD_OFF + s * C::LDB) + 32 * g;
       tmem_wait_ld();
       reg_fence(sr);
-      const float* ldp = reinterpret_cast<const float*>(gb + C::LD_OFF + s * C::LDB);
-      // causal: query 64 i + c sees this key iff 64 i + c >= key
-      const int first_vis = a.causal ? (key - C::BQ * i) : -1;  // smallest visible column
-      float p[64];
+      // causal: query 64 i + 32 g + c sees this key iff it is >= key
+      const int first_vis = a.causal ? (key - C::BQ * i - 32 * g) : -1;  // first visible column
+      float p[32];
 #pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
+      for (int c4 = 0; c4 < 8; ++c4) {
         const float4 l2 = *reinterpret_cast<const float4*>(ldp + 4 * c4);
         p[4 * c4 + 0] = ex2(fmaf(__uint_as_float(sr[4 * c4 + 0]), cs, -l2.x));
         p[4 * c4 + 1] = ex2(fmaf(__uint_as_float(sr[4 * c4 + 1]), cs, -l2.y));
@@ -306,16 +350,16 @@ __global__ void __launch_bounds__(320, 1)
       }
       if (!key_ok) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) p[c] = 0.f;
+        for (int c = 0; c < 32; ++c) p[c] = 0.f;
       } else if (first_vis > 0) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
+        for (int c = 0; c < 32; ++c)
           if (c < first_vis) p[c] = 0.f;
       }
-      uint32_t pk[32];
+      uint32_t pk[16];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(p[2 * c], p[2 * c + 1]);
-      tmem_st32(tmem + lane_off + C::T_S, pk);
+      for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(p[2 * c], p[2 * c + 1]);
+      tmem_st16(tS, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_ready);
@@ -323,12 +367,11 @@ __global__ void __launch_bounds__(320, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(dp_full, n & 1, wc));
       if (!ok) break;
       tc_fence_after();
-      tmem_ld32(tmem + lane_off + C::T_DP, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tmem + lane_off + C::T_DP + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tDP, sr);
       tmem_wait_ld();
       reg_fence(sr);
 #pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
+      for (int c4 = 0; c4 < 8; ++c4) {
         const float4 dd = *reinterpret_cast<const float4*>(ldp + 64 + 4 * c4);
         p[4 * c4 + 0] *= __uint_as_float(sr[4 * c4 + 0]) - dd.x;
         p[4 * c4 + 1] *= __uint_as_float(sr[4 * c4 + 1]) - dd.y;
@@ -336,28 +379,30 @@ __global__ void __launch_bounds__(320, 1)
         p[4 * c4 + 3] *= __uint_as_float(sr[4 * c4 + 3]) - dd.w;
       }
 #pragma unroll
-      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(p[2 * c], p[2 * c + 1]);
-      tmem_st32(tmem + lane_off + C::T_DP, pk);
-      // dS^T row r into the shared buffer read by the dQ MMA (128-byte swizzled rows)
+      for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(p[2 * c], p[2 * c + 1]);
+      tmem_st16(tDP, pk);
+      // dS^T row r, query columns [32 g, 32 g + 32), into the shared buffer read by the dQ MMA
       ok = __all_sync(0xffffffffu, mbar_wait(ds_free(b), ((n >> 1) & 1) ^ 1, wc));
       if (!ok) break;
       uint8_t* dsrow = gb + C::DS_OFF + b * C::DS_BYTES + r * 128;
 #pragma unroll
-      for (int c16 = 0; c16 < 8; ++c16)
-        *reinterpret_cast<uint4*>(dsrow + ((c16 ^ (r & 7)) << 4)) =
+      for (int c16 = 0; c16 < 4; ++c16) {
+        const int chunk = 4 * g + c16;
+        *reinterpret_cast<uint4*>(dsrow + ((chunk ^ (r & 7)) << 4)) =
             make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
+      }
       fence_proxy_async_smem();
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(ds_ready);
     }
-    (void)i0;
   } else {
     // ------------------------------------------------------------ dQ^T drain (one d index each)
     const int wq = warp & 3;
-    const int dd = wq * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    bool ok = true;
+    float* stage = reinterpret_cast<float*>(gb + C::DQS_OFF + wq * C::DQS_WARP);
+    const uint32_t stage_s = sb + C::DQS_OFF + wq * C::DQS_WARP;
+    bool ok = !*abort_flag;
     for (int n = 0; n < count && ok; ++n) {
       const int b = n & 1;
       const int i = i0 + n;
@@ -371,13 +416,20 @@ __global__ void __launch_bounds__(320, 1)
       reg_fence(v);
       tc_fence_before();
       mbar_arrive(dq_free(b));
-      const int q0 = C::BQ * i;
-      const int nvalid = min(C::BQ, a.N - q0);
-      float* dst = a.dq_acc + ((size_t)bh * a.N + q0) * C::D + dd;
+      // [64 queries][32 d] fp32 slice of this warp; lane = d, so each row is one 128-byte store
+      if (lane == 0) bulk_wait_read0();  // the previous reduce has finished reading the staging
+      __syncwarp();
 #pragma unroll
-      for (int c = 0; c < 64; ++c)
-        if (c < nvalid) atomicAdd(dst + (size_t)c * C::D, __uint_as_float(v[c]));
+      for (int c = 0; c < 64; ++c) stage[c * 32 + lane] = __uint_as_float(v[c]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_reduce_add_3d(&tmdQ, stage_s, 32 * wq, C::BQ * i, bh);
+        bulk_commit();
+      }
     }
+    if (lane == 0) bulk_wait0();
+    __syncwarp();
   }
 
   // ---------------------------------------------------------------- epilogue: dK, dV
@@ -433,9 +485,9 @@ __global__ void __launch_bounds__(320, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 12) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    tmem_dealloc(*tmem_slot, C::TMEM_COLS);
   }
 }
 
@@ -459,7 +511,7 @@ cudaError_t launch_bwd_pre(const void* o, const void* dO, const float* lse, floa
 
 cudaError_t launch_bwd_main(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
-                            const BwdArgs& a, cudaStream_t stream) {
+                            const CUtensorMap& tdq, const BwdArgs& a, cudaStream_t stream) {
   if (d != 128) return cudaErrorNotSupported;
   using C = BwdCfg;
   static_assert(C::SMEM <= 232448, "shared memory budget");
@@ -468,7 +520,8 @@ cudaError_t launch_bwd_main(int d, const CUtensorMap& tq, const CUtensorMap& tk,
   const int Tk = (a.N + 127) / 128;
   const int Tq = (a.N + 63) / 64;
   const long long grid = (long long)a.BH * Tk;
-  fa_bwd_main_kernel<<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, tdo, tdk, tdv, a, Tk, Tq);
+  fa_bwd_main_kernel<<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, tdo, tdk, tdv, tdq, a, Tk,
+                                                                        Tq);
   return cudaGetLastError();
 }
 

@@ -40,6 +40,8 @@ struct FwdCfg {
   static constexpr int SMEM = MISC_OFF + 16 + 1024;  // + slack to align the base to 1024
   static constexpr int THREADS = 320;
   static constexpr uint32_t TMEM_COLS = 512;
+  // TMEM columns (a 512-column allocation always starts at column 0, lane 0)
+  static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_O0 = 256, T_O1 = 256 + D;
   static constexpr uint32_t IDESC_QK = idesc_bf16(128, 128, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);
 };
@@ -99,32 +101,40 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  // All TMEM addresses below are compile-time column offsets from address 0.
+  if (*tmem_slot != 0u) {
+    if (threadIdx.x == 0) atomicOr(a.status, FA_DEV_TMEM_BASE);
+    *abort_flag = 1;
+  }
+  const uint32_t tmem = 0u;
 
   if (warp == 9) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && !*abort_flag) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
+    // ------------------------------------------------------------ TMA producer (whole warp)
+    if (!*abort_flag) {
+      if (elect_one()) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+      }
       const uint64_t keep = policy_evict_last();
       const int nq = has1 ? 2 : 1;
-      mbar_arrive_expect_tx(q_full, nq * C::TILE);
+      mbar_arrive_expect_tx_e(q_full, nq * C::TILE);
       for (int t = 0; t < nq; ++t)
         for (int b = 0; b < C::NBOX; ++b)
-          tma_load_3d(sb + C::Q_OFF + t * C::TILE + b * 16384, &tmQ, q_full, 64 * b, q0 + 128 * t, bh);
+          tma_load_3d_e(sb + C::Q_OFF + t * C::TILE + b * 16384, &tmQ, q_full, 64 * b, q0 + 128 * t, bh,
+                        keep);
       int it = 0;
       bool ok = true;
       for (int j = 0; j < nmax && ok; ++j) {
         for (int kv = 0; kv < 2; ++kv, ++it) {
           const int s = it % C::NS;
           const uint32_t ph = (it / C::NS) & 1;
-          if (!mbar_wait(kv_empty(s), ph ^ 1, wc)) { ok = false; break; }
-          mbar_arrive_expect_tx(kv_full(s), C::TILE);
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(kv_empty(s), ph ^ 1, wc)))) break;
+          mbar_arrive_expect_tx_e(kv_full(s), C::TILE);
           const CUtensorMap* m = kv ? &tmV : &tmK;
           for (int b = 0; b < C::NBOX; ++b)
-            tma_load_3d_hint(sb + C::KV_OFF + s * C::TILE + b * 16384, m, kv_full(s), 64 * b, 128 * j,
-                             bh, keep);
+            tma_load_3d_e(sb + C::KV_OFF + s * C::TILE + b * 16384, m, kv_full(s), 64 * b, 128 * j, bh,
+                          keep);
         }
       }
       if (!ok) {  // let copies already issued land before the CTA exits
@@ -137,63 +147,64 @@ __global__ void __launch_bounds__(320, 1)
     }
     __syncwarp();
   } else if (warp == 8) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && !*abort_flag) {
-      const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
-      const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
+    // ------------------------------------------------------------ MMA issuer (whole warp)
+    if (!*abort_flag) {
       const int nt[2] = {n0, n1};
       auto issue_qk = [&](uint32_t dst, uint32_t qaddr, uint32_t kaddr) {
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-          mma_ss(dst, sdesc_sw128(qaddr + off, 16, 1024), sdesc_sw128(kaddr + off, 16, 1024),
-                 C::IDESC_QK, k > 0);
+          mma_ss_e(dst, sdesc_sw128(qaddr + off, 16, 1024), sdesc_sw128(kaddr + off, 16, 1024),
+                   C::IDESC_QK, k > 0);
         }
       };
       auto issue_pv = [&](uint32_t dst, uint32_t ptm, uint32_t vaddr, bool acc) {
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          mma_ts(dst, ptm + 8 * k, sdesc_sw128(vaddr + k * 2048, 16384, 1024), C::IDESC_PV,
-                 (acc || k > 0) ? 1u : 0u);
+          mma_ts_e(dst, ptm + 8 * k, sdesc_sw128(vaddr + k * 2048, 16384, 1024), C::IDESC_PV,
+                   (acc || k > 0) ? 1u : 0u);
       };
       auto stage_addr = [&](int it) { return sb + C::KV_OFF + (it % C::NS) * C::TILE; };
       auto stage_par = [&](int it) { return (uint32_t)((it / C::NS) & 1); };
-      bool ok = mbar_wait(q_full, 0, wc);
-      if (ok) ok = mbar_wait(kv_full(0), 0, wc);
+      bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, wc));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(kv_full(0), 0, wc));
       if (ok) {
         tc_fence_after();
-        for (int t = 0; t < 2; ++t)
-          if (nt[t] > 0) {
-            issue_qk(tS[t], sb + C::Q_OFF + t * C::TILE, stage_addr(0));
-            mma_commit(s_full(t));
-          }
-        mma_commit(kv_empty(0));
+        issue_qk(C::T_S0, sb + C::Q_OFF, stage_addr(0));
+        mma_commit_e(s_full(0));
+        if (n1 > 0) {
+          issue_qk(C::T_S1, sb + C::Q_OFF + C::TILE, stage_addr(0));
+          mma_commit_e(s_full(1));
+        }
+        mma_commit_e(kv_empty(0));
       }
       for (int j = 0; j < nmax && ok; ++j) {
         const int itK = 2 * (j + 1), itV = 2 * j + 1;  // ring positions of K_{j+1} and V_j
-        if (!(ok = mbar_wait(kv_full(itV % C::NS), stage_par(itV), wc))) break;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(kv_full(itV % C::NS), stage_par(itV), wc)))) break;
         tc_fence_after();
         bool k_ready = false;
-        for (int t = 0; t < 2 && ok; ++t) {
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
           if (j >= nt[t]) continue;
-          if (!(ok = mbar_wait(p_full(t), j & 1, wc))) break;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(p_full(t), j & 1, wc)))) break;
           tc_fence_after();
-          issue_pv(tO[t], tS[t], stage_addr(itV), j > 0);
+          issue_pv(t ? C::T_O1 : C::T_O0, t ? C::T_S1 : C::T_S0, stage_addr(itV), j > 0);
           if (j + 1 < nt[t]) {
             if (!k_ready) {
-              if (!(ok = mbar_wait(kv_full(itK % C::NS), stage_par(itK), wc))) break;
+              if (!(ok = __all_sync(0xffffffffu, mbar_wait(kv_full(itK % C::NS), stage_par(itK), wc))))
+                break;
               tc_fence_after();
               k_ready = true;
             }
-            issue_qk(tS[t], sb + C::Q_OFF + t * C::TILE, stage_addr(itK));
-            mma_commit(s_full(t));
+            issue_qk(t ? C::T_S1 : C::T_S0, sb + C::Q_OFF + t * C::TILE, stage_addr(itK));
+            mma_commit_e(s_full(t));
           }
         }
         if (!ok) break;
-        mma_commit(kv_empty(itV % C::NS));
-        if (k_ready) mma_commit(kv_empty(itK % C::NS));
+        mma_commit_e(kv_empty(itV % C::NS));
+        if (k_ready) mma_commit_e(kv_empty(itK % C::NS));
       }
-      mma_commit(o_full);
+      mma_commit_e(o_full);
       if (!ok) mbar_wait_drain(o_full, 0);  // every issued MMA has completed before TMEM is freed
     }
     __syncwarp();
@@ -329,7 +340,7 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   if (warp == 8) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    tmem_dealloc(*tmem_slot, C::TMEM_COLS);
   }
 }
 

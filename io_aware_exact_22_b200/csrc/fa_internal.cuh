@@ -41,10 +41,13 @@ cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, cons
 
 cudaError_t launch_bwd_pre(const void* o, const void* dO, const float* lse, float* ld, float* dq_acc,
                            int BH, int N, int d, cudaStream_t stream);
+// fp32 [BH, N, d] tensor map without swizzle, box = box_inner columns x box_rows rows.
+bool make_tmap_f32(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_inner, int box_rows);
+
 cudaError_t launch_bwd_main(int d, const CUtensorMap& tq, const CUtensorMap& tk,
                             const CUtensorMap& tv, const CUtensorMap& tdo,
-                            const CUtensorMap& tdk, const CUtensorMap& tdv, const BwdArgs& a,
-                            cudaStream_t stream);
+                            const CUtensorMap& tdk, const CUtensorMap& tdv,
+                            const CUtensorMap& tdq, const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_post(const float* dq_acc, void* dq, long long elems, float scale,
                             cudaStream_t stream);
 
