@@ -242,25 +242,31 @@ __global__ void __launch_bounds__(448, 1)
     // issued by one thread execute in order.
     if (!*abort_flag) {
       bool ok = __all_sync(0xffffffffu, mbar_wait(kv_full, 0, wc));
-      const uint32_t kA = sb + C::K_OFF, vA = sb + C::V_OFF;
-      auto q_addr = [&](int n) { return sb + C::ST_OFF + (n % C::NSQ) * C::ST_BYTES; };
+      // Base descriptors; each MMA adds its byte offset (see sdesc_add).
+      const uint64_t dK_k = sdesc_sw128(sb + C::K_OFF, 16, 1024);        // K_j, K-major (S^T)
+      const uint64_t dV_k = sdesc_sw128(sb + C::V_OFF, 16, 1024);        // V_j, K-major (dP^T)
+      const uint64_t dK_mn = sdesc_sw128(sb + C::K_OFF, 16384, 1024);    // K_j, MN-major (dQ^T)
+      const uint64_t dQ_k = sdesc_sw128(sb + C::ST_OFF, 16, 1024);       // Q_i, K-major (S^T)
+      const uint64_t dO_k = sdesc_sw128(sb + C::ST_OFF + C::QT, 16, 1024);  // dO_i, K-major (dP^T)
+      const uint64_t dQ_mn = sdesc_sw128(sb + C::ST_OFF, 8192, 1024);    // Q_i, MN-major (dK)
+      const uint64_t dO_mn = sdesc_sw128(sb + C::ST_OFF + C::QT, 8192, 1024);  // dO_i, MN-major (dV)
+      const uint64_t dS_mn = sdesc_sw128(sb + C::DS_OFF, 8192, 1024);    // dS^T, MN-major (dQ^T)
+      auto st_off = [&](int n) { return (uint32_t)((n % C::NSQ) * C::ST_BYTES); };
       auto issue_s = [&](int n) {  // S^T = K_j Q_i^T  (K over d)
-        const uint32_t qA = q_addr(n);
+        const uint32_t so = st_off(n);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32, qo = (k >> 2) * 8192 + (k & 3) * 32;
-          mma_ss_e(tmem + C::T_S, sdesc_sw128(kA + ko, 16, 1024), sdesc_sw128(qA + qo, 16, 1024),
-                   C::IDESC_S, k > 0);
+          mma_ss_e(tmem + C::T_S, sdesc_add(dK_k, ko), sdesc_add(dQ_k, so + qo), C::IDESC_S, k > 0);
         }
         mma_commit_e(s_full);
       };
       auto issue_dp = [&](int n) {  // dP^T = V_j dO_i^T
-        const uint32_t doA = q_addr(n) + C::QT;
+        const uint32_t so = st_off(n);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32, qo = (k >> 2) * 8192 + (k & 3) * 32;
-          mma_ss_e(tmem + C::T_DP, sdesc_sw128(vA + ko, 16, 1024), sdesc_sw128(doA + qo, 16, 1024),
-                   C::IDESC_S, k > 0);
+          mma_ss_e(tmem + C::T_DP, sdesc_add(dV_k, ko), sdesc_add(dO_k, so + qo), C::IDESC_S, k > 0);
         }
         mma_commit_e(dp_full);
       };
@@ -274,14 +280,13 @@ __global__ void __launch_bounds__(448, 1)
       for (int n = 0; n < count && ok; ++n) {
         const int s = n % C::NSQ;
         const int b = n & 1;
-        const uint32_t qA = q_addr(n);
-        const uint32_t doA = qA + C::QT;
+        const uint32_t so = st_off(n);
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(p_ready, n & 1, wc)))) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 4; ++k)  // dV += P^T dO_i  (K over the 64 queries)
-          mma_ts_e(tmem + C::T_DV, tmem + C::T_S + 32 * (k >> 1) + 8 * (k & 1),
-                   sdesc_sw128(doA + k * 2048, 8192, 1024), C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
+          mma_ts_e(tmem + C::T_DV, tmem + C::T_S + 32 * (k >> 1) + 8 * (k & 1), sdesc_add(dO_mn, so + k * 2048),
+                   C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
         const bool more = n + 1 < count;
         if (more) {
           if (!(ok = __all_sync(0xffffffffu,
@@ -294,15 +299,14 @@ __global__ void __launch_bounds__(448, 1)
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 4; ++k)  // dK += dS^T Q_i
-          mma_ts_e(tmem + C::T_DK, tmem + C::T_DP + 32 * (k >> 1) + 8 * (k & 1),
-                   sdesc_sw128(qA + k * 2048, 8192, 1024), C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
+          mma_ts_e(tmem + C::T_DK, tmem + C::T_DP + 32 * (k >> 1) + 8 * (k & 1), sdesc_add(dQ_mn, so + k * 2048),
+                   C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(dq_free(b), ((n >> 1) & 1) ^ 1, wc)))) break;
         tc_fence_after();
-        const uint32_t dsA = sb + C::DS_OFF + b * C::DS_BYTES;
 #pragma unroll
         for (int k = 0; k < 8; ++k)  // dQ_i^T = K_j^T dS^T  (K over the 128 keys)
-          mma_ss_e(tmem + C::T_DQ + 64 * b, sdesc_sw128(kA + k * 2048, 16384, 1024),
-                   sdesc_sw128(dsA + k * 2048, 8192, 1024), C::IDESC_Q, k > 0);
+          mma_ss_e(tmem + C::T_DQ + 64 * b, sdesc_add(dK_mn, k * 2048), sdesc_add(dS_mn, b * C::DS_BYTES + k * 2048),
+                   C::IDESC_Q, k > 0);
         mma_commit_e(dq_full(b));
         mma_commit_e(ds_free(b));
         mma_commit_e(qd_empty(s));

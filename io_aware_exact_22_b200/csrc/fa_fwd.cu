@@ -26,6 +26,9 @@ namespace fa {
 
 using namespace ptx;
 
+// Column pairs (out of every 8 pairs) whose exponential is evaluated on the FMA pipe.
+constexpr int kPolyPairsOf8 = 3;
+
 template <int D>
 struct FwdCfg {
   static constexpr int NBOX = D / 64;              // 64-column (128-byte) swizzle boxes per row
@@ -150,30 +153,32 @@ __global__ void __launch_bounds__(320, 1)
     // ------------------------------------------------------------ MMA issuer (whole warp)
     if (!*abort_flag) {
       const int nt[2] = {n0, n1};
-      auto issue_qk = [&](uint32_t dst, uint32_t qaddr, uint32_t kaddr) {
+      // Base descriptors; each MMA adds its byte offset (see sdesc_add).
+      const uint64_t dQ_k = sdesc_sw128(sb + C::Q_OFF, 16, 1024);       // Q tiles, K-major
+      const uint64_t dK_k = sdesc_sw128(sb + C::KV_OFF, 16, 1024);      // K stages, K-major
+      const uint64_t dV_mn = sdesc_sw128(sb + C::KV_OFF, 16384, 1024);  // V stages, MN-major
+      auto issue_qk = [&](uint32_t dst, uint32_t qoff, uint32_t koff) {
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-          mma_ss_e(dst, sdesc_sw128(qaddr + off, 16, 1024), sdesc_sw128(kaddr + off, 16, 1024),
-                   C::IDESC_QK, k > 0);
+          mma_ss_e(dst, sdesc_add(dQ_k, qoff + off), sdesc_add(dK_k, koff + off), C::IDESC_QK, k > 0);
         }
       };
-      auto issue_pv = [&](uint32_t dst, uint32_t ptm, uint32_t vaddr, bool acc) {
+      auto issue_pv = [&](uint32_t dst, uint32_t ptm, uint32_t voff, bool acc) {
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          mma_ts_e(dst, ptm + 8 * k, sdesc_sw128(vaddr + k * 2048, 16384, 1024), C::IDESC_PV,
-                   (acc || k > 0) ? 1u : 0u);
+          mma_ts_e(dst, ptm + 8 * k, sdesc_add(dV_mn, voff + k * 2048), C::IDESC_PV, (acc || k > 0) ? 1u : 0u);
       };
-      auto stage_addr = [&](int it) { return sb + C::KV_OFF + (it % C::NS) * C::TILE; };
+      auto stage_addr = [&](int it) { return (uint32_t)((it % C::NS) * C::TILE); };
       auto stage_par = [&](int it) { return (uint32_t)((it / C::NS) & 1); };
       bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, wc));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(kv_full(0), 0, wc));
       if (ok) {
         tc_fence_after();
-        issue_qk(C::T_S0, sb + C::Q_OFF, stage_addr(0));
+        issue_qk(C::T_S0, 0u, stage_addr(0));
         mma_commit_e(s_full(0));
         if (n1 > 0) {
-          issue_qk(C::T_S1, sb + C::Q_OFF + C::TILE, stage_addr(0));
+          issue_qk(C::T_S1, (uint32_t)C::TILE, stage_addr(0));
           mma_commit_e(s_full(1));
         }
         mma_commit_e(kv_empty(0));
@@ -196,7 +201,7 @@ __global__ void __launch_bounds__(320, 1)
               tc_fence_after();
               k_ready = true;
             }
-            issue_qk(t ? C::T_S1 : C::T_S0, sb + C::Q_OFF + t * C::TILE, stage_addr(itK));
+            issue_qk(t ? C::T_S1 : C::T_S0, (uint32_t)(t * C::TILE), stage_addr(itK));
             mma_commit_e(s_full(t));
           }
         }
@@ -237,22 +242,61 @@ __global__ void __launch_bounds__(320, 1)
       float x[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
-      if (j == ntile - 1) {  // the only block that can hold the diagonal or the ragged tail
-        int lim = a.N - 1 - 128 * j;
+      const bool edge = (j == ntile - 1);  // the only block that can hold the diagonal or the tail
+      uint32_t pk[64];
+
+      // Exponentials of a full (unmasked) block against reference -mneg: y = s * cs - m for a
+      // pair of columns in one f32x2 FMA; kPolyPairsOf8 of every 8 pairs take the FMA-pipe
+      // exponential, the rest the special-function unit; the row sum is kept in two f32x2
+      // accumulators.  Returns the row sum of the block.
+      auto exp_full = [&](float mneg) -> float {
+        const uint64_t cs2 = f2_pack(cs, cs), mn2 = f2_pack(mneg, mneg);
+        uint64_t sa = f2_pack(0.f, 0.f), sb2 = f2_pack(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          const uint64_t y = f2_fma(f2_pack(x[c], x[c + 1]), cs2, mn2);
+          float p0, p1;
+          if (((c >> 1) & 7) < kPolyPairsOf8) {
+            ex2_poly2(y, p0, p1);
+          } else {
+            float y0, y1;
+            f2_unpack(y, y0, y1);
+            p0 = ex2(y0);
+            p1 = ex2(y1);
+          }
+          if ((c >> 1) & 1)
+            sb2 = f2_add(sb2, f2_pack(p0, p1));
+          else
+            sa = f2_add(sa, f2_pack(p0, p1));
+          pk[c >> 1] = pack_bf16(p0, p1);
+        }
+        float s0, s1, s2, s3;
+        f2_unpack(sa, s0, s1);
+        f2_unpack(sb2, s2, s3);
+        return (s0 + s1) + (s2 + s3);
+      };
+      // Row max with 3-input max (two new columns per instruction, four chains), scaled.
+      auto block_max = [&]() -> float {
+        float mx0 = fmaxf(x[0], x[1]), mx1 = fmaxf(x[2], x[3]), mx2 = fmaxf(x[4], x[5]), mx3 = fmaxf(x[6], x[7]);
+#pragma unroll
+        for (int c = 8; c < 128; c += 8) {
+          mx0 = max3(mx0, x[c], x[c + 1]);
+          mx1 = max3(mx1, x[c + 2], x[c + 3]);
+          mx2 = max3(mx2, x[c + 4], x[c + 5]);
+          mx3 = max3(mx3, x[c + 6], x[c + 7]);
+        }
+        return max3(mx0, mx1, fmaxf(mx2, mx3)) * cs;
+      };
+
+      int lim = 127;  // last visible column of this row in this block
+      if (edge) {
+        lim = a.N - 1 - 128 * j;
         if (a.causal) lim = min(lim, qrow - 128 * j);
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c > lim) x[c] = -INFINITY;
       }
-      float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
-#pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, x[c]);
-        mx1 = fmaxf(mx1, x[c + 1]);
-        mx2 = fmaxf(mx2, x[c + 2]);
-        mx3 = fmaxf(mx3, x[c + 3]);
-      }
-      const float mblk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * cs;
+      const float mblk = block_max();
       const bool move = mblk > m_ref + 8.0f;
       float alpha = 1.f;
       if (move) {
@@ -274,17 +318,23 @@ __global__ void __launch_bounds__(320, 1)
       }
       l *= alpha;
       const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
-      float rs0 = 0.f, rs1 = 0.f;
-      uint32_t pk[64];
+      float rsum;
+      if (!edge) {
+        rsum = exp_full(mneg);
+      } else {
+        // the block with the diagonal or the ragged tail: masked columns are exactly 0
+        float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = ex2(fmaf(x[c], cs, mneg));
-        const float p1 = ex2(fmaf(x[c + 1], cs, mneg));
-        rs0 += p0;
-        rs1 += p1;
-        pk[c >> 1] = pack_bf16(p0, p1);
+        for (int c = 0; c < 128; c += 2) {
+          const float p0 = (c > lim) ? 0.f : ex2(fmaf(x[c], cs, mneg));
+          const float p1 = (c + 1 > lim) ? 0.f : ex2(fmaf(x[c + 1], cs, mneg));
+          rs0 += p0;
+          rs1 += p1;
+          pk[c >> 1] = pack_bf16(p0, p1);
+        }
+        rsum = rs0 + rs1;
       }
-      l += rs0 + rs1;
+      l += rsum;
       tmem_st32(tSrow + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
       tmem_st32(tSrow + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tmem_wait_st();

@@ -66,26 +66,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Bounded wait for the phase with the given parity.  Returns false when the CTA-wide abort
 // flag is raised or the time limit runs out (then it raises the CTA flag and the device
-// status word), so that every waiter leaves its loop and the kernel exits.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& w) {
-  if (mbar_try_wait(bar, parity)) return true;
+// status word), so that every waiter leaves its loop and the kernel exits.  The slow path is
+// kept out of line so that hot loops only carry the first probe.
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                            uint32_t* status) {
   const uint64_t t0 = globaltimer();
   uint32_t it = 0;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((++it & 63u) == 0) {
-      if (*w.abort_flag) return false;
-      if ((*(volatile uint32_t*)w.status) & FA_DEV_TIMEOUT) {
-        *w.abort_flag = 1;
+      if (*abort_flag) return false;
+      if ((*(volatile uint32_t*)status) & FA_DEV_TIMEOUT) {
+        *abort_flag = 1;
         return false;
       }
       if (globaltimer() - t0 > kWaitLimitNs) {
-        *w.abort_flag = 1;
-        atomicOr(w.status, FA_DEV_TIMEOUT);
+        *abort_flag = 1;
+        atomicOr(status, FA_DEV_TIMEOUT);
         return false;
       }
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& w) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, w.abort_flag, w.status);
 }
 
 // Wait used only on the abort path, to let copies already in flight land before exit.
@@ -221,6 +226,11 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       FA_W8(0), FA_W8(8)
       : "memory");
 }
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               FA_W8(0)
+               : "memory");
+}
 #undef FA_R8
 #undef FA_W8
 
@@ -338,6 +348,12 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
+// The start-address field sits in the low bits, so a descriptor for base + off (off a multiple
+// of 16 bytes, base + off below 256 KB) is the base descriptor plus off >> 4.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t byte_off) {
+  return desc + static_cast<uint64_t>(byte_off >> 4);
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D:
 //   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format (1 = bf16),
 //   bit 15 A major (1 = MN-major), bit 16 B major, bits 17-22 N >> 3, bits 24-28 M >> 4.
@@ -351,6 +367,63 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+// 2^x on the FMA pipe, for x <= 126 (x below -126, including -inf, gives 2^-126): split
+// x = n + f with n = round(x), f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose
+// coefficients minimise the maximum relative error on that interval (Remez exchange; fitted by
+// csrc/gen_exp2_poly.py, max relative error 7.5e-5 in float32); 2^n added to the exponent
+// field.  Adding 1.5 * 2^23 rounds x to an integer held in the low mantissa bits of t, and
+// (bits(t) << 23) is then n << 23 modulo 2^32.
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = __fadd_rn(x, 12582912.f);
+  const float f = __fsub_rn(x, __fsub_rn(t, 12582912.f));
+  float p = fmaf(__uint_as_float(0x3d61fbb0u), f, __uint_as_float(0x3e786f0du));
+  p = fmaf(p, f, __uint_as_float(0x3f31798du));
+  p = fmaf(p, f, __uint_as_float(0x3f7ffb49u));
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction for two lanes of work)
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// ex2_poly on a pair of lanes, with the reduction and Horner steps in f32x2 arithmetic.
+__device__ __forceinline__ void ex2_poly2(uint64_t y, float& r0, float& r1) {
+  float a, b;
+  f2_unpack(y, a, b);
+  const uint64_t x = f2_pack(fmaxf(a, -126.f), fmaxf(b, -126.f));
+  const uint64_t t = f2_add(x, f2_pack(12582912.f, 12582912.f));    // round(x) + 1.5 * 2^23
+  const uint64_t n = f2_add(t, f2_pack(-12582912.f, -12582912.f));   // round(x), exactly
+  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), x);              // x - round(x)
+  uint64_t p = f2_fma(f2_pack(__uint_as_float(0x3d61fbb0u), __uint_as_float(0x3d61fbb0u)), f,
+                      f2_pack(__uint_as_float(0x3e786f0du), __uint_as_float(0x3e786f0du)));
+  p = f2_fma(p, f, f2_pack(__uint_as_float(0x3f31798du), __uint_as_float(0x3f31798du)));
+  p = f2_fma(p, f, f2_pack(__uint_as_float(0x3f7ffb49u), __uint_as_float(0x3f7ffb49u)));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 // Pack two fp32 into bf16x2 with round-to-nearest-even; `lo` lands in the low 16 bits.
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
