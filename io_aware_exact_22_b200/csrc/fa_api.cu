@@ -188,7 +188,7 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
   if (!make_tmap_bf16(&tq, q, BH, N, d, 64) || !make_tmap_bf16(&tk, k, BH, N, d, 128) ||
       !make_tmap_bf16(&tv, v, BH, N, d, 128) || !make_tmap_bf16(&tdo, dO, BH, N, d, 64) ||
       !make_tmap_bf16(&tdk, dk, BH, N, d, 32) || !make_tmap_bf16(&tdv, dv, BH, N, d, 32) ||
-      !make_tmap_f32(&tdq, dq_acc, BH, N, d, 32, 64))
+      !make_tmap_f32(&tdq, dq_acc, BH, N, d, 32, 64 - kBwdDqRedRows))
     return FA_ERR_CUDA;
   BwdArgs a;
   if (!(a.status = device_status_word())) return FA_ERR_CUDA;

@@ -103,8 +103,8 @@ struct BwdCfg {
   static constexpr int ST_BYTES = 2 * QT;
   static constexpr int DS_OFF = ST_OFF + NSQ * ST_BYTES;  // dS^T, two buffers of 128 x 64 bf16
   static constexpr int DS_BYTES = 128 * BQ * 2;
-  static constexpr int DQS_OFF = DS_OFF + 2 * DS_BYTES;   // dQ staging: 4 warps x [64 q][32 d] fp32
-  static constexpr int DQS_WARP = BQ * 32 * 4;
+  static constexpr int DQS_OFF = DS_OFF + 2 * DS_BYTES;   // dQ staging: 4 warps x [rows][32 d] fp32
+  static constexpr int DQS_WARP = (BQ - kBwdDqRedRows) * 32 * 4;
   static constexpr int LD_OFF = DQS_OFF + 4 * DQS_WARP;
   static constexpr int BAR_OFF = LD_OFF + NSQ * LDB;
   // kv_full, qd_full[3], qd_empty[3], s_full, dp_full, p_ready, ds_ready, dq_full[2],
@@ -420,16 +420,27 @@ __global__ void __launch_bounds__(448, 1)
       reg_fence(v);
       tc_fence_before();
       mbar_arrive(dq_free(b));
-      // [64 queries][32 d] fp32 slice of this warp; lane = d, so each row is one 128-byte store
-      if (lane == 0) bulk_wait_read0();  // the previous reduce has finished reading the staging
-      __syncwarp();
+      // Split between two paths that use different resources: the first kBwdDqRedRows query
+      // rows are added with fp32 reductions straight from registers (lane = d, so each row is
+      // one coalesced 128-byte request), the rest are staged as a [rows][32 d] fp32 slice in
+      // shared memory and added by one TMA reduce-add.
+      const int q0 = C::BQ * i;
+      const int nred = min(kBwdDqRedRows, a.N - q0);
+      float* dst = a.dq_acc + ((size_t)bh * a.N + q0) * C::D + wq * 32 + lane;
 #pragma unroll
-      for (int c = 0; c < 64; ++c) stage[c * 32 + lane] = __uint_as_float(v[c]);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        tma_reduce_add_3d(&tmdQ, stage_s, 32 * wq, C::BQ * i, bh);
-        bulk_commit();
+      for (int c = 0; c < kBwdDqRedRows; ++c)
+        if (c < nred) atomicAdd(dst + (size_t)c * C::D, __uint_as_float(v[c]));
+      if (q0 + kBwdDqRedRows < a.N) {
+        if (lane == 0) bulk_wait_read0();  // the previous reduce has finished reading the staging
+        __syncwarp();
+#pragma unroll
+        for (int c = kBwdDqRedRows; c < 64; ++c) stage[(c - kBwdDqRedRows) * 32 + lane] = __uint_as_float(v[c]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_3d(&tmdQ, stage_s, 32 * wq, q0 + kBwdDqRedRows, bh);
+          bulk_commit();
+        }
       }
     }
     if (lane == 0) bulk_wait0();

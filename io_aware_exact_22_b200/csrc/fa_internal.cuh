@@ -30,6 +30,11 @@ struct BwdArgs {
   float scale_log2;  // scale * log2(e)
 };
 
+// Backward dQ accumulation: of each 64-row query tile, the first kBwdDqRedRows rows are added
+// into the fp32 accumulator with per-thread reductions, the rest with one TMA reduce-add
+// (tensor-map box of 64 - kBwdDqRedRows rows).
+constexpr int kBwdDqRedRows = 32;
+
 // Device address of this library's status word on the current device (nullptr on error).
 uint32_t* device_status_word();
 
