@@ -128,6 +128,18 @@ fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const vo
  */
 fa_status_t fa_get_device_status(void* stream);
 
+/*
+ * Self-test of the bounded waits (failure detection; no counterpart on the pages).
+ * Launches one CTA whose single thread waits on an mbarrier phase that nothing completes,
+ * for at most limit_ms milliseconds (1..1000) of %globaltimer; the wait then runs out, the
+ * kernel records the timeout in the device status word and exits normally (no trap, no
+ * fault: the context stays usable).  A following fa_get_device_status(stream) returns
+ * FA_ERR_TIMEOUT and clears the word.  Returns FA_ERR_INVALID_ARG for a limit out of range,
+ * FA_ERR_CUDA if the launch fails.  Kernels launched while the timeout bit is set exit early,
+ * so read the status before launching anything else.
+ */
+fa_status_t fa_selftest_wait_timeout(int limit_ms, void* stream);
+
 /* Static, human-readable name of a status code. */
 const char* fa_status_string(fa_status_t s);
 

@@ -100,6 +100,26 @@ bool make_tmap_bf16(CUtensorMap* m, const void* ptr, int BH, int N, int d, int b
   return r == CUDA_SUCCESS;
 }
 
+// One thread waits on a phase that never completes; the bounded wait records the timeout.
+__global__ void fa_wait_probe_kernel(uint32_t* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = ptx::smem_u32(&bar);
+  ptx::mbar_init(b, 1);
+  ptx::fence_mbar_init();
+  const uint64_t t0 = ptx::globaltimer();
+  while (!ptx::mbar_try_wait(b, 0)) {
+    if (ptx::globaltimer() - t0 > limit_ns) {
+      atomicOr(status, FA_DEV_TIMEOUT);
+      return;
+    }
+  }
+}
+
+cudaError_t launch_wait_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t stream) {
+  fa_wait_probe_kernel<<<1, 1, 0, stream>>>(status, limit_ns);
+  return cudaGetLastError();
+}
+
 bool make_tmap_f32(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_inner, int box_rows) {
   auto enc = encode_fn();
   if (!enc) return false;
@@ -206,6 +226,15 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
   if (e != cudaSuccess) return FA_ERR_CUDA;
   if (launch_bwd_post(dq_acc, dq, rows * d, scale, s) != cudaSuccess) return FA_ERR_CUDA;
   return FA_OK;
+}
+
+fa_status_t fa_selftest_wait_timeout(int limit_ms, void* stream) {
+  if (limit_ms < 1 || limit_ms > 1000) return FA_ERR_INVALID_ARG;
+  uint32_t* status = device_status_word();
+  if (!status) return FA_ERR_CUDA;
+  return launch_wait_probe(status, (uint64_t)limit_ms * 1000000ull, (cudaStream_t)stream) == cudaSuccess
+             ? FA_OK
+             : FA_ERR_CUDA;
 }
 
 fa_status_t fa_get_device_status(void* stream) {

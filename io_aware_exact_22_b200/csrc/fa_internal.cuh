@@ -38,6 +38,9 @@ constexpr int kBwdDqRedRows = 32;
 // Device address of this library's status word on the current device (nullptr on error).
 uint32_t* device_status_word();
 
+// Launches the bounded-wait self-test kernel (see fa_selftest_wait_timeout).
+cudaError_t launch_wait_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);
+
 // Tensor maps for a bf16 [BH, N, d] tensor, 128-byte swizzle, box = 64 columns x `rows`.
 bool make_tmap_bf16(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_rows);
 

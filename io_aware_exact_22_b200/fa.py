@@ -22,7 +22,7 @@ LIB_PATH = os.environ.get("FA_LIB_PATH", os.path.join(_HERE, "libfa.so"))
 STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_CUDA",
           4: "FA_ERR_TIMEOUT"}
 EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_device_status",
-           "fa_status_string", "fa_version", "fa_bwd_noalloc")
+           "fa_status_string", "fa_version", "fa_bwd_noalloc", "fa_selftest_wait_timeout")
 # Size of the library's built-in scratch used by fa_bwd_noalloc (include/fa.h).
 NOALLOC_MAX_SCRATCH_BYTES = 64 << 20
 
@@ -58,6 +58,8 @@ def lib() -> ctypes.CDLL:
         L.fa_version.restype = i
         L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
         L.fa_bwd_noalloc.restype = i
+        L.fa_selftest_wait_timeout.argtypes = [i, vp]
+        L.fa_selftest_wait_timeout.restype = i
         _lib = L
     return _lib
 
@@ -106,6 +108,10 @@ def fa_bwd_workspace_bytes(B, H, N, d) -> int:
 
 def fa_get_device_status(stream=None) -> int:
     return lib().fa_get_device_status(_stream(stream))
+
+
+def fa_selftest_wait_timeout(limit_ms: int, stream=None) -> int:
+    return lib().fa_selftest_wait_timeout(int(limit_ms), _stream(stream))
 
 
 def fa_status_string(code: int) -> str:
