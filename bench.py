@@ -253,7 +253,10 @@ def run_gpu(args):
         return None
 
     peaks, peak_src = load_peaks()
-    peak = peaks["bf16_tflops"]
+    # The step loop keeps the GPU busy for the whole timed region (under the power cap), so the
+    # sustained cuBLAS figure is the denominator; the burst-based fraction is reported too.
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    peak_burst = peaks["bf16_tflops"]
     bwd_tflops = w.bwd_flops() / (bwd_ms * 1e-3) / 1e12
     fwd_tflops = w.fwd_flops() / (fwd_ms * 1e-3) / 1e12
     line = {
@@ -281,11 +284,13 @@ def run_gpu(args):
                      "bound": "tensor", "achieved": round(bwd_tflops, 1), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(bwd_tflops / peak, 4),
                      "traffic": kernel_traffic("fa_bwd_main_kernel"),
-                     "peak_source": f"{peak_src} bf16_tflops (burst)",
+                     "peak_source": f"{peak_src} bf16_tflops_sustained",
+                     "frac_of_burst_peak": round(bwd_tflops / peak_burst, 4),
                      "algorithmic_flops_per_launch": w.bwd_flops()},
         "roofline_fwd": {"kernel": "fa_fwd_kernel<128>", "bound": "tensor",
                          "achieved": round(fwd_tflops, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(fwd_tflops / peak, 4),
+                         "frac_of_burst_peak": round(fwd_tflops / peak_burst, 4),
                          "traffic": kernel_traffic("fa_fwd_kernel"),
                          "algorithmic_flops_per_launch": w.fwd_flops()},
         "clocks": clk,
