@@ -73,6 +73,28 @@ fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* 
                    int B, int H, int N, int d, float scale, int causal, void* stream);
 
 /*
+ * Forward pass split over the key range (split-KV), for problems too small to fill the GPU
+ * (few heads or few query rows against many keys).  Each (head, 256 query rows) work item is
+ * divided into num_splits contiguous ranges of 128-key blocks; every range yields the
+ * normalised partial output O_s (fp32) and its LSE_s, and a second kernel combines them with
+ * the two-block softmax merge of "Flash Attention" (special-jiahao.github.io, section 增量求解
+ * softmax) extended to num_splits blocks:
+ *     M = max_s LSE_s,  w_s = exp(LSE_s - M),  O = sum_s w_s O_s / sum_s w_s,
+ *     LSE = M + ln sum_s w_s.
+ * The result equals fa_fwd's up to rounding.  Arguments as in fa_fwd, plus:
+ *   num_splits      : >= 1, or <= 0 for fa_fwd_splitkv_default_splits(...); values above the
+ *                     number of 128-key blocks are clamped to it.  1 runs fa_fwd itself.
+ *   workspace       : device scratch, 256-byte aligned, at least
+ *                     fa_fwd_splitkv_workspace_bytes(B,H,N,d,splits) bytes for the number of
+ *                     splits used (not needed, may be NULL, when that number is 1).
+ */
+int fa_fwd_splitkv_default_splits(int B, int H, int N, int d, int causal);
+size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int N, int d, int num_splits);
+fa_status_t fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int B, int H, int N, int d, float scale, int causal, int num_splits,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Bytes of device workspace that fa_bwd needs: per 64-row query tile, the fp32 base-2 LSE and
  * row term D_i of its 64 rows (B*H*ceil(N/64)*128 floats, rounded up to 256 bytes), followed
  * by the fp32 dQ accumulator [B*H*N*d].  Returns 0 for an empty or invalid shape.

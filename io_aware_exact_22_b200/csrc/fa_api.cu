@@ -120,7 +120,8 @@ cudaError_t launch_wait_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t 
   return cudaGetLastError();
 }
 
-bool make_tmap_f32(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_inner, int box_rows) {
+bool make_tmap_f32(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_inner, int box_rows,
+                   bool swizzle128) {
   auto enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
@@ -128,7 +129,8 @@ bool make_tmap_f32(CUtensorMap* m, const void* ptr, int BH, int N, int d, int bo
   cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box,
-                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -174,8 +176,79 @@ fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* 
   a.nqb = (N + 255) / 256;
   a.causal = causal;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  a.nsplit = 1;
   if ((long long)a.BH * a.nqb > INT_MAX) return FA_ERR_INVALID_ARG;
   return launch_fwd(d, tq, tk, tv, to, a, (cudaStream_t)stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// Split count used when the caller passes num_splits <= 0: enough CTAs to cover the SMs once,
+// at most one split per 128-key block and at most 32.
+int fa_fwd_splitkv_default_splits(int B, int H, int N, int d, int causal) {
+  (void)d;
+  (void)causal;
+  if (B <= 0 || H <= 0 || N <= 0) return 1;
+  int nsm = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) nsm = v;
+  }
+  const long long items = (long long)B * H * ((N + 255) / 256);
+  if (items >= nsm) return 1;
+  long long sp = (nsm + items - 1) / items;
+  const long long kblocks = (N + 127) / 128;
+  if (sp > kblocks) sp = kblocks;
+  if (sp > 32) sp = 32;
+  return sp < 1 ? 1 : (int)sp;
+}
+
+static size_t splitkv_o_bytes(long long rows, int d, int sp) {
+  return (((size_t)sp * rows * d * 4) + 255) & ~(size_t)255;
+}
+
+size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int N, int d, int num_splits) {
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || num_splits <= 1) return 0;
+  const long long rows = (long long)B * H * N;
+  return splitkv_o_bytes(rows, d, num_splits) + (size_t)num_splits * rows * 4;
+}
+
+fa_status_t fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                           int N, int d, float scale, int causal, int num_splits, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  bool empty = false;
+  fa_status_t st = check_shape(B, H, N, d, scale, causal, &empty);
+  if (st != FA_OK || empty) return st;
+  int sp = num_splits > 0 ? num_splits : fa_fwd_splitkv_default_splits(B, H, N, d, causal);
+  const int kblocks = (N + 127) / 128;
+  if (sp > kblocks) sp = kblocks;
+  if (sp <= 1) return fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, stream);
+  if (!q || !k || !v || !o || !lse || !workspace) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(workspace, 256))
+    return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < fa_fwd_splitkv_workspace_bytes(B, H, N, d, sp)) return FA_ERR_INVALID_ARG;
+  if ((st = check_device()) != FA_OK) return st;
+  const int BH = B * H;
+  const long long rows = (long long)BH * N;
+  if ((long long)BH * sp > INT_MAX || (long long)BH * ((N + 255) / 256) * sp > INT_MAX) return FA_ERR_INVALID_ARG;
+  float* o_part = reinterpret_cast<float*>(workspace);
+  float* lse_part = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + splitkv_o_bytes(rows, d, sp));
+  CUtensorMap tq, tk, tv, to;
+  if (!make_tmap_bf16(&tq, q, BH, N, d, 128) || !make_tmap_bf16(&tk, k, BH, N, d, 128) ||
+      !make_tmap_bf16(&tv, v, BH, N, d, 128) || !make_tmap_f32(&to, o_part, BH * sp, N, d, 32, 32, true))
+    return FA_ERR_CUDA;
+  FwdArgs a;
+  if (!(a.status = device_status_word())) return FA_ERR_CUDA;
+  a.lse = lse_part;
+  a.N = N;
+  a.BH = BH;
+  a.nqb = (N + 255) / 256;
+  a.causal = causal;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  a.nsplit = sp;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (launch_fwd(d, tq, tk, tv, to, a, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (launch_fwd_merge(o_part, lse_part, o, lse, sp, rows, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  return FA_OK;
 }
 
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {

@@ -49,7 +49,9 @@ struct FwdCfg {
   static constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);
 };
 
-template <int D>
+// PARTIAL: the CTA covers only its split's range of key blocks and writes the normalised
+// partial output O_s (fp32) and its LSE_s, to be combined by fa_fwd_merge_kernel.
+template <int D, bool PARTIAL>
 __global__ void __launch_bounds__(320, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -62,14 +64,23 @@ __global__ void __launch_bounds__(320, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: (head bh, block of 256 query rows); heavier causal blocks first
-  const int bh = blockIdx.x / a.nqb;
-  const int qb = a.nqb - 1 - (blockIdx.x % a.nqb);
+  // ---- work item: (head bh, block of 256 query rows, key split); heavier causal blocks first
+  const int split = blockIdx.x % a.nsplit;
+  const int item = blockIdx.x / a.nsplit;
+  const int bh = item / a.nqb;
+  const int qb = a.nqb - 1 - (item % a.nqb);
   const int q0 = qb * 256;
   const int Tk = (a.N + 127) >> 7;
   const bool has1 = (q0 + 128) < a.N;
-  const int n0 = a.causal ? min(Tk, 2 * qb + 1) : Tk;
-  const int n1 = has1 ? (a.causal ? min(Tk, 2 * qb + 2) : Tk) : 0;
+  // visible key blocks of each query tile, over the whole key range
+  const int n0g = a.causal ? min(Tk, 2 * qb + 1) : Tk;
+  const int n1g = has1 ? (a.causal ? min(Tk, 2 * qb + 2) : Tk) : 0;
+  // this split's contiguous share [kb0, kb1) of the key blocks, and each tile's count in it
+  const int nmaxg = max(n0g, n1g);
+  const int kb0 = (int)((long long)split * nmaxg / a.nsplit);
+  const int kb1 = (int)((long long)(split + 1) * nmaxg / a.nsplit);
+  const int n0 = max(0, min(kb1, n0g) - kb0);
+  const int n1 = max(0, min(kb1, n1g) - kb0);
   const int nmax = max(n0, n1);
 
   const uint32_t bar = sb + C::BAR_OFF;
@@ -113,7 +124,7 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 9) {
     // ------------------------------------------------------------ TMA producer (whole warp)
-    if (!*abort_flag) {
+    if (!*abort_flag && nmax > 0) {
       if (elect_one()) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
@@ -136,7 +147,7 @@ __global__ void __launch_bounds__(320, 1)
           mbar_arrive_expect_tx_e(kv_full(s), C::TILE);
           const CUtensorMap* m = kv ? &tmV : &tmK;
           for (int b = 0; b < C::NBOX; ++b)
-            tma_load_3d_e(sb + C::KV_OFF + s * C::TILE + b * 16384, m, kv_full(s), 64 * b, 128 * j, bh,
+            tma_load_3d_e(sb + C::KV_OFF + s * C::TILE + b * 16384, m, kv_full(s), 64 * b, 128 * (kb0 + j), bh,
                           keep);
         }
       }
@@ -151,7 +162,7 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer (whole warp)
-    if (!*abort_flag) {
+    if (!*abort_flag && nmax > 0) {
       const int nt[2] = {n0, n1};
       // Base descriptors; each MMA adds its byte offset (see sdesc_add).
       const uint64_t dQ_k = sdesc_sw128(sb + C::Q_OFF, 16, 1024);       // Q tiles, K-major
@@ -175,8 +186,10 @@ __global__ void __launch_bounds__(320, 1)
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(kv_full(0), 0, wc));
       if (ok) {
         tc_fence_after();
-        issue_qk(C::T_S0, 0u, stage_addr(0));
-        mma_commit_e(s_full(0));
+        if (n0 > 0) {
+          issue_qk(C::T_S0, 0u, stage_addr(0));
+          mma_commit_e(s_full(0));
+        }
         if (n1 > 0) {
           issue_qk(C::T_S1, (uint32_t)C::TILE, stage_addr(0));
           mma_commit_e(s_full(1));
@@ -218,7 +231,8 @@ __global__ void __launch_bounds__(320, 1)
     const int t = warp >> 2;
     const int wq = warp & 3;
     const int r = wq * 32 + lane;  // row within the query tile == TMEM lane
-    const int ntile = t ? n1 : n0;
+    const int ntile = t ? n1 : n0;      // blocks of this split
+    const int ntile_g = t ? n1g : n0g;  // blocks of the whole key range
     const int qrow = q0 + 128 * t + r;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tSrow = tmem + lane_off + 128u * t;
@@ -242,7 +256,8 @@ __global__ void __launch_bounds__(320, 1)
       float x[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
-      const bool edge = (j == ntile - 1);  // the only block that can hold the diagonal or the tail
+      const int jg = kb0 + j;                 // key block index in the whole key range
+      const bool edge = (jg == ntile_g - 1);  // the only block that can hold the diagonal or the tail
       uint32_t pk[64];
 
       // Exponentials of a full (unmasked) block against reference -mneg: y = s * cs - m for a
@@ -290,8 +305,8 @@ __global__ void __launch_bounds__(320, 1)
 
       int lim = 127;  // last visible column of this row in this block
       if (edge) {
-        lim = a.N - 1 - 128 * j;
-        if (a.causal) lim = min(lim, qrow - 128 * j);
+        lim = a.N - 1 - 128 * jg;
+        if (a.causal) lim = min(lim, qrow - 128 * jg);
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c > lim) x[c] = -INFINITY;
@@ -342,46 +357,82 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive(p_full(t));
     }
 
-    if (ntile > 0 && ok) {
+    if (PARTIAL && ntile == 0 && ok) {
+      // this split holds no key block of this tile: an empty partial (weight 0 in the merge)
+      if (qrow < a.N) a.lse[((size_t)split * a.BH + bh) * a.N + qrow] = -INFINITY;
+    } else if (ntile > 0 && ok) {
       // ---------------------------------------------------------- epilogue
       ok = __all_sync(0xffffffffu, mbar_wait(o_full, 0, wc));
       if (ok) {
         tc_fence_after();
         const float inv = (l > 0.f) ? 1.f / l : 0.f;
-        uint8_t* stage = gb + C::Q_OFF + t * C::TILE;  // Q_t is dead once o_full has fired
+        const int row0 = q0 + 128 * t + 32 * wq;
+        if (!PARTIAL) {
+          uint8_t* stage = gb + C::Q_OFF + t * C::TILE;  // Q_t is dead once o_full has fired
 #pragma unroll
-        for (int b = 0; b < C::NBOX; ++b) {
+          for (int b = 0; b < C::NBOX; ++b) {
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
+            for (int h = 0; h < 2; ++h) {
+              uint32_t o[32];
+              tmem_ld32(tOrow + 64 * b + 32 * h, o);
+              tmem_wait_ld();
+              reg_fence(o);
+#pragma unroll
+              for (int cc = 0; cc < 4; ++cc) {
+                uint4 v;
+                v.x = pack_bf16(__uint_as_float(o[8 * cc + 0]) * inv, __uint_as_float(o[8 * cc + 1]) * inv);
+                v.y = pack_bf16(__uint_as_float(o[8 * cc + 2]) * inv, __uint_as_float(o[8 * cc + 3]) * inv);
+                v.z = pack_bf16(__uint_as_float(o[8 * cc + 4]) * inv, __uint_as_float(o[8 * cc + 5]) * inv);
+                v.w = pack_bf16(__uint_as_float(o[8 * cc + 6]) * inv, __uint_as_float(o[8 * cc + 7]) * inv);
+                const int chunk = h * 4 + cc;  // 16-byte chunk within the 128-byte row
+                *reinterpret_cast<uint4*>(stage + b * 16384 + r * 128 + ((chunk ^ (r & 7)) << 4)) = v;
+              }
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < a.N) {
+            for (int b = 0; b < C::NBOX; ++b)
+              tma_store_3d(&tmO, sb + C::Q_OFF + t * C::TILE + b * 16384 + wq * 4096, 64 * b, row0, bh);
+            bulk_commit();
+            bulk_wait_read0();
+          }
+          __syncwarp();
+          if (qrow < a.N)
+            a.lse[(size_t)bh * a.N + qrow] =
+                (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+        } else {
+          // fp32 partial O_s = O / l of this split, staged in the (now idle) K/V ring as
+          // 32-column, 128-byte-swizzled boxes and written by TMA; then LSE_s.
+          constexpr int PBOX = D / 32;
+          const uint32_t pstage = C::KV_OFF + t * (128 * D * 4);
+          uint8_t* stage = gb + pstage;
+#pragma unroll
+          for (int b = 0; b < PBOX; ++b) {
             uint32_t o[32];
-            tmem_ld32(tOrow + 64 * b + 32 * h, o);
+            tmem_ld32(tOrow + 32 * b, o);
             tmem_wait_ld();
             reg_fence(o);
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-              uint4 v;
-              v.x = pack_bf16(__uint_as_float(o[8 * cc + 0]) * inv, __uint_as_float(o[8 * cc + 1]) * inv);
-              v.y = pack_bf16(__uint_as_float(o[8 * cc + 2]) * inv, __uint_as_float(o[8 * cc + 3]) * inv);
-              v.z = pack_bf16(__uint_as_float(o[8 * cc + 4]) * inv, __uint_as_float(o[8 * cc + 5]) * inv);
-              v.w = pack_bf16(__uint_as_float(o[8 * cc + 6]) * inv, __uint_as_float(o[8 * cc + 7]) * inv);
-              const int chunk = h * 4 + cc;  // 16-byte chunk within the 128-byte row
-              *reinterpret_cast<uint4*>(stage + b * 16384 + r * 128 + ((chunk ^ (r & 7)) << 4)) = v;
+            for (int cc = 0; cc < 8; ++cc) {
+              float4 v = make_float4(__uint_as_float(o[4 * cc + 0]) * inv, __uint_as_float(o[4 * cc + 1]) * inv,
+                                     __uint_as_float(o[4 * cc + 2]) * inv, __uint_as_float(o[4 * cc + 3]) * inv);
+              *reinterpret_cast<float4*>(stage + b * 16384 + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
             }
           }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < a.N) {
+            for (int b = 0; b < PBOX; ++b)
+              tma_store_3d(&tmO, sb + pstage + b * 16384 + wq * 4096, 32 * b, row0, split * a.BH + bh);
+            bulk_commit();
+            bulk_wait_read0();
+          }
+          __syncwarp();
+          if (qrow < a.N)
+            a.lse[((size_t)split * a.BH + bh) * a.N + qrow] =
+                (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994530942f : -INFINITY;
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        const int row0 = q0 + 128 * t + 32 * wq;
-        if (lane == 0 && row0 < a.N) {
-          for (int b = 0; b < C::NBOX; ++b)
-            tma_store_3d(&tmO, sb + C::Q_OFF + t * C::TILE + b * 16384 + wq * 4096, 64 * b, row0, bh);
-          bulk_commit();
-          bulk_wait_read0();
-        }
-        __syncwarp();
-        if (qrow < a.N)
-          a.lse[(size_t)bh * a.N + qrow] =
-              (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994530942f : -INFINITY;
       }
     }
   }
@@ -394,22 +445,91 @@ __global__ void __launch_bounds__(320, 1)
   }
 }
 
-template <int D>
+template <int D, bool PARTIAL>
 static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const CUtensorMap& to, const FwdArgs& a, cudaStream_t stream) {
   using C = FwdCfg<D>;
   static_assert(C::SMEM <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(fa_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  static_assert(2 * 128 * D * 4 <= C::NS * C::TILE, "partial-output staging must fit the K/V ring");
+  cudaError_t e =
+      cudaFuncSetAttribute(fa_fwd_kernel<D, PARTIAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  const long long grid = (long long)a.BH * a.nqb;
-  fa_fwd_kernel<D><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, to, a);
+  const long long grid = (long long)a.BH * a.nqb * a.nsplit;
+  fa_fwd_kernel<D, PARTIAL><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, to, a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& to, const FwdArgs& a, cudaStream_t stream) {
-  if (d == 64) return launch_fwd_t<64>(tq, tk, tv, to, a, stream);
-  return launch_fwd_t<128>(tq, tk, tv, to, a, stream);
+  if (a.nsplit > 1) {
+    if (d == 64) return launch_fwd_t<64, true>(tq, tk, tv, to, a, stream);
+    return launch_fwd_t<128, true>(tq, tk, tv, to, a, stream);
+  }
+  if (d == 64) return launch_fwd_t<64, false>(tq, tk, tv, to, a, stream);
+  return launch_fwd_t<128, false>(tq, tk, tv, to, a, stream);
+}
+
+// Combines the split-wise partial results of one query row, using the two-block softmax merge
+// of "Flash Attention" (special-jiahao.github.io), section 增量求解 softmax, applied to nsplit
+// blocks: with M = max_s LSE_s and weights w_s = e^{LSE_s - M} (each block's sum rescaled to
+// the common max), O = sum_s w_s O_s / sum_s w_s and LSE = M + ln sum_s w_s.  Splits with
+// LSE_s = -inf hold no visible key and are skipped.  One warp per row; lane holds D/32 columns.
+template <int D>
+__global__ void __launch_bounds__(256) fa_fwd_merge_kernel(const float* __restrict__ o_part,
+                                                           const float* __restrict__ lse_part,
+                                                           __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
+                                                           int nsplit, long long rows) {
+  constexpr int V = D / 32;
+  const int lane = threadIdx.x & 31;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < rows; row += nw) {
+    float m = -INFINITY;
+    for (int sp = 0; sp < nsplit; ++sp) m = fmaxf(m, lse_part[sp * rows + row]);
+    float acc[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) acc[e] = 0.f;
+    float wsum = 0.f;
+    if (m != -INFINITY) {
+      for (int sp = 0; sp < nsplit; ++sp) {
+        const float L = lse_part[sp * rows + row];
+        if (L == -INFINITY) continue;
+        const float w = expf(L - m);
+        wsum += w;
+        const float* src = o_part + ((size_t)sp * rows + row) * D + lane * V;
+        if (V == 4) {
+          const float4 x = *reinterpret_cast<const float4*>(src);
+          acc[0] += w * x.x; acc[1] += w * x.y; acc[2] += w * x.z; acc[3] += w * x.w;
+        } else {
+          const float2 x = *reinterpret_cast<const float2*>(src);
+          acc[0] += w * x.x; acc[1] += w * x.y;
+        }
+      }
+    }
+    const float inv = (wsum > 0.f) ? 1.f / wsum : 0.f;
+    __nv_bfloat16* dst = o + (size_t)row * D + lane * V;
+    if (V == 4) {
+      uint2 u;
+      u.x = pack_bf16(acc[0] * inv, acc[1] * inv);
+      u.y = pack_bf16(acc[2] * inv, acc[3] * inv);
+      *reinterpret_cast<uint2*>(dst) = u;
+    } else {
+      *reinterpret_cast<uint32_t*>(dst) = pack_bf16(acc[0] * inv, acc[1] * inv);
+    }
+    if (lane == 0) lse[row] = (wsum > 0.f) ? m + logf(wsum) : -INFINITY;
+  }
+}
+
+cudaError_t launch_fwd_merge(const float* o_part, const float* lse_part, void* o, float* lse, int nsplit,
+                             long long rows, int d, cudaStream_t stream) {
+  long long blocks = (rows + 7) / 8;
+  if (blocks > 148LL * 16) blocks = 148LL * 16;
+  if (blocks < 1) blocks = 1;
+  auto* out = reinterpret_cast<__nv_bfloat16*>(o);
+  if (d == 64)
+    fa_fwd_merge_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(o_part, lse_part, out, lse, nsplit, rows);
+  else
+    fa_fwd_merge_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(o_part, lse_part, out, lse, nsplit, rows);
+  return cudaGetLastError();
 }
 
 }  // namespace fa

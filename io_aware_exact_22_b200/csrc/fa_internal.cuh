@@ -9,12 +9,13 @@ namespace fa {
 
 struct FwdArgs {
   uint32_t* status;  // device status word
-  float* lse;        // [BH, N] fp32
+  float* lse;        // [BH, N] fp32; with key splits: [nsplit, BH, N] partial LSEs
   int N;             // sequence length
   int BH;            // batch * heads
   int nqb;           // query blocks of 256 rows per head
   int causal;        // 0 / 1
   float scale_log2;  // scale * log2(e)
+  int nsplit;        // key-range splits per (head, query block); 1 = whole key range
 };
 
 struct BwdArgs {
@@ -44,13 +45,19 @@ cudaError_t launch_wait_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t 
 // Tensor maps for a bf16 [BH, N, d] tensor, 128-byte swizzle, box = 64 columns x `rows`.
 bool make_tmap_bf16(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_rows);
 
+// With a.nsplit == 1, `to` maps the bf16 output; with a.nsplit > 1 it maps the fp32 partial
+// outputs [nsplit * BH, N, d] (box 32 x 32, 128-byte swizzle) and a.lse the partial LSEs.
 cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& to, const FwdArgs& a, cudaStream_t stream);
+// Combines nsplit partial (O_s, LSE_s) into bf16 O and fp32 LSE.
+cudaError_t launch_fwd_merge(const float* o_part, const float* lse_part, void* o, float* lse, int nsplit,
+                             long long rows, int d, cudaStream_t stream);
 
 cudaError_t launch_bwd_pre(const void* o, const void* dO, const float* lse, float* ld, float* dq_acc,
                            int BH, int N, int d, cudaStream_t stream);
 // fp32 [BH, N, d] tensor map without swizzle, box = box_inner columns x box_rows rows.
-bool make_tmap_f32(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_inner, int box_rows);
+bool make_tmap_f32(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_inner, int box_rows,
+                   bool swizzle128 = false);
 
 cudaError_t launch_bwd_main(int d, const CUtensorMap& tq, const CUtensorMap& tk,
                             const CUtensorMap& tv, const CUtensorMap& tdo,

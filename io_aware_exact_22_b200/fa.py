@@ -22,7 +22,8 @@ LIB_PATH = os.environ.get("FA_LIB_PATH", os.path.join(_HERE, "libfa.so"))
 STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_CUDA",
           4: "FA_ERR_TIMEOUT"}
 EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_device_status",
-           "fa_status_string", "fa_version", "fa_bwd_noalloc", "fa_selftest_wait_timeout")
+           "fa_status_string", "fa_version", "fa_bwd_noalloc", "fa_selftest_wait_timeout",
+           "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_default_splits")
 # Size of the library's built-in scratch used by fa_bwd_noalloc (include/fa.h).
 NOALLOC_MAX_SCRATCH_BYTES = 64 << 20
 
@@ -60,6 +61,12 @@ def lib() -> ctypes.CDLL:
         L.fa_bwd_noalloc.restype = i
         L.fa_selftest_wait_timeout.argtypes = [i, vp]
         L.fa_selftest_wait_timeout.restype = i
+        L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp, sz, vp]
+        L.fa_fwd_splitkv.restype = i
+        L.fa_fwd_splitkv_workspace_bytes.argtypes = [i, i, i, i, i]
+        L.fa_fwd_splitkv_workspace_bytes.restype = sz
+        L.fa_fwd_splitkv_default_splits.argtypes = [i, i, i, i, i]
+        L.fa_fwd_splitkv_default_splits.restype = i
         _lib = L
     return _lib
 
@@ -84,6 +91,21 @@ def _stream(stream):
 def fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, stream=None) -> int:
     return lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
                         float(scale), int(causal), _stream(stream))
+
+
+def fa_fwd_splitkv(q, k, v, o, lse, B, H, N, d, scale, causal, num_splits, workspace,
+                   workspace_bytes, stream=None) -> int:
+    return lib().fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                                float(scale), int(causal), int(num_splits), _ptr(workspace),
+                                int(workspace_bytes), _stream(stream))
+
+
+def fa_fwd_splitkv_workspace_bytes(B, H, N, d, num_splits) -> int:
+    return lib().fa_fwd_splitkv_workspace_bytes(B, H, N, d, num_splits)
+
+
+def fa_fwd_splitkv_default_splits(B, H, N, d, causal) -> int:
+    return lib().fa_fwd_splitkv_default_splits(B, H, N, d, int(causal))
 
 
 def fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes, B, H, N, d, scale,
@@ -141,6 +163,29 @@ def forward(q, k, v, causal: bool, scale: float | None = None, out=None, lse=Non
     rc = fa_fwd(q, k, v, out, lse, B, H, N, d, scale, causal)
     if rc:
         raise FAError(rc, "fa_fwd")
+    return out, lse
+
+
+def forward_splitkv(q, k, v, causal: bool, scale: float | None = None, num_splits: int = 0,
+                    out=None, lse=None, workspace=None):
+    """Split-KV forward (fa_fwd_splitkv); the workspace is allocated with torch if not given."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n)
+    B, H, N, d = q.shape
+    scale = d ** -0.5 if scale is None else scale
+    sp = num_splits if num_splits > 0 else fa_fwd_splitkv_default_splits(B, H, N, d, causal)
+    sp = max(1, min(sp, (N + 127) // 128))
+    nbytes = fa_fwd_splitkv_workspace_bytes(B, H, N, d, sp)
+    if workspace is None and nbytes > 0:
+        workspace = torch.empty(nbytes, device=q.device, dtype=torch.uint8)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+    rc = fa_fwd_splitkv(q, k, v, out, lse, B, H, N, d, scale, causal, sp, workspace,
+                        0 if workspace is None else workspace.numel())
+    if rc:
+        raise FAError(rc, "fa_fwd_splitkv")
     return out, lse
 
 

@@ -1,0 +1,95 @@
+"""Split-KV forward (fa_fwd_splitkv): partial results over key ranges combined by the two-block
+softmax merge ("Flash Attention", special-jiahao.github.io, section 增量求解 softmax), checked
+against the fp64 oracle and against the unsplit forward."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from io_aware_exact_22_b200 import fa
+from io_aware_exact_22_b200.inputs import WORKLOADS, custom, make_inputs, to_f64
+from tests._helpers import check_lse, check_o, f64
+
+A16 = 0x10000
+OK, INVALID = 0, 1
+
+
+def test_workspace_size():
+    B, H, N, d, sp = 1, 3, 1000, 128, 4
+    rows = B * H * N
+    want = ((sp * rows * d * 4 + 255) // 256) * 256 + sp * rows * 4
+    assert fa.fa_fwd_splitkv_workspace_bytes(B, H, N, d, sp) == want
+    assert fa.fa_fwd_splitkv_workspace_bytes(B, H, N, d, 1) == 0
+    assert fa.fa_fwd_splitkv_workspace_bytes(0, H, N, d, 4) == 0
+
+
+@pytest.mark.parametrize("kw", [dict(ws=0), dict(ws=A16 + 16), dict(wsb=100), dict(q=0),
+                                dict(scale=0.0), dict(causal=2)])
+def test_rejects_bad_arguments(kw):
+    args = dict(q=A16, k=A16, v=A16, o=A16, lse=A16, B=1, H=1, N=1024, d=128, scale=0.1, causal=1,
+                sp=4, ws=A16, wsb=1 << 40)
+    args.update(kw)
+    rc = fa.fa_fwd_splitkv(args["q"], args["k"], args["v"], args["o"], args["lse"], args["B"],
+                           args["H"], args["N"], args["d"], args["scale"], args["causal"],
+                           args["sp"], args["ws"], args["wsb"], 0)
+    assert rc == INVALID
+
+
+def test_empty_problem_is_a_no_op():
+    assert fa.fa_fwd_splitkv(A16, A16, A16, A16, A16, 1, 0, 100, 64, 0.1, 0, 4, 0, 0, 0) == OK
+
+
+def _check(w, splits, inputs=None):
+    q, k, v = inputs if inputs is not None else make_inputs(w, with_grad=False)[:3]
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    o, lse = fa.forward_splitkv(qd, kd, vd, w.causal, w.scale, num_splits=splits)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status() == 0
+    o_ref, lse_ref = oracle.attention_forward(to_f64(q), to_f64(k), to_f64(v), w.scale, w.causal)
+    check_o(f64(o), o_ref)
+    check_lse(f64(lse), lse_ref)
+    return (qd, kd, vd), o, lse
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("splits", [2, 3, 4])
+def test_single_head_workload(cuda_ok, splits):
+    _check(WORKLOADS[1], splits)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("B,H,N,d,causal,splits", [
+    (1, 2, 1000, 128, True, 3), (1, 1, 2048, 64, False, 16), (2, 1, 700, 128, False, 5),
+    (1, 2, 513, 64, True, 4), (1, 1, 300, 128, True, 8), (1, 3, 4096, 128, True, 32),
+    (1, 1, 129, 64, False, 2), (1, 2, 1, 128, True, 4)])
+def test_ragged_and_causal(cuda_ok, B, H, N, d, causal, splits):
+    # causal query blocks near the start have fewer key blocks than splits: some splits are empty
+    _check(custom(B, H, N, d, causal, seed=N + splits), splits)
+
+
+@pytest.mark.gpu
+def test_large_scores(cuda_ok):
+    _check(custom(1, 2, 2048, 128, True, seed=5, qk_std=math.sqrt(3.0)), 6)
+
+
+@pytest.mark.gpu
+def test_matches_unsplit_forward_and_default_choice(cuda_ok):
+    w = custom(1, 4, 1536, 128, True, seed=19)
+    (q, k, v), o_s, l_s = _check(w, 0)  # default number of splits
+    o_u, l_u = fa.forward(q, k, v, True, w.scale)
+    torch.cuda.synchronize()
+    assert (o_s.float() - o_u.float()).abs().max().item() <= 1.6e-2
+    assert (l_s - l_u).abs().max().item() <= 1e-4
+    assert fa.fa_fwd_splitkv_default_splits(1, 4, 1536, 128, 1) > 1
+
+
+@pytest.mark.gpu
+def test_one_split_is_the_plain_forward(cuda_ok):
+    w = custom(1, 2, 640, 64, False, seed=4)
+    q, k, v = (t.cuda() for t in make_inputs(w, with_grad=False))
+    o1, l1 = fa.forward_splitkv(q, k, v, False, w.scale, num_splits=1)
+    o2, l2 = fa.forward(q, k, v, False, w.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
