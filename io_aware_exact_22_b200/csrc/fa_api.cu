@@ -10,7 +10,9 @@
 #include <climits>
 #include <cmath>
 #include <cstdint>
+#include <functional>
 #include <mutex>
+#include <unordered_map>
 
 namespace fa {
 
@@ -87,7 +89,51 @@ size_t ld_bytes(long long bh, int N) {
 
 }  // namespace
 
+// Tensor maps depend only on (address, shape, box, element type, swizzle), so encoded maps are
+// cached under that key: a map found here is exactly what encoding again would produce.
+namespace {
+struct TmapKey {
+  uintptr_t ptr;
+  int BH, N, d, box_inner, box_rows, kind;
+  bool operator==(const TmapKey& o) const {
+    return ptr == o.ptr && BH == o.BH && N == o.N && d == o.d && box_inner == o.box_inner &&
+           box_rows == o.box_rows && kind == o.kind;
+  }
+};
+struct TmapKeyHash {
+  size_t operator()(const TmapKey& k) const {
+    size_t h = std::hash<uintptr_t>()(k.ptr);
+    for (int v : {k.BH, k.N, k.d, k.box_inner, k.box_rows, k.kind}) h = h * 1000003u ^ std::hash<int>()(v);
+    return h;
+  }
+};
+std::mutex g_tmap_mu;
+std::unordered_map<TmapKey, CUtensorMap, TmapKeyHash> g_tmap_cache;
+
+template <class F>
+bool cached_tmap(CUtensorMap* m, const TmapKey& key, F&& encode) {
+  {
+    std::lock_guard<std::mutex> lock(g_tmap_mu);
+    auto it = g_tmap_cache.find(key);
+    if (it != g_tmap_cache.end()) {
+      *m = it->second;
+      return true;
+    }
+  }
+  if (!encode(m)) return false;
+  std::lock_guard<std::mutex> lock(g_tmap_mu);
+  if (g_tmap_cache.size() >= 4096) g_tmap_cache.clear();
+  g_tmap_cache.emplace(key, *m);
+  return true;
+}
+}  // namespace
+
 bool make_tmap_bf16(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_rows) {
+  return cached_tmap(m, TmapKey{reinterpret_cast<uintptr_t>(ptr), BH, N, d, 64, box_rows, 0},
+                     [&](CUtensorMap* out) { return encode_tmap_bf16(out, ptr, BH, N, d, box_rows); });
+}
+
+bool encode_tmap_bf16(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_rows) {
   auto enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
@@ -122,6 +168,15 @@ cudaError_t launch_wait_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t 
 
 bool make_tmap_f32(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_inner, int box_rows,
                    bool swizzle128) {
+  return cached_tmap(m,
+                     TmapKey{reinterpret_cast<uintptr_t>(ptr), BH, N, d, box_inner, box_rows, swizzle128 ? 2 : 1},
+                     [&](CUtensorMap* out) {
+                       return encode_tmap_f32(out, ptr, BH, N, d, box_inner, box_rows, swizzle128);
+                     });
+}
+
+bool encode_tmap_f32(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_inner, int box_rows,
+                     bool swizzle128) {
   auto enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
@@ -192,13 +247,15 @@ int fa_fwd_splitkv_default_splits(int B, int H, int N, int d, int causal) {
     int v = 0;
     if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) nsm = v;
   }
+  // Splitting pays only when few work items leave most SMs idle and every split still has
+  // several key blocks to amortise its partial-output traffic and the merge.
   const long long items = (long long)B * H * ((N + 255) / 256);
-  if (items >= nsm) return 1;
-  long long sp = (nsm + items - 1) / items;
+  if (4 * items > nsm) return 1;
+  long long sp = nsm / items;
   const long long kblocks = (N + 127) / 128;
-  if (sp > kblocks) sp = kblocks;
+  if (sp > kblocks / 4) sp = kblocks / 4;
   if (sp > 32) sp = 32;
-  return sp < 1 ? 1 : (int)sp;
+  return sp < 2 ? 1 : (int)sp;
 }
 
 static size_t splitkv_o_bytes(long long rows, int d, int sp) {

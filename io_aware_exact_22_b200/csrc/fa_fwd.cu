@@ -451,9 +451,15 @@ static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, co
   using C = FwdCfg<D>;
   static_assert(C::SMEM <= 232448, "shared memory budget");
   static_assert(2 * 128 * D * 4 <= C::NS * C::TILE, "partial-output staging must fit the K/V ring");
-  cudaError_t e =
-      cudaFuncSetAttribute(fa_fwd_kernel<D, PARTIAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  static bool attr_set[64];  // per device: the attribute outlives the call
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(fa_fwd_kernel<D, PARTIAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
   const long long grid = (long long)a.BH * a.nqb * a.nsplit;
   fa_fwd_kernel<D, PARTIAL><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, to, a);
   return cudaGetLastError();

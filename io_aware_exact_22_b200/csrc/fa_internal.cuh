@@ -42,8 +42,12 @@ uint32_t* device_status_word();
 // Launches the bounded-wait self-test kernel (see fa_selftest_wait_timeout).
 cudaError_t launch_wait_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);
 
-// Tensor maps for a bf16 [BH, N, d] tensor, 128-byte swizzle, box = 64 columns x `rows`.
+// Tensor maps for a bf16 [BH, N, d] tensor, 128-byte swizzle, box = 64 columns x `rows`
+// (make_*: served from a cache of encoded maps; encode_*: always encodes).
 bool make_tmap_bf16(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_rows);
+bool encode_tmap_bf16(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_rows);
+bool encode_tmap_f32(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_inner, int box_rows,
+                     bool swizzle128);
 
 // With a.nsplit == 1, `to` maps the bf16 output; with a.nsplit > 1 it maps the fp32 partial
 // outputs [nsplit * BH, N, d] (box 32 x 32, 128-byte swizzle) and a.lse the partial LSEs.
