@@ -144,6 +144,18 @@ fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const vo
                            int B, int H, int N, int d, float scale, int causal, void* stream);
 
 /*
+ * fa_bwd with a deterministic dQ: same arguments, workspace and results (within rounding), but
+ * dQ is accumulated per 128-row query tile in a fixed order (a query-tile-outer pass that
+ * recomputes S and dP and keeps dQ on chip until it is written once) instead of with
+ * floating-point atomics, so repeated calls on the same inputs give bitwise-identical dQ, dK
+ * and dV.  Supported: d == 128.
+ */
+fa_status_t fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
+                                 const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                                 void* workspace, size_t workspace_bytes,
+                                 int B, int H, int N, int d, float scale, int causal, void* stream);
+
+/*
  * Synchronises `stream`, reads and clears the device status word of the current device.
  * Returns FA_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call,
  * FA_ERR_CUDA if the synchronisation itself failed, FA_OK otherwise.

@@ -358,6 +358,50 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
   return FA_OK;
 }
 
+fa_status_t fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                                 const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                                 size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
+                                 void* stream) {
+  bool empty = false;
+  fa_status_t st = check_shape(B, H, N, d, scale, causal, &empty);
+  if (st != FA_OK || empty) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dO, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) || !aligned(workspace, 256))
+    return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  if ((st = check_device()) != FA_OK) return st;
+  const int BH = B * H;
+  float* ld = reinterpret_cast<float*>(workspace);
+  cudaStream_t s = (cudaStream_t)stream;
+  // main kernel (dK, dV): Q/dO in 64-row boxes, K/V in 128-row boxes
+  CUtensorMap tq64, tk128, tv128, tdo64, tdk, tdv;
+  // dQ kernel: Q/dO in 128-row boxes, K/V in 64-row boxes, dQ stored in 32-row boxes
+  CUtensorMap tq128, tk64, tv64, tdo128, tdq;
+  if (!make_tmap_bf16(&tq64, q, BH, N, d, 64) || !make_tmap_bf16(&tk128, k, BH, N, d, 128) ||
+      !make_tmap_bf16(&tv128, v, BH, N, d, 128) || !make_tmap_bf16(&tdo64, dO, BH, N, d, 64) ||
+      !make_tmap_bf16(&tdk, dk, BH, N, d, 32) || !make_tmap_bf16(&tdv, dv, BH, N, d, 32) ||
+      !make_tmap_bf16(&tq128, q, BH, N, d, 128) || !make_tmap_bf16(&tk64, k, BH, N, d, 64) ||
+      !make_tmap_bf16(&tv64, v, BH, N, d, 64) || !make_tmap_bf16(&tdo128, dO, BH, N, d, 128) ||
+      !make_tmap_bf16(&tdq, dq, BH, N, d, 32))
+    return FA_ERR_CUDA;
+  BwdArgs a;
+  if (!(a.status = device_status_word())) return FA_ERR_CUDA;
+  a.lse = lse;
+  a.ld = ld;
+  a.dq_acc = nullptr;
+  a.N = N;
+  a.BH = BH;
+  a.causal = causal;
+  a.scale = scale;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  if (launch_bwd_pre(o, dO, lse, ld, nullptr, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (launch_bwd_main(d, tq64, tk128, tv128, tdo64, tdk, tdv, tdk, a, s, false) != cudaSuccess) return FA_ERR_CUDA;
+  if (launch_bwd_dq(d, tq128, tk64, tv64, tdo128, tdq, a, s) != cudaSuccess) return FA_ERR_CUDA;
+  return FA_OK;
+}
+
 fa_status_t fa_selftest_wait_timeout(int limit_ms, void* stream) {
   if (limit_ms < 1 || limit_ms > 1000) return FA_ERR_INVALID_ARG;
   uint32_t* status = device_status_word();

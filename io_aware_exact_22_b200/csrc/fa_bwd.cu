@@ -39,12 +39,14 @@ constexpr float kLog2e = 1.4426950408889634074f;
 }
 
 // ------------------------------------------------------------------ K2
+template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dO,
                                                          const float* __restrict__ lse,
                                                          float* __restrict__ ld,
                                                          float* __restrict__ dq_acc, int BH, int N,
                                                          int Tq) {
+  constexpr int V = D / 32;  // columns per lane
   const int lane = threadIdx.x & 31;
   const long long total = (long long)BH * Tq * 64;
   const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
@@ -53,19 +55,30 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
     const int qp = (int)(row % ((long long)Tq * 64));
     float dsum = 0.f, l2 = INFINITY;
     if (qp < N) {
-      const size_t base = ((size_t)bh * N + qp) * 128 + lane * 4;
-      const uint2 ov = *reinterpret_cast<const uint2*>(o + base);
-      const uint2 gv = *reinterpret_cast<const uint2*>(dO + base);
-      const float2 o01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ov.x));
-      const float2 o23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ov.y));
-      const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv.x));
-      const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv.y));
-      dsum = o01.x * g01.x + o01.y * g01.y + o23.x * g23.x + o23.y * g23.y;
+      const size_t base = ((size_t)bh * N + qp) * D + lane * V;
+      if (V == 4) {
+        const uint2 ov = *reinterpret_cast<const uint2*>(o + base);
+        const uint2 gv = *reinterpret_cast<const uint2*>(dO + base);
+        const float2 o01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ov.x));
+        const float2 o23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ov.y));
+        const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv.x));
+        const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv.y));
+        dsum = o01.x * g01.x + o01.y * g01.y + o23.x * g23.x + o23.y * g23.y;
+      } else {
+        const float2 o01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(o + base));
+        const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dO + base));
+        dsum = o01.x * g01.x + o01.y * g01.y;
+      }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
       const float L = lse[(size_t)bh * N + qp];
       l2 = (L == -INFINITY) ? INFINITY : L * kLog2e;  // a row with no visible key gets P = 0
-      *reinterpret_cast<float4*>(dq_acc + base) = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (dq_acc) {
+        if (V == 4)
+          *reinterpret_cast<float4*>(dq_acc + base) = make_float4(0.f, 0.f, 0.f, 0.f);
+        else
+          *reinterpret_cast<float2*>(dq_acc + base) = make_float2(0.f, 0.f);
+      }
     }
     if (lane == 0) {
       float* t = ld + ((size_t)bh * Tq + (qp >> 6)) * 128;
@@ -130,6 +143,9 @@ struct BwdCfg {
 // Each compute warpgroup writes its packed P^T (and dS^T) inside its own S^T (dP^T) columns,
 // so neither overwrites scores the other has not read yet: P^T of query columns [32g, 32g+32)
 // sits at TMEM columns [32g, 32g+16), dS^T at [64+32g, 64+32g+16).
+// WITH_DQ = false: dK and dV only (dQ comes from fa_bwd_dq_kernel): no dQ^T MMA, no dS^T in
+// shared memory, no drain.
+template <bool WITH_DQ>
 __global__ void __launch_bounds__(448, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -301,14 +317,16 @@ __global__ void __launch_bounds__(448, 1)
         for (int k = 0; k < 4; ++k)  // dK += dS^T Q_i
           mma_ts_e(tmem + C::T_DK, tmem + C::T_DP + 32 * (k >> 1) + 8 * (k & 1), sdesc_add(dQ_mn, so + k * 2048),
                    C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(dq_free(b), ((n >> 1) & 1) ^ 1, wc)))) break;
-        tc_fence_after();
+        if (WITH_DQ) {
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(dq_free(b), ((n >> 1) & 1) ^ 1, wc)))) break;
+          tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < 8; ++k)  // dQ_i^T = K_j^T dS^T  (K over the 128 keys)
-          mma_ss_e(tmem + C::T_DQ + 64 * b, sdesc_add(dK_mn, k * 2048), sdesc_add(dS_mn, b * C::DS_BYTES + k * 2048),
-                   C::IDESC_Q, k > 0);
-        mma_commit_e(dq_full(b));
-        mma_commit_e(ds_free(b));
+          for (int k = 0; k < 8; ++k)  // dQ_i^T = K_j^T dS^T  (K over the 128 keys)
+            mma_ss_e(tmem + C::T_DQ + 64 * b, sdesc_add(dK_mn, k * 2048),
+                     sdesc_add(dS_mn, b * C::DS_BYTES + k * 2048), C::IDESC_Q, k > 0);
+          mma_commit_e(dq_full(b));
+          mma_commit_e(ds_free(b));
+        }
         mma_commit_e(qd_empty(s));
         if (more) issue_dp(n + 1);
       }
@@ -385,17 +403,19 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
       for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(p[2 * c], p[2 * c + 1]);
       tmem_st16(tDP, pk);
-      // dS^T row r, query columns [32 g, 32 g + 32), into the shared buffer read by the dQ MMA
-      ok = __all_sync(0xffffffffu, mbar_wait(ds_free(b), ((n >> 1) & 1) ^ 1, wc));
-      if (!ok) break;
-      uint8_t* dsrow = gb + C::DS_OFF + b * C::DS_BYTES + r * 128;
+      if (WITH_DQ) {
+        // dS^T row r, query columns [32 g, 32 g + 32), into the shared buffer read by the dQ MMA
+        ok = __all_sync(0xffffffffu, mbar_wait(ds_free(b), ((n >> 1) & 1) ^ 1, wc));
+        if (!ok) break;
+        uint8_t* dsrow = gb + C::DS_OFF + b * C::DS_BYTES + r * 128;
 #pragma unroll
-      for (int c16 = 0; c16 < 4; ++c16) {
-        const int chunk = 4 * g + c16;
-        *reinterpret_cast<uint4*>(dsrow + ((chunk ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
+        for (int c16 = 0; c16 < 4; ++c16) {
+          const int chunk = 4 * g + c16;
+          *reinterpret_cast<uint4*>(dsrow + ((chunk ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
+        }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(ds_ready);
@@ -407,7 +427,7 @@ __global__ void __launch_bounds__(448, 1)
     float* stage = reinterpret_cast<float*>(gb + C::DQS_OFF + wq * C::DQS_WARP);
     const uint32_t stage_s = sb + C::DQS_OFF + wq * C::DQS_WARP;
     bool ok = !*abort_flag;
-    for (int n = 0; n < count && ok; ++n) {
+    for (int n = 0; n < (WITH_DQ ? count : 0) && ok; ++n) {
       const int b = n & 1;
       const int i = i0 + n;
       ok = __all_sync(0xffffffffu, mbar_wait(dq_full(b), (n >> 1) & 1, wc));
@@ -515,19 +535,21 @@ static int grid_for(long long work, int per_block) {
 
 cudaError_t launch_bwd_pre(const void* o, const void* dO, const float* lse, float* ld, float* dq_acc,
                            int BH, int N, int d, cudaStream_t stream) {
-  if (d != 128) return cudaErrorNotSupported;
   const int Tq = (N + 63) / 64;
   const long long rows = (long long)BH * Tq * 64;
-  fa_bwd_pre_kernel<<<grid_for(rows, 8), 256, 0, stream>>>(
-      reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(dO), lse, ld,
-      dq_acc, BH, N, Tq);
+  auto* po = reinterpret_cast<const __nv_bfloat16*>(o);
+  auto* pg = reinterpret_cast<const __nv_bfloat16*>(dO);
+  if (d == 64)
+    fa_bwd_pre_kernel<64><<<grid_for(rows, 8), 256, 0, stream>>>(po, pg, lse, ld, dq_acc, BH, N, Tq);
+  else
+    fa_bwd_pre_kernel<128><<<grid_for(rows, 8), 256, 0, stream>>>(po, pg, lse, ld, dq_acc, BH, N, Tq);
   return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_main(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
-                            const CUtensorMap& tdq, const BwdArgs& a, cudaStream_t stream) {
-  if (d != 128) return cudaErrorNotSupported;
+template <bool WITH_DQ>
+static cudaError_t launch_bwd_main_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                     const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
+                                     const CUtensorMap& tdq, const BwdArgs& a, cudaStream_t stream) {
   using C = BwdCfg;
   static_assert(C::SMEM <= 232448, "shared memory budget");
   static bool attr_set[64];  // per device: the attribute outlives the call
@@ -535,16 +557,24 @@ cudaError_t launch_bwd_main(int d, const CUtensorMap& tq, const CUtensorMap& tk,
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(fa_bwd_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    e = cudaFuncSetAttribute(fa_bwd_main_kernel<WITH_DQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   const int Tk = (a.N + 127) / 128;
   const int Tq = (a.N + 63) / 64;
   const long long grid = (long long)a.BH * Tk;
-  fa_bwd_main_kernel<<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, tdo, tdk, tdv, tdq, a, Tk,
-                                                                        Tq);
+  fa_bwd_main_kernel<WITH_DQ><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, tdo, tdk, tdv, tdq, a,
+                                                                                 Tk, Tq);
   return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_main(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
+                            const CUtensorMap& tdq, const BwdArgs& a, cudaStream_t stream, bool with_dq) {
+  if (d != 128) return cudaErrorNotSupported;
+  return with_dq ? launch_bwd_main_t<true>(tq, tk, tv, tdo, tdk, tdv, tdq, a, stream)
+                 : launch_bwd_main_t<false>(tq, tk, tv, tdo, tdk, tdv, tdq, a, stream);
 }
 
 cudaError_t launch_bwd_post(const float* dq_acc, void* dq, long long elems, float scale, cudaStream_t stream) {

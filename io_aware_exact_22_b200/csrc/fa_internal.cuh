@@ -63,10 +63,17 @@ cudaError_t launch_bwd_pre(const void* o, const void* dO, const float* lse, floa
 bool make_tmap_f32(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_inner, int box_rows,
                    bool swizzle128 = false);
 
+// with_dq = false: dK and dV only (no dQ accumulation; tdq and a.dq_acc unused).
 cudaError_t launch_bwd_main(int d, const CUtensorMap& tq, const CUtensorMap& tk,
                             const CUtensorMap& tv, const CUtensorMap& tdo,
                             const CUtensorMap& tdk, const CUtensorMap& tdv,
-                            const CUtensorMap& tdq, const BwdArgs& a, cudaStream_t stream);
+                            const CUtensorMap& tdq, const BwdArgs& a, cudaStream_t stream,
+                            bool with_dq = true);
+// Deterministic dQ (query-tile-outer, accumulated in TMEM, written once): tq/tdo with 128-row
+// boxes, tk/tv with 64-row boxes, tdq the bf16 dQ with 32-row boxes; needs a.ld filled.
+cudaError_t launch_bwd_dq(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a,
+                          cudaStream_t stream);
 cudaError_t launch_bwd_post(const float* dq_acc, void* dq, long long elems, float scale,
                             cudaStream_t stream);
 

@@ -23,7 +23,8 @@ STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_E
           4: "FA_ERR_TIMEOUT"}
 EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_device_status",
            "fa_status_string", "fa_version", "fa_bwd_noalloc", "fa_selftest_wait_timeout",
-           "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_default_splits")
+           "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_default_splits",
+           "fa_bwd_deterministic")
 # Size of the library's built-in scratch used by fa_bwd_noalloc (include/fa.h).
 NOALLOC_MAX_SCRATCH_BYTES = 64 << 20
 
@@ -67,6 +68,8 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd_splitkv_workspace_bytes.restype = sz
         L.fa_fwd_splitkv_default_splits.argtypes = [i, i, i, i, i]
         L.fa_fwd_splitkv_default_splits.restype = i
+        L.fa_bwd_deterministic.argtypes = L.fa_bwd.argtypes
+        L.fa_bwd_deterministic.restype = i
         _lib = L
     return _lib
 
@@ -113,6 +116,14 @@ def fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes, B, H, N,
     return lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq),
                         _ptr(dk), _ptr(dv), _ptr(workspace), int(workspace_bytes), B, H, N, d,
                         float(scale), int(causal), _stream(stream))
+
+
+def fa_bwd_deterministic(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes, B, H, N, d,
+                         scale, causal, stream=None) -> int:
+    return lib().fa_bwd_deterministic(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse),
+                                      _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+                                      int(workspace_bytes), B, H, N, d, float(scale), int(causal),
+                                      _stream(stream))
 
 
 def fa_bwd_noalloc(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal,
@@ -190,8 +201,9 @@ def forward_splitkv(q, k, v, causal: bool, scale: float | None = None, num_split
 
 
 def backward(q, k, v, o, do, lse, causal: bool, scale: float | None = None, workspace=None,
-             dq=None, dk=None, dv=None):
-    """dQ, dK, dV through fa_bwd (workspace allocated with torch when not given)."""
+             dq=None, dk=None, dv=None, deterministic: bool = False):
+    """dQ, dK, dV through fa_bwd, or fa_bwd_deterministic (workspace allocated with torch when
+    not given)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "dO")):
         _check(t, n)
     B, H, N, d = q.shape
@@ -202,8 +214,8 @@ def backward(q, k, v, o, do, lse, causal: bool, scale: float | None = None, work
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    rc = fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, workspace.numel(), B, H, N, d, scale,
-                causal)
+    fn = fa_bwd_deterministic if deterministic else fa_bwd
+    rc = fn(q, k, v, o, do, lse, dq, dk, dv, workspace, workspace.numel(), B, H, N, d, scale, causal)
     if rc:
-        raise FAError(rc, "fa_bwd")
+        raise FAError(rc, fn.__name__)
     return dq, dk, dv
