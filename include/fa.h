@@ -21,7 +21,7 @@
  *
  * Layout.  Q, K, V, O, dO, dQ, dK, dV are bf16 tensors [B, H, N, d], contiguous
  * (row-major: d fastest, then N, then H, then B).  LSE is fp32 [B, H, N], contiguous.
- * Supported: d in {64, 128} for the forward, d == 128 for the backward; N >= 0;
+ * Supported: d in {64, 128} for the forward and the backward; N >= 0;
  * B * H * N * d < 2^62.  B, H or N equal to 0 is an empty problem: the call returns FA_OK
  * without launching anything.
  *
@@ -109,6 +109,8 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
  *   workspace      : device scratch of at least fa_bwd_workspace_bytes(B,H,N,d) bytes,
  *                    256-byte aligned; its contents on entry do not matter and on exit
  *                    are unspecified.  Concurrent calls need distinct workspaces.
+ * At d == 128, dQ is summed over key tiles with fp32 atomics (dK, dV in a fixed order); at
+ * d == 64 the call runs fa_bwd_deterministic's two passes.
  */
 fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o,
                    const void* dO, const float* lse, void* dq, void* dk, void* dv,
@@ -148,7 +150,7 @@ fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const vo
  * dQ is accumulated per 128-row query tile in a fixed order (a query-tile-outer pass that
  * recomputes S and dP and keeps dQ on chip until it is written once) instead of with
  * floating-point atomics, so repeated calls on the same inputs give bitwise-identical dQ, dK
- * and dV.  Supported: d == 128.
+ * and dV.  Supported: d in {64, 128}.
  */
 fa_status_t fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
                                  const void* dO, const float* lse, void* dq, void* dk, void* dv,

@@ -321,6 +321,10 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
   bool empty = false;
   fa_status_t st = check_shape(B, H, N, d, scale, causal, &empty);
   if (st != FA_OK || empty) return st;
+  // d = 64: the key pass has no atomic dQ path there, so dQ comes from the query pass
+  if (d == 64)
+    return fa_bwd_deterministic(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes, B, H, N, d, scale,
+                                causal, stream);
   if (d != 128) return FA_ERR_UNSUPPORTED;
   if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dO, 16) ||
@@ -365,7 +369,6 @@ fa_status_t fa_bwd_deterministic(const void* q, const void* k, const void* v, co
   bool empty = false;
   fa_status_t st = check_shape(B, H, N, d, scale, causal, &empty);
   if (st != FA_OK || empty) return st;
-  if (d != 128) return FA_ERR_UNSUPPORTED;
   if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dO, 16) ||
       !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) || !aligned(workspace, 256))

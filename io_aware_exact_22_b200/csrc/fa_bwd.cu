@@ -103,8 +103,10 @@ __global__ void __launch_bounds__(256) fa_bwd_post_kernel(const float4* __restri
 }
 
 // ------------------------------------------------------------------ K3
+template <int D_>
 struct BwdCfg {
-  static constexpr int D = 128;
+  static constexpr int D = D_;
+  static constexpr int NBOX = D / 64;       // 64-column (128-byte) swizzle boxes per row
   static constexpr int BQ = 64;             // query rows per step
   static constexpr int NSQ = 3;             // Q/dO ring stages
   static constexpr int KT = 128 * D * 2;    // bytes of K_j (or V_j)
@@ -144,15 +146,18 @@ struct BwdCfg {
 // so neither overwrites scores the other has not read yet: P^T of query columns [32g, 32g+32)
 // sits at TMEM columns [32g, 32g+16), dS^T at [64+32g, 64+32g+16).
 // WITH_DQ = false: dK and dV only (dQ comes from fa_bwd_dq_kernel): no dQ^T MMA, no dS^T in
-// shared memory, no drain.
-template <bool WITH_DQ>
+// shared memory, no drain.  The dQ^T MMA puts d on the M dimension (128 TMEM lanes), so the
+// atomic dQ path exists for D = 128 only; D = 64 always runs with WITH_DQ = false.
+template <int D, bool WITH_DQ>
 __global__ void __launch_bounds__(448, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                        const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
                        const __grid_constant__ CUtensorMap tmdQ, const BwdArgs a, const int Tk,
                        const int Tq) {
-  using C = BwdCfg;
+  static_assert(D == 64 || D == 128, "head dimension");
+  static_assert(!WITH_DQ || D == 128, "the dQ^T MMA needs M = d = 128");
+  using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
@@ -224,7 +229,7 @@ __global__ void __launch_bounds__(448, 1)
       const uint64_t keep = policy_evict_last();
       const uint64_t once = policy_evict_first();
       mbar_arrive_expect_tx_e(kv_full, 2 * C::KT);
-      for (int b = 0; b < 2; ++b) {
+      for (int b = 0; b < C::NBOX; ++b) {
         tma_load_3d_e(sb + C::K_OFF + b * 16384, &tmK, kv_full, 64 * b, 128 * j, bh, once);
         tma_load_3d_e(sb + C::V_OFF + b * 16384, &tmV, kv_full, 64 * b, 128 * j, bh, once);
       }
@@ -235,7 +240,7 @@ __global__ void __launch_bounds__(448, 1)
         if (!__all_sync(0xffffffffu, mbar_wait(qd_empty(s), ((n / C::NSQ) & 1) ^ 1, wc))) break;
         mbar_arrive_expect_tx_e(qd_full(s), 2 * C::QT + C::LDB);
         const uint32_t st = sb + C::ST_OFF + s * C::ST_BYTES;
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < C::NBOX; ++b) {
           tma_load_3d_e(st + b * 8192, &tmQ, qd_full(s), 64 * b, C::BQ * i, bh, keep);
           tma_load_3d_e(st + C::QT + b * 8192, &tmdO, qd_full(s), 64 * b, C::BQ * i, bh, keep);
         }
@@ -271,7 +276,7 @@ __global__ void __launch_bounds__(448, 1)
       auto issue_s = [&](int n) {  // S^T = K_j Q_i^T  (K over d)
         const uint32_t so = st_off(n);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < D / 16; ++k) {
           const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32, qo = (k >> 2) * 8192 + (k & 3) * 32;
           mma_ss_e(tmem + C::T_S, sdesc_add(dK_k, ko), sdesc_add(dQ_k, so + qo), C::IDESC_S, k > 0);
         }
@@ -280,7 +285,7 @@ __global__ void __launch_bounds__(448, 1)
       auto issue_dp = [&](int n) {  // dP^T = V_j dO_i^T
         const uint32_t so = st_off(n);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < D / 16; ++k) {
           const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32, qo = (k >> 2) * 8192 + (k & 3) * 32;
           mma_ss_e(tmem + C::T_DP, sdesc_add(dV_k, ko), sdesc_add(dO_k, so + qo), C::IDESC_S, k > 0);
         }
@@ -481,7 +486,7 @@ __global__ void __launch_bounds__(448, 1)
       const uint32_t src = tmem + lane_off + (is_dk ? C::T_DK : C::T_DV);
       uint8_t* stage = gb + C::ST_OFF + (is_dk ? 0 : C::ST_BYTES);  // the Q/dO ring is idle now
 #pragma unroll
-      for (int bx = 0; bx < 2; ++bx) {
+      for (int bx = 0; bx < C::NBOX; ++bx) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t o[32];
@@ -509,7 +514,7 @@ __global__ void __launch_bounds__(448, 1)
       const int row0 = 128 * j + 32 * wq;
       if (lane == 0 && row0 < a.N) {
         const uint32_t sbuf = sb + C::ST_OFF + (is_dk ? 0 : C::ST_BYTES);
-        for (int bx = 0; bx < 2; ++bx)
+        for (int bx = 0; bx < C::NBOX; ++bx)
           tma_store_3d(is_dk ? &tmdK : &tmdV, sbuf + bx * 16384 + wq * 4096, 64 * bx, row0, bh);
         bulk_commit();
         bulk_wait_read0();
@@ -546,35 +551,40 @@ cudaError_t launch_bwd_pre(const void* o, const void* dO, const float* lse, floa
   return cudaGetLastError();
 }
 
-template <bool WITH_DQ>
+template <int D, bool WITH_DQ>
 static cudaError_t launch_bwd_main_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                      const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
                                      const CUtensorMap& tdq, const BwdArgs& a, cudaStream_t stream) {
-  using C = BwdCfg;
+  using C = BwdCfg<D>;
   static_assert(C::SMEM <= 232448, "shared memory budget");
+  static_assert(C::SMEM > 116 * 1024, "one CTA per SM: each allocates all 512 TMEM columns");
   static bool attr_set[64];  // per device: the attribute outlives the call
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(fa_bwd_main_kernel<WITH_DQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    e = cudaFuncSetAttribute(fa_bwd_main_kernel<D, WITH_DQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   const int Tk = (a.N + 127) / 128;
   const int Tq = (a.N + 63) / 64;
   const long long grid = (long long)a.BH * Tk;
-  fa_bwd_main_kernel<WITH_DQ><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, tdo, tdk, tdv, tdq, a,
-                                                                                 Tk, Tq);
+  fa_bwd_main_kernel<D, WITH_DQ><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, tdo, tdk, tdv,
+                                                                                    tdq, a, Tk, Tq);
   return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_main(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
                             const CUtensorMap& tdq, const BwdArgs& a, cudaStream_t stream, bool with_dq) {
+  if (d == 64) {
+    if (with_dq) return cudaErrorNotSupported;
+    return launch_bwd_main_t<64, false>(tq, tk, tv, tdo, tdk, tdv, tdq, a, stream);
+  }
   if (d != 128) return cudaErrorNotSupported;
-  return with_dq ? launch_bwd_main_t<true>(tq, tk, tv, tdo, tdk, tdv, tdq, a, stream)
-                 : launch_bwd_main_t<false>(tq, tk, tv, tdo, tdk, tdv, tdq, a, stream);
+  return with_dq ? launch_bwd_main_t<128, true>(tq, tk, tv, tdo, tdk, tdv, tdq, a, stream)
+                 : launch_bwd_main_t<128, false>(tq, tk, tv, tdo, tdk, tdv, tdq, a, stream);
 }
 
 cudaError_t launch_bwd_post(const float* dq_acc, void* dq, long long elems, float scale, cudaStream_t stream) {

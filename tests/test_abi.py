@@ -95,7 +95,8 @@ def test_forward_empty_problem_is_a_no_op(kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(dO=0), INVALID), (dict(ws=0), INVALID), (dict(dq=0), INVALID), (dict(lse=0), INVALID),
     (dict(ws=A16 + 16), INVALID), (dict(dk=A16 + 8), INVALID), (dict(dO=A16 + 2), INVALID),
-    (dict(wsb=10), INVALID), (dict(d=64), UNSUPPORTED), (dict(d=80), UNSUPPORTED),
+    (dict(wsb=10), INVALID), (dict(d=32), UNSUPPORTED), (dict(d=80), UNSUPPORTED),
+    (dict(d=256), UNSUPPORTED),
     (dict(N=-5), INVALID), (dict(scale=-0.1), INVALID), (dict(causal=3), INVALID),
 ])
 def test_backward_rejects_bad_arguments(kw, code):

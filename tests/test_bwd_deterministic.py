@@ -113,3 +113,42 @@ def test_zero_upstream_gradient(cuda_ok):
     q, k, v, do = make_inputs(w)
     _, grads = _run(w, (q, k, v, torch.zeros_like(do)))
     assert all((g == 0).all() for g in grads)
+
+
+# ---------------------------------------------------------------- head dimension 64
+# fa_bwd at d = 64 runs the same two passes (the key pass has no atomic dQ path there).
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("N", [1, 3, 64, 65, 127, 128, 129, 200, 257, 513])
+@pytest.mark.parametrize("causal", [True, False])
+def test_d64_ragged_lengths(cuda_ok, N, causal):
+    _check(custom(1, 2, N, 64, causal, seed=100 + N, backward=True),
+           rel_tol=3e-2 if N <= 4 else None)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("B,H,N,causal", [(2, 3, 1000, True), (4, 2, 1024, False)])
+def test_d64_multi_head(cuda_ok, B, H, N, causal):
+    _check(custom(B, H, N, 64, causal, seed=77, backward=True))
+
+
+@pytest.mark.gpu
+def test_d64_large_scores(cuda_ok):
+    _check(custom(1, 2, 777, 64, True, seed=5, qk_std=math.sqrt(3.0), backward=True))
+
+
+@pytest.mark.gpu
+def test_d64_multi_head_workload_sampled(cuda_ok):
+    # B=4, H=16, N=1024, d=64 non-causal (the multi-head forward workload's shape): two heads
+    w = custom(4, 16, 1024, 64, False, seed=0, backward=True)
+    _check(w, heads=[(0, 0), (3, 15)])
+
+
+@pytest.mark.gpu
+def test_d64_fa_bwd_is_the_two_pass_path(cuda_ok):
+    w = custom(1, 3, 700, 64, True, seed=9, backward=True)
+    inputs = make_inputs(w)
+    _, gd = _run(w, inputs, deterministic=True)
+    _, ga = _run(w, inputs, deterministic=False)
+    for a, b in zip(gd, ga):
+        assert torch.equal(a, b)
