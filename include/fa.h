@@ -95,6 +95,26 @@ fa_status_t fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o,
                            void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Forward pass with FP8 operands for both tile GEMMs ("xinc.fun archive 235", section 4: matmuls
+ * in a low-precision format, accumulation and softmax kept at higher precision).
+ *   q, k, v   : in,  E4M3 (1 byte per element) [B,H,N,d]; the values are x * descale
+ *   descale_q, descale_k, descale_v
+ *             : in,  fp32 [B*H] per-(b,h) dequantisation factors (index b*H + h), or NULL
+ *               for 1.0 each
+ *   o, lse, scale, causal : as for fa_fwd; O = softmax(scale * Q K^T [masked]) V of the
+ *               dequantised values
+ * S = Q K^T and O += P V run as E4M3 x E4M3 -> fp32 MMAs; P (scaled by 2^8, so that it spans
+ * E4M3's range) is rounded to E4M3 for the PV product, while the row sums and the normaliser
+ * use the unrounded fp32 P.  Each element of O is then within 2^-4 * max|v| (P's rounding)
+ * plus bf16 output rounding of the exact attention of the dequantised inputs.
+ * Supported: d == 128.  Same layout, alignment (16 bytes for q, k, v, o; 4 for lse and the
+ * descale arrays), error and empty-problem rules as fa_fwd.
+ */
+fa_status_t fa_fwd_fp8(const void* q, const void* k, const void* v, const float* descale_q,
+                       const float* descale_k, const float* descale_v, void* o, float* lse,
+                       int B, int H, int N, int d, float scale, int causal, void* stream);
+
+/*
  * Bytes of device workspace that fa_bwd needs: per 64-row query tile, the fp32 base-2 LSE and
  * row term D_i of its 64 rows (B*H*ceil(N/64)*128 floats, rounded up to 256 bytes), followed
  * by the fp32 dQ accumulator [B*H*N*d].  Returns 0 for an empty or invalid shape.

@@ -133,6 +133,20 @@ bool make_tmap_bf16(CUtensorMap* m, const void* ptr, int BH, int N, int d, int b
                      [&](CUtensorMap* out) { return encode_tmap_bf16(out, ptr, BH, N, d, box_rows); });
 }
 
+bool make_tmap_e4m3(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_rows) {
+  return cached_tmap(m, TmapKey{reinterpret_cast<uintptr_t>(ptr), BH, N, d, 128, box_rows, 3}, [&](CUtensorMap* out) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)d, (cuuint64_t)N * d};
+    cuuint32_t box[3] = {128, (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(out, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  });
+}
+
 bool encode_tmap_bf16(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_rows) {
   auto enc = encode_fn();
   if (!enc) return false;
@@ -234,6 +248,39 @@ fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* 
   a.nsplit = 1;
   if ((long long)a.BH * a.nqb > INT_MAX) return FA_ERR_INVALID_ARG;
   return launch_fwd(d, tq, tk, tv, to, a, (cudaStream_t)stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status_t fa_fwd_fp8(const void* q, const void* k, const void* v, const float* descale_q,
+                       const float* descale_k, const float* descale_v, void* o, float* lse, int B, int H,
+                       int N, int d, float scale, int causal, void* stream) {
+  bool empty = false;
+  fa_status_t st = check_shape(B, H, N, d, scale, causal, &empty);
+  if (st != FA_OK || empty) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(descale_q, 4) || !aligned(descale_k, 4) || !aligned(descale_v, 4))
+    return FA_ERR_INVALID_ARG;
+  if ((st = check_device()) != FA_OK) return st;
+  const int BH = B * H;
+  CUtensorMap tq, tk, tv, to;
+  if (!make_tmap_e4m3(&tq, q, BH, N, d, 128) || !make_tmap_e4m3(&tk, k, BH, N, d, 128) ||
+      !make_tmap_e4m3(&tv, v, BH, N, d, 128) || !make_tmap_bf16(&to, o, BH, N, d, 32))
+    return FA_ERR_CUDA;
+  FwdArgs a;
+  if (!(a.status = device_status_word())) return FA_ERR_CUDA;
+  a.lse = lse;
+  a.N = N;
+  a.BH = BH;
+  a.nqb = (N + 255) / 256;
+  a.causal = causal;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  a.nsplit = 1;
+  a.descale_q = descale_q;
+  a.descale_k = descale_k;
+  a.descale_v = descale_v;
+  if ((long long)a.BH * a.nqb > INT_MAX) return FA_ERR_INVALID_ARG;
+  return launch_fwd_fp8(d, tq, tk, tv, to, a, (cudaStream_t)stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 // Split count used when the caller passes num_splits <= 0: enough CTAs to cover the SMs once,

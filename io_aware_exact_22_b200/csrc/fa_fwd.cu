@@ -29,11 +29,20 @@ using namespace ptx;
 // Column pairs (out of every 8 pairs) whose exponential is evaluated on the FMA pipe.
 constexpr int kPolyPairsOf8 = 3;
 
-template <int D>
+// FP8: Q, K, V are E4M3 (one byte per element) and both tile GEMMs run as kind::f8f6f4; P is
+// quantised to E4M3 for the PV GEMM.  Softmax, accumulators and the output are as for bf16.
+template <int D, bool FP8 = false>
 struct FwdCfg {
-  static constexpr int NBOX = D / 64;              // 64-column (128-byte) swizzle boxes per row
-  static constexpr int TILE = 128 * D * 2;         // bytes of one 128-row bf16 tile
-  static constexpr int NS = (D == 128) ? 4 : 8;    // K/V ring stages (one K or one V each)
+  static constexpr int EB = FP8 ? 1 : 2;           // bytes per input element
+  static constexpr int BOXW = 128 / EB;            // elements per 128-byte swizzle box row
+  static constexpr int NBOX = D / BOXW;            // swizzle boxes per row
+  static constexpr int TILE = 128 * D * EB;        // bytes of one 128-row input tile
+  static constexpr int NS = (TILE == 32768) ? 4 : 8;  // K/V ring stages (one K or one V each)
+  static constexpr int KSTEP = 32 / EB;            // elements of K per MMA (32 bytes)
+  static constexpr int P_COLS = 128 * EB / 4;      // TMEM columns of packed P for 128 keys
+  static constexpr int OTILE = 128 * D * 2;        // bytes of one 128-row bf16 output tile
+  // O staging: the dead Q tiles (bf16) or the idle K/V ring (FP8: Q tiles are half as large)
+  static constexpr int OST_OFF = FP8 ? 2 * TILE : 0;
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = 2 * TILE;
   static constexpr int BAR_OFF = KV_OFF + NS * TILE;
@@ -45,18 +54,24 @@ struct FwdCfg {
   static constexpr uint32_t TMEM_COLS = 512;
   // TMEM columns (a 512-column allocation always starts at column 0, lane 0)
   static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_O0 = 256, T_O1 = 256 + D;
-  static constexpr uint32_t IDESC_QK = idesc_bf16(128, 128, false, false);
-  static constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);
+  static constexpr uint32_t IDESC_QK = FP8 ? idesc_e4m3(128, 128, false, false) : idesc_bf16(128, 128, false, false);
+  static constexpr uint32_t IDESC_PV = FP8 ? idesc_e4m3(128, D, false, true) : idesc_bf16(128, D, false, true);
+  // P is computed as 2^(s c - m + P_OFF) and the reference m moves once a block's max exceeds
+  // it by more than MOVE (both base 2).  bf16: P <= 2^8.  FP8: P <= 2^8.75 < 448 (the largest
+  // E4M3 value) and values down to 2^-17 of the reference term stay representable.
+  static constexpr float P_OFF = FP8 ? 8.0f : 0.0f;
+  static constexpr float MOVE = FP8 ? 0.75f : 8.0f;
 };
 
 // PARTIAL: the CTA covers only its split's range of key blocks and writes the normalised
 // partial output O_s (fp32) and its LSE_s, to be combined by fa_fwd_merge_kernel.
-template <int D, bool PARTIAL>
+template <int D, bool PARTIAL, bool FP8 = false>
 __global__ void __launch_bounds__(320, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const FwdArgs a) {
-  using C = FwdCfg<D>;
+  static_assert(!FP8 || (D == 128 && !PARTIAL), "FP8: d = 128, whole key range");
+  using C = FwdCfg<D, FP8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
@@ -135,8 +150,8 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive_expect_tx_e(q_full, nq * C::TILE);
       for (int t = 0; t < nq; ++t)
         for (int b = 0; b < C::NBOX; ++b)
-          tma_load_3d_e(sb + C::Q_OFF + t * C::TILE + b * 16384, &tmQ, q_full, 64 * b, q0 + 128 * t, bh,
-                        keep);
+          tma_load_3d_e(sb + C::Q_OFF + t * C::TILE + b * 16384, &tmQ, q_full, C::BOXW * b, q0 + 128 * t,
+                        bh, keep);
       int it = 0;
       bool ok = true;
       for (int j = 0; j < nmax && ok; ++j) {
@@ -147,8 +162,8 @@ __global__ void __launch_bounds__(320, 1)
           mbar_arrive_expect_tx_e(kv_full(s), C::TILE);
           const CUtensorMap* m = kv ? &tmV : &tmK;
           for (int b = 0; b < C::NBOX; ++b)
-            tma_load_3d_e(sb + C::KV_OFF + s * C::TILE + b * 16384, m, kv_full(s), 64 * b, 128 * (kb0 + j), bh,
-                          keep);
+            tma_load_3d_e(sb + C::KV_OFF + s * C::TILE + b * 16384, m, kv_full(s), C::BOXW * b, 128 * (kb0 + j),
+                          bh, keep);
         }
       }
       if (!ok) {  // let copies already issued land before the CTA exits
@@ -170,15 +185,23 @@ __global__ void __launch_bounds__(320, 1)
       const uint64_t dV_mn = sdesc_sw128(sb + C::KV_OFF, 16384, 1024);  // V stages, MN-major
       auto issue_qk = [&](uint32_t dst, uint32_t qoff, uint32_t koff) {
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
+        for (int k = 0; k < D / C::KSTEP; ++k) {  // 32 bytes of d per MMA
           const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-          mma_ss_e(dst, sdesc_add(dQ_k, qoff + off), sdesc_add(dK_k, koff + off), C::IDESC_QK, k > 0);
+          if constexpr (FP8)
+            mma_ss_e8(dst, sdesc_add(dQ_k, qoff + off), sdesc_add(dK_k, koff + off), C::IDESC_QK, k > 0);
+          else
+            mma_ss_e(dst, sdesc_add(dQ_k, qoff + off), sdesc_add(dK_k, koff + off), C::IDESC_QK, k > 0);
         }
       };
       auto issue_pv = [&](uint32_t dst, uint32_t ptm, uint32_t voff, bool acc) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          mma_ts_e(dst, ptm + 8 * k, sdesc_add(dV_mn, voff + k * 2048), C::IDESC_PV, (acc || k > 0) ? 1u : 0u);
+        for (int k = 0; k < 128 / C::KSTEP; ++k) {  // KSTEP keys per MMA: 8 TMEM columns of P
+          const uint32_t vo = voff + k * C::KSTEP * 128;
+          if constexpr (FP8)
+            mma_ts_e8(dst, ptm + 8 * k, sdesc_add(dV_mn, vo), C::IDESC_PV, (acc || k > 0) ? 1u : 0u);
+          else
+            mma_ts_e(dst, ptm + 8 * k, sdesc_add(dV_mn, vo), C::IDESC_PV, (acc || k > 0) ? 1u : 0u);
+        }
       };
       auto stage_addr = [&](int it) { return (uint32_t)((it % C::NS) * C::TILE); };
       auto stage_par = [&](int it) { return (uint32_t)((it / C::NS) & 1); };
@@ -237,7 +260,13 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tSrow = tmem + lane_off + 128u * t;
     const uint32_t tOrow = tmem + lane_off + 256u + (uint32_t)(D * t);
-    const float cs = a.scale_log2;
+    float cs = a.scale_log2;
+    float vmul = 1.f;  // FP8: V's dequantisation factor, applied to O at the end
+    if constexpr (FP8) {
+      if (a.descale_q) cs *= a.descale_q[bh];
+      if (a.descale_k) cs *= a.descale_k[bh];
+      if (a.descale_v) vmul = a.descale_v[bh];
+    }
     float m_ref = -INFINITY;  // reference max, base-2 scaled units
     float l = 0.f;
     bool ok = !*abort_flag;
@@ -267,6 +296,7 @@ __global__ void __launch_bounds__(320, 1)
       auto exp_full = [&](float mneg) -> float {
         const uint64_t cs2 = f2_pack(cs, cs), mn2 = f2_pack(mneg, mneg);
         uint64_t sa = f2_pack(0.f, 0.f), sb2 = f2_pack(0.f, 0.f);
+        float q0p = 0.f, q1p = 0.f;  // FP8: the previous pair, packed with the next one
 #pragma unroll
         for (int c = 0; c < 128; c += 2) {
           const uint64_t y = f2_fma(f2_pack(x[c], x[c + 1]), cs2, mn2);
@@ -283,7 +313,14 @@ __global__ void __launch_bounds__(320, 1)
             sb2 = f2_add(sb2, f2_pack(p0, p1));
           else
             sa = f2_add(sa, f2_pack(p0, p1));
-          pk[c >> 1] = pack_bf16(p0, p1);
+          if constexpr (FP8) {
+            if ((c >> 1) & 1)
+              pk[c >> 2] = pack_e4m3x4(q0p, q1p, p0, p1);
+            else
+              q0p = p0, q1p = p1;
+          } else {
+            pk[c >> 1] = pack_bf16(p0, p1);
+          }
         }
         float s0, s1, s2, s3;
         f2_unpack(sa, s0, s1);
@@ -312,7 +349,7 @@ __global__ void __launch_bounds__(320, 1)
           if (c > lim) x[c] = -INFINITY;
       }
       const float mblk = block_max();
-      const bool move = mblk > m_ref + 8.0f;
+      const bool move = mblk > m_ref + C::MOVE;
       float alpha = 1.f;
       if (move) {
         alpha = ex2(m_ref - mblk);  // 0 when m_ref is still -inf
@@ -332,26 +369,42 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       l *= alpha;
-      const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      if constexpr (FP8) mneg += C::P_OFF;
       float rsum;
       if (!edge) {
         rsum = exp_full(mneg);
       } else {
         // the block with the diagonal or the ragged tail: masked columns are exactly 0
         float rs0 = 0.f, rs1 = 0.f;
+        if constexpr (FP8) {
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const float p0 = (c > lim) ? 0.f : ex2(fmaf(x[c], cs, mneg));
-          const float p1 = (c + 1 > lim) ? 0.f : ex2(fmaf(x[c + 1], cs, mneg));
-          rs0 += p0;
-          rs1 += p1;
-          pk[c >> 1] = pack_bf16(p0, p1);
+          for (int c = 0; c < 128; c += 4) {
+            const float p0 = (c > lim) ? 0.f : ex2(fmaf(x[c], cs, mneg));
+            const float p1 = (c + 1 > lim) ? 0.f : ex2(fmaf(x[c + 1], cs, mneg));
+            const float p2 = (c + 2 > lim) ? 0.f : ex2(fmaf(x[c + 2], cs, mneg));
+            const float p3 = (c + 3 > lim) ? 0.f : ex2(fmaf(x[c + 3], cs, mneg));
+            rs0 += p0;
+            rs1 += p1;
+            rs0 += p2;
+            rs1 += p3;
+            pk[c >> 2] = pack_e4m3x4(p0, p1, p2, p3);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; c += 2) {
+            const float p0 = (c > lim) ? 0.f : ex2(fmaf(x[c], cs, mneg));
+            const float p1 = (c + 1 > lim) ? 0.f : ex2(fmaf(x[c + 1], cs, mneg));
+            rs0 += p0;
+            rs1 += p1;
+            pk[c >> 1] = pack_bf16(p0, p1);
+          }
         }
         rsum = rs0 + rs1;
       }
       l += rsum;
       tmem_st32(tSrow + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(tSrow + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      if constexpr (!FP8) tmem_st32(tSrow + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full(t));
@@ -365,12 +418,13 @@ __global__ void __launch_bounds__(320, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(o_full, 0, wc));
       if (ok) {
         tc_fence_after();
-        const float inv = (l > 0.f) ? 1.f / l : 0.f;
+        const float inv = (l > 0.f) ? vmul / l : 0.f;
         const int row0 = q0 + 128 * t + 32 * wq;
         if (!PARTIAL) {
-          uint8_t* stage = gb + C::Q_OFF + t * C::TILE;  // Q_t is dead once o_full has fired
+          // Q_t (bf16) or the K/V ring (FP8) is dead once o_full has fired
+          uint8_t* stage = gb + C::OST_OFF + t * C::OTILE;
 #pragma unroll
-          for (int b = 0; b < C::NBOX; ++b) {
+          for (int b = 0; b < D / 64; ++b) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               uint32_t o[32];
@@ -392,15 +446,15 @@ __global__ void __launch_bounds__(320, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0 && row0 < a.N) {
-            for (int b = 0; b < C::NBOX; ++b)
-              tma_store_3d(&tmO, sb + C::Q_OFF + t * C::TILE + b * 16384 + wq * 4096, 64 * b, row0, bh);
+            for (int b = 0; b < D / 64; ++b)
+              tma_store_3d(&tmO, sb + C::OST_OFF + t * C::OTILE + b * 16384 + wq * 4096, 64 * b, row0, bh);
             bulk_commit();
             bulk_wait_read0();
           }
           __syncwarp();
           if (qrow < a.N)
             a.lse[(size_t)bh * a.N + qrow] =
-                (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+                (l > 0.f) ? (m_ref - C::P_OFF + log2f(l)) * 0.69314718055994530942f : -INFINITY;
         } else {
           // fp32 partial O_s = O / l of this split, staged in the (now idle) K/V ring as
           // 32-column, 128-byte-swizzled boxes and written by TMA; then LSE_s.
@@ -445,23 +499,25 @@ __global__ void __launch_bounds__(320, 1)
   }
 }
 
-template <int D, bool PARTIAL>
+template <int D, bool PARTIAL, bool FP8 = false>
 static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const CUtensorMap& to, const FwdArgs& a, cudaStream_t stream) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, FP8>;
   static_assert(C::SMEM <= 232448, "shared memory budget");
+  static_assert(C::SMEM > 116 * 1024, "one CTA per SM: each allocates all 512 TMEM columns");
   static_assert(2 * 128 * D * 4 <= C::NS * C::TILE, "partial-output staging must fit the K/V ring");
+  static_assert(C::OST_OFF + 2 * C::OTILE <= C::BAR_OFF, "output staging must fit");
   static bool attr_set[64];  // per device: the attribute outlives the call
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(fa_fwd_kernel<D, PARTIAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    e = cudaFuncSetAttribute(fa_fwd_kernel<D, PARTIAL, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   const long long grid = (long long)a.BH * a.nqb * a.nsplit;
-  fa_fwd_kernel<D, PARTIAL><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, to, a);
+  fa_fwd_kernel<D, PARTIAL, FP8><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, to, a);
   return cudaGetLastError();
 }
 
@@ -473,6 +529,12 @@ cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, cons
   }
   if (d == 64) return launch_fwd_t<64, false>(tq, tk, tv, to, a, stream);
   return launch_fwd_t<128, false>(tq, tk, tv, to, a, stream);
+}
+
+cudaError_t launch_fwd_fp8(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const CUtensorMap& to, const FwdArgs& a, cudaStream_t stream) {
+  if (d != 128 || a.nsplit != 1) return cudaErrorNotSupported;
+  return launch_fwd_t<128, false, true>(tq, tk, tv, to, a, stream);
 }
 
 // Combines the split-wise partial results of one query row, using the two-block softmax merge

@@ -16,6 +16,10 @@ struct FwdArgs {
   int causal;        // 0 / 1
   float scale_log2;  // scale * log2(e)
   int nsplit;        // key-range splits per (head, query block); 1 = whole key range
+  // FP8 forward only: per-(b,h) dequantisation factors [BH], or null for 1
+  const float* descale_q = nullptr;
+  const float* descale_k = nullptr;
+  const float* descale_v = nullptr;
 };
 
 struct BwdArgs {
@@ -44,6 +48,9 @@ cudaError_t launch_wait_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t 
 
 // Tensor maps for a bf16 [BH, N, d] tensor, 128-byte swizzle, box = 64 columns x `rows`
 // (make_*: served from a cache of encoded maps; encode_*: always encodes).
+// 3-D map over an E4M3 tensor [BH, N, d] (one byte per element), box {128, box_rows},
+// 128-byte swizzle.
+bool make_tmap_e4m3(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_rows);
 bool make_tmap_bf16(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_rows);
 bool encode_tmap_bf16(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_rows);
 bool encode_tmap_f32(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_inner, int box_rows,
@@ -53,6 +60,9 @@ bool encode_tmap_f32(CUtensorMap* m, const void* ptr, int BH, int N, int d, int 
 // outputs [nsplit * BH, N, d] (box 32 x 32, 128-byte swizzle) and a.lse the partial LSEs.
 cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& to, const FwdArgs& a, cudaStream_t stream);
+// FP8 (E4M3) inputs, d = 128, whole key range; Q/K/V maps from make_tmap_e4m3 (128-row boxes)
+cudaError_t launch_fwd_fp8(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const CUtensorMap& to, const FwdArgs& a, cudaStream_t stream);
 // Combines nsplit partial (O_s, LSE_s) into bf16 O and fp32 LSE.
 cudaError_t launch_fwd_merge(const float* o_part, const float* lse_part, void* o, float* lse, int nsplit,
                              long long rows, int d, cudaStream_t stream);

@@ -24,7 +24,7 @@ STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_E
 EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_device_status",
            "fa_status_string", "fa_version", "fa_bwd_noalloc", "fa_selftest_wait_timeout",
            "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_default_splits",
-           "fa_bwd_deterministic")
+           "fa_bwd_deterministic", "fa_fwd_fp8")
 # Size of the library's built-in scratch used by fa_bwd_noalloc (include/fa.h).
 NOALLOC_MAX_SCRATCH_BYTES = 64 << 20
 
@@ -48,6 +48,8 @@ def lib() -> ctypes.CDLL:
         vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
         L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
         L.fa_fwd.restype = i
+        L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+        L.fa_fwd_fp8.restype = i
         L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, vp]
         L.fa_bwd.restype = i
         L.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
@@ -94,6 +96,13 @@ def _stream(stream):
 def fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, stream=None) -> int:
     return lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
                         float(scale), int(causal), _stream(stream))
+
+
+def fa_fwd_fp8(q, k, v, descale_q, descale_k, descale_v, o, lse, B, H, N, d, scale, causal,
+               stream=None) -> int:
+    return lib().fa_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(descale_q), _ptr(descale_k),
+                            _ptr(descale_v), _ptr(o), _ptr(lse), B, H, N, d, float(scale),
+                            int(causal), _stream(stream))
 
 
 def fa_fwd_splitkv(q, k, v, o, lse, B, H, N, d, scale, causal, num_splits, workspace,
@@ -174,6 +183,31 @@ def forward(q, k, v, causal: bool, scale: float | None = None, out=None, lse=Non
     rc = fa_fwd(q, k, v, out, lse, B, H, N, d, scale, causal)
     if rc:
         raise FAError(rc, "fa_fwd")
+    return out, lse
+
+
+def forward_fp8(q8, k8, v8, descale_q, descale_k, descale_v, causal: bool,
+                scale: float | None = None, out=None, lse=None):
+    """O (bf16), LSE = attention of FP8 inputs through fa_fwd_fp8.  q8, k8, v8: contiguous
+    CUDA tensors [B,H,N,d] of E4M3 codes (torch.uint8 or torch.float8_e4m3fn); descale_*:
+    fp32 CUDA tensors with B*H elements, or None for 1."""
+    for t, n in ((q8, "q8"), (k8, "k8"), (v8, "v8")):
+        if not (t.is_cuda and t.element_size() == 1 and t.dim() == 4 and t.is_contiguous()):
+            raise ValueError(f"{n} must be a contiguous CUDA tensor of E4M3 codes [B,H,N,d]")
+    B, H, N, d = q8.shape
+    for t, n in ((descale_q, "descale_q"), (descale_k, "descale_k"), (descale_v, "descale_v")):
+        if t is not None and not (t.is_cuda and t.dtype == torch.float32 and t.numel() == B * H
+                                  and t.is_contiguous()):
+            raise ValueError(f"{n} must be a contiguous CUDA fp32 tensor of B*H elements")
+    scale = d ** -0.5 if scale is None else scale
+    if out is None:
+        out = torch.empty((B, H, N, d), device=q8.device, dtype=torch.bfloat16)
+    if lse is None:
+        lse = torch.empty((B, H, N), device=q8.device, dtype=torch.float32)
+    rc = fa_fwd_fp8(q8, k8, v8, descale_q, descale_k, descale_v, out, lse, B, H, N, d, scale,
+                    causal)
+    if rc:
+        raise FAError(rc, "fa_fwd_fp8")
     return out, lse
 
 

@@ -91,6 +91,32 @@ def make_inputs(w: Workload, with_grad: bool | None = None):
     return tuple(out)
 
 
+E4M3_MAX = 448.0  # largest finite FP8 E4M3 value
+
+
+def make_fp8_inputs(w: Workload):
+    """FP8 (E4M3) inputs for workload ``w``: q, k, v are drawn exactly as in make_inputs (same
+    generator, order and standard deviations, in fp32), then each (b, h) slice x of each tensor
+    is stored as E4M3 codes c = e4m3(x / descale) with descale = max|x| / 448, the conversion
+    being torch's float8_e4m3fn cast (round to nearest even).  The slice then stands for
+    c * descale.  Returns ((q8, k8, v8) uint8 code tensors [B,H,N,d],
+    (descale_q, descale_k, descale_v) fp32 tensors [B,H]).  Codes and factors are the inputs
+    of both the FP8 kernel and the oracle."""
+    g = torch.Generator("cpu").manual_seed(w.seed)
+    shape = w.shape
+    xs = [torch.randn(shape, generator=g, dtype=torch.float32) * w.qk_std,
+          torch.randn(shape, generator=g, dtype=torch.float32) * w.qk_std,
+          torch.randn(shape, generator=g, dtype=torch.float32)]
+    codes, descales = [], []
+    for x in xs:
+        amax = x.abs().amax(dim=(2, 3))
+        ds = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
+        c = (x / ds[:, :, None, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+        codes.append(c)
+        descales.append(ds.to(torch.float32))
+    return tuple(codes), tuple(descales)
+
+
 def custom(B: int, H: int, N: int, d: int, causal: bool, seed: int = 0,
            qk_std: float = 1.0, backward: bool = False) -> Workload:
     """An ad-hoc workload (used for ragged tails and edge cases in the tests)."""

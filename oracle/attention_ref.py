@@ -125,6 +125,50 @@ def attention_forward(q, k, v, scale: float, causal: bool):
     return o, lse
 
 
+# ---------------------------------------------------------------------------- FP8 inputs
+# [xinc] section 4 (减少访存的几种办法): matmul operands may be held in a low-precision format
+# such as FP8 while accumulation and softmax stay at higher precision.  With FP8 inputs the
+# attention to compute is that of the values the codes represent; the oracle decodes them
+# exactly and runs the fp64 attention above on them.
+
+def e4m3_decode(codes) -> np.ndarray:
+    """fp64 values of FP8 E4M3 codes (uint8), from the format's definition (the "FN" variant:
+    no infinities): bit 7 sign, bits 3-6 exponent e with bias 7, bits 0-2 mantissa m.
+      e = 0          : subnormal, (m / 8) * 2^-6   (so 0x01 = 2^-9 and 0x00 = +0)
+      e = 1..15      : (1 + m / 8) * 2^(e - 7)     (largest finite: e = 15, m = 6 -> 448)
+      e = 15, m = 7  : NaN
+    """
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where((c & 0x80) != 0, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
+def attention_forward_fp8(q8, k8, v8, descale_q, descale_k, descale_v, scale: float,
+                          causal: bool):
+    """Exact attention of FP8 (E4M3) inputs [B,H,N,d] given as uint8 codes, each (b, h) slice
+    representing code value * descale[b, h] (descale arrays [B, H]; None means 1).  Returns
+    (O [B,H,N,d], LSE [B,H,N]) in fp64."""
+    q = e4m3_decode(q8)
+    k = e4m3_decode(k8)
+    v = e4m3_decode(v8)
+    B, H = q.shape[:2]
+    ones = np.ones((B, H))
+    dq = ones if descale_q is None else _f64(descale_q).reshape(B, H)
+    dk = ones if descale_k is None else _f64(descale_k).reshape(B, H)
+    dv = ones if descale_v is None else _f64(descale_v).reshape(B, H)
+    o = np.zeros(v.shape)
+    lse = np.zeros(q.shape[:3])
+    for b in range(B):
+        for h in range(H):
+            o[b, h], lse[b, h] = attention_forward_head(q[b, h] * dq[b, h], k[b, h] * dk[b, h],
+                                                        v[b, h] * dv[b, h], scale, causal)
+    return o, lse
+
+
 def attention_backward_head(q, k, v, do, scale: float, causal: bool, row_chunk: int = 4096,
                             rows: np.ndarray | None = None):
     """Gradients of O = softmax(scale * Q K^T) V for one head, by plain calculus of the
