@@ -299,9 +299,98 @@ def run_gpu(args):
     }
     if e2e is not None:
         line["e2e"] = e2e
+    if not args.no_variants and world == 1:
+        line["variants"] = measure_variants(w, dev, stream, qd, kd, vd, o, lse, dod, dq, dk, dv, ws,
+                                            ws_bytes, peak)
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(w, q, k, v, do)
     return line
+
+
+# ---------------------------------------------------------------------- variants
+def _time_ms(fn, stream, iters=10, warmup=3):
+    """Mean device time of fn() in ms: CUDA events on the launching stream, after warm-up."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(iters):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def measure_variants(w, dev, stream, qd, kd, vd, o, lse, dod, dq, dk, dv, ws, ws_bytes, peak):
+    """The other entry points of the library, each timed on its own after the step's timed
+    region: FP8 forward and deterministic backward at the step's shape, split-KV forward where
+    it matters (few (b,h) pairs, long keys), and the d = 64 backward at the multi-head
+    workload's shape.  TFLOPS use the same algorithmic FLOP formulas as the step."""
+    from io_aware_exact_22_b200 import fa
+    from io_aware_exact_22_b200.inputs import custom, make_fp8_inputs
+    B, H, N, d = w.shape
+    sp = stream.cuda_stream
+    out = {}
+
+    def chk(rc, name):
+        if rc:
+            raise RuntimeError(f"{name} failed: {rc}")
+
+    # FP8 (E4M3) forward, same shape; peak = 2 x the bf16 peak (the nominal fp8 : bf16 ratio)
+    (q8, k8, v8), dsc = make_fp8_inputs(w)
+    q8, k8, v8 = (t.to(dev) for t in (q8, k8, v8))
+    dsc = [t.reshape(-1).to(dev) for t in dsc]
+    ms = _time_ms(lambda: chk(fa.fa_fwd_fp8(q8, k8, v8, *dsc, o, lse, B, H, N, d, w.scale, w.causal, sp),
+                              "fa_fwd_fp8"), stream)
+    tf = w.fwd_flops() / (ms * 1e-3) / 1e12
+    out["fwd_fp8"] = {"kernel": "fa_fwd_kernel<128, fp8>", "ms": round(ms, 4), "tflops": round(tf, 1),
+                      "peak": 2 * peak, "frac": round(tf / (2 * peak), 4), "shape": w.name}
+    del q8, k8, v8
+    # deterministic backward, same shape (inputs from the step)
+    chk(fa.fa_fwd(qd, kd, vd, o, lse, B, H, N, d, w.scale, w.causal, sp), "fa_fwd")
+    ms = _time_ms(lambda: chk(fa.fa_bwd_deterministic(qd, kd, vd, o, dod, lse, dq, dk, dv, ws, ws_bytes,
+                                                      B, H, N, d, w.scale, w.causal, sp),
+                              "fa_bwd_deterministic"), stream, iters=5)
+    tf = w.bwd_flops() / (ms * 1e-3) / 1e12
+    out["bwd_deterministic"] = {"kernels": "fa_bwd_main_kernel<128, no dQ> + fa_bwd_dq_kernel<128>",
+                                "ms": round(ms, 4), "tflops": round(tf, 1), "peak": peak,
+                                "frac": round(tf / peak, 4), "shape": w.name}
+    # split-KV: two (b,h) pairs of a long causal sequence leave most SMs idle without splits
+    ws2 = custom(1, 2, N, 128, True, seed=3)
+    q2, k2, v2 = (t[:, :2].contiguous() for t in (qd, kd, vd))
+    o2 = torch.empty_like(q2)
+    l2 = torch.empty((1, 2, N), device=dev, dtype=torch.float32)
+    nsp = fa.fa_fwd_splitkv_default_splits(1, 2, N, 128, 1)
+    wsb = fa.fa_fwd_splitkv_workspace_bytes(1, 2, N, 128, nsp)
+    wsk = torch.empty(max(wsb, 256), device=dev, dtype=torch.uint8)
+    ms_s = _time_ms(lambda: chk(fa.fa_fwd_splitkv(q2, k2, v2, o2, l2, 1, 2, N, 128, ws2.scale, 1, nsp, wsk,
+                                                  wsb, sp), "fa_fwd_splitkv"), stream)
+    ms_u = _time_ms(lambda: chk(fa.fa_fwd(q2, k2, v2, o2, l2, 1, 2, N, 128, ws2.scale, 1, sp), "fa_fwd"), stream)
+    tf_s = ws2.fwd_flops() / (ms_s * 1e-3) / 1e12
+    out["fwd_splitkv"] = {"kernels": "fa_fwd_kernel<128, partial> + fa_fwd_merge_kernel<128>",
+                          "shape": f"B=1 H=2 N={N} d=128 causal", "splits": nsp, "ms": round(ms_s, 4),
+                          "tflops": round(tf_s, 1), "frac": round(tf_s / peak, 4), "peak": peak,
+                          "unsplit_ms": round(ms_u, 4),
+                          "unsplit_tflops": round(ws2.fwd_flops() / (ms_u * 1e-3) / 1e12, 1)}
+    del q2, k2, v2, o2, l2, wsk
+    # d = 64 backward (two-pass path), B=4 H=16 N=1024 d=64 non-causal
+    w64 = custom(4, 16, 1024, 64, False, seed=0, backward=True)
+    q6, k6, v6, d6 = (t.to(dev) for t in make_inputs(w64, with_grad=True))
+    o6, l6 = torch.empty_like(q6), torch.empty((4, 16, 1024), device=dev, dtype=torch.float32)
+    g6 = [torch.empty_like(q6) for _ in range(3)]
+    wb6 = fa.fa_bwd_workspace_bytes(4, 16, 1024, 64)
+    w6 = torch.empty(wb6, device=dev, dtype=torch.uint8)
+    chk(fa.fa_fwd(q6, k6, v6, o6, l6, 4, 16, 1024, 64, w64.scale, 0, sp), "fa_fwd")
+    ms = _time_ms(lambda: chk(fa.fa_bwd(q6, k6, v6, o6, d6, l6, *g6, w6, wb6, 4, 16, 1024, 64, w64.scale, 0, sp),
+                              "fa_bwd d=64"), stream)
+    tf = w64.bwd_flops() / (ms * 1e-3) / 1e12
+    out["bwd_d64"] = {"kernels": "fa_bwd_main_kernel<64, no dQ> + fa_bwd_dq_kernel<64>",
+                      "shape": "B=4 H=16 N=1024 d=64", "ms": round(ms, 4), "tflops": round(tf, 1),
+                      "peak": peak, "frac": round(tf / peak, 4)}
+    if fa.fa_get_device_status(sp) != 0:
+        raise RuntimeError("device-side timeout while timing the variants")
+    return out
 
 
 # ---------------------------------------------------------------------- CPU (oracle) arms
@@ -377,6 +466,8 @@ def main():
     ap.add_argument("--workload", type=int, default=4, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the timing of the FP8, deterministic, split-KV and d=64 variants")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

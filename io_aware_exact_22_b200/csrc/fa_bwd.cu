@@ -12,15 +12,16 @@
 //                   zeroes the fp32 dQ accumulator.  Memory-bound.
 //   K3 fa_bwd_main  one CTA per (head, 128-key tile j); K_j and V_j stay in shared memory and
 //                   the 64-row query tiles i stream through a 3-stage TMA ring.  Per tile:
-//                     S^T  = K_j Q_i^T          (tcgen05, TMEM)
+//                     S^T  = K_j Q_i^T          (tcgen05, TMEM, two buffers)
 //                     dP^T = V_j dO_i^T         (tcgen05, TMEM)
 //                     P^T  = exp2(S^T * scale*log2e - LSE2_i)          (registers)
 //                     dV  += P^T dO_i           (tcgen05, A = P^T from TMEM)
-//                     dS^T = P^T o (dP^T - D_i)                         (registers)
-//                     dK  += dS^T Q_i           (tcgen05, A = dS^T from TMEM)
+//                     dS^T = P^T o (dP^T - D_i)                         (registers -> smem)
+//                     dK  += dS^T Q_i           (tcgen05, A = dS^T from shared memory)
 //                     dQ_i^T = K_j^T dS^T        (tcgen05, B = dS^T from shared memory)
-//                   and dQ_i^T is added into the fp32 accumulator by TMA reduce-add.
-//                   TMEM columns: S^T [0,64), dP^T [64,128), dQ^T x2 [128,256),
+//                   and dQ_i^T is added into the fp32 accumulator (reductions from registers
+//                   for half of its rows, TMA reduce-add for the other half).
+//                   TMEM columns: S^T x2 [0,128), dP^T [128,192), dQ^T [192,256),
 //                   dV [256,384), dK [384,512).
 //   K4 fa_bwd_post  dQ = scale * accumulator, rounded to bf16.
 #include "fa_internal.cuh"
@@ -122,17 +123,18 @@ struct BwdCfg {
   static constexpr int DQS_WARP = (BQ - kBwdDqRedRows) * 32 * 4;
   static constexpr int LD_OFF = DQS_OFF + 4 * DQS_WARP;
   static constexpr int BAR_OFF = LD_OFF + NSQ * LDB;
-  // kv_full, qd_full[3], qd_empty[3], s_full, dp_full, p_ready, ds_ready, dq_full[2],
-  // dq_free[2], ds_free[2], kv_done
-  static constexpr int NBAR = 1 + 2 * NSQ + 4 + 6 + 1;
+  // kv_full, qd_full[3], qd_empty[3], s_full[2], dp_full, p_ready, ds_ready, dq_full,
+  // dq_free, ds_free[2], kv_done
+  static constexpr int NBAR = 1 + 2 * NSQ + 10;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM = MISC_OFF + 16 + 1024;
   static constexpr int THREADS = 448;
   static constexpr uint32_t TMEM_COLS = 512;
   // TMEM columns (a 512-column allocation always starts at column 0, lane 0)
-  static constexpr uint32_t T_S = 0, T_DP = 64, T_DQ = 128, T_DV = 256, T_DK = 384;
+  // S^T is double-buffered: [0,64) for even query tiles, [64,128) for odd ones
+  static constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 192, T_DV = 256, T_DK = 384;
   static constexpr uint32_t IDESC_S = idesc_bf16(128, BQ, false, false);   // S^T, dP^T
-  static constexpr uint32_t IDESC_KV = idesc_bf16(128, D, false, true);    // dV, dK
+  static constexpr uint32_t IDESC_KV = idesc_bf16(128, D, false, true);    // dV, dK (B MN-major)
   static constexpr uint32_t IDESC_Q = idesc_bf16(128, BQ, true, true);     // dQ^T
 };
 
@@ -142,11 +144,16 @@ struct BwdCfg {
 //   warps 8-11  dQ^T drain: TMEM -> shared staging -> TMA reduce-add into the fp32 accumulator
 //   warp 12     MMA issuer (whole warp, one elected lane issues)
 //   warp 13     TMA producer (whole warp, one elected lane issues)
-// Each compute warpgroup writes its packed P^T (and dS^T) inside its own S^T (dP^T) columns,
-// so neither overwrites scores the other has not read yet: P^T of query columns [32g, 32g+32)
-// sits at TMEM columns [32g, 32g+16), dS^T at [64+32g, 64+32g+16).
-// WITH_DQ = false: dK and dV only (dQ comes from fa_bwd_dq_kernel): no dQ^T MMA, no dS^T in
-// shared memory, no drain.  The dQ^T MMA puts d on the M dimension (128 TMEM lanes), so the
+// Each compute warpgroup writes its packed P^T inside its own S^T columns, so neither
+// overwrites scores the other has not read yet: P^T of query columns [32g, 32g+32) sits at
+// TMEM columns [32g, 32g+16) of the tile's S^T buffer.  dS^T goes to shared memory only,
+// where it is the A operand of dK += dS^T Q_i and the B operand of dQ^T = K_j^T dS^T.
+//
+// The schedule keeps the slow chains (scores -> P on the compute warps, P -> dV on the tensor
+// core) off each other's critical path: S^T is double-buffered, so S_{n+2} is issued right
+// after dV_n; and since dK reads dS^T from shared memory, the dP^T columns are free as soon
+// as dS_n is computed, so dP_{n+1} is issued before dK_n and dQ_n.
+// WITH_DQ = false: dK and dV only (dQ comes from fa_bwd_dq_kernel): no dQ^T MMA, no drain.  The dQ^T MMA puts d on the M dimension (128 TMEM lanes), so the
 // atomic dQ path exists for D = 128 only; D = 64 always runs with WITH_DQ = false.
 template <int D, bool WITH_DQ>
 __global__ void __launch_bounds__(448, 1)
@@ -174,14 +181,15 @@ __global__ void __launch_bounds__(448, 1)
   const uint32_t kv_full = bar;
   auto qd_full = [&](int s) { return bar + 8u * (1 + s); };
   auto qd_empty = [&](int s) { return bar + 8u * (1 + C::NSQ + s); };
-  const uint32_t s_full = bar + 8u * (1 + 2 * C::NSQ);
-  const uint32_t dp_full = s_full + 8;
-  const uint32_t p_ready = s_full + 16;
-  const uint32_t ds_ready = s_full + 24;
-  auto dq_full = [&](int b) { return s_full + 32 + 8u * b; };
-  auto dq_free = [&](int b) { return s_full + 48 + 8u * b; };
-  auto ds_free = [&](int b) { return s_full + 64 + 8u * b; };
-  const uint32_t kv_done = s_full + 80;
+  const uint32_t bar2 = bar + 8u * (1 + 2 * C::NSQ);
+  auto s_full = [&](int b) { return bar2 + 8u * b; };
+  const uint32_t dp_full = bar2 + 16;
+  const uint32_t p_ready = bar2 + 24;
+  const uint32_t ds_ready = bar2 + 32;
+  const uint32_t dq_full = bar2 + 40;
+  const uint32_t dq_free = bar2 + 48;
+  auto ds_free = [&](int b) { return bar2 + 56 + 8u * b; };
+  const uint32_t kv_done = bar2 + 72;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gb + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + C::MISC_OFF + 4);
   const WaitCtx wc{abort_flag, a.status};
@@ -192,13 +200,13 @@ __global__ void __launch_bounds__(448, 1)
       mbar_init(qd_full(s), 1);
       mbar_init(qd_empty(s), 1);
     }
-    mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
     mbar_init(p_ready, 256);
     mbar_init(ds_ready, 256);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, 128);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(dq_full(b), 1);
-      mbar_init(dq_free(b), 128);
+      mbar_init(s_full(b), 1);
       mbar_init(ds_free(b), 1);
     }
     mbar_init(kv_done, 1);
@@ -255,12 +263,12 @@ __global__ void __launch_bounds__(448, 1)
     __syncwarp();
   } else if (warp == 12) {
     // ------------------------------------------------------------ MMA issuer (whole warp)
-    // Issue order, software-pipelined by one query tile so that the tensor core never waits
-    // for the compute warps in steady state:
-    //   S_0, dP_0 | dV_n, S_{n+1}, dK_n, dQ_n, dP_{n+1} | ...
-    // S_{n+1} overwrites the S^T/P^T columns only after dV_n (which reads P^T_n) and dP_{n+1}
-    // overwrites the dP^T/dS^T columns only after dK_n (which reads dS^T_n): tcgen05 MMAs
-    // issued by one thread execute in order.
+    // Issue order:  S_0, S_1, dP_0 | [P_n ready] dV_n, [dS_n ready] dP_{n+1}, dK_n, dQ_n, S_{n+2} | ...
+    // Every overwrite follows the last reader in issue order (tcgen05 MMAs issued by one
+    // thread execute in order): S_{n+2} follows dV_n, which reads P_n from the same buffer;
+    // dP_{n+1} follows the compute warps' read of dP_n (signalled by ds_ready).  S_{n+2} comes
+    // last because its Q tile is the most recently requested load; it is needed only after
+    // the compute warps have finished tile n+1.
     if (!*abort_flag) {
       bool ok = __all_sync(0xffffffffu, mbar_wait(kv_full, 0, wc));
       // Base descriptors; each MMA adds its byte offset (see sdesc_add).
@@ -271,16 +279,17 @@ __global__ void __launch_bounds__(448, 1)
       const uint64_t dO_k = sdesc_sw128(sb + C::ST_OFF + C::QT, 16, 1024);  // dO_i, K-major (dP^T)
       const uint64_t dQ_mn = sdesc_sw128(sb + C::ST_OFF, 8192, 1024);    // Q_i, MN-major (dK)
       const uint64_t dO_mn = sdesc_sw128(sb + C::ST_OFF + C::QT, 8192, 1024);  // dO_i, MN-major (dV)
+      const uint64_t dS_k = sdesc_sw128(sb + C::DS_OFF, 16, 1024);       // dS^T, K-major (dK)
       const uint64_t dS_mn = sdesc_sw128(sb + C::DS_OFF, 8192, 1024);    // dS^T, MN-major (dQ^T)
       auto st_off = [&](int n) { return (uint32_t)((n % C::NSQ) * C::ST_BYTES); };
-      auto issue_s = [&](int n) {  // S^T = K_j Q_i^T  (K over d)
+      auto issue_s = [&](int n) {  // S^T = K_j Q_i^T  (K over d), into buffer n & 1
         const uint32_t so = st_off(n);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32, qo = (k >> 2) * 8192 + (k & 3) * 32;
-          mma_ss_e(tmem + C::T_S, sdesc_add(dK_k, ko), sdesc_add(dQ_k, so + qo), C::IDESC_S, k > 0);
+          mma_ss_e(tmem + C::T_S + 64 * (n & 1), sdesc_add(dK_k, ko), sdesc_add(dQ_k, so + qo), C::IDESC_S, k > 0);
         }
-        mma_commit_e(s_full);
+        mma_commit_e(s_full(n & 1));
       };
       auto issue_dp = [&](int n) {  // dP^T = V_j dO_i^T
         const uint32_t so = st_off(n);
@@ -291,11 +300,18 @@ __global__ void __launch_bounds__(448, 1)
         }
         mma_commit_e(dp_full);
       };
+      auto wait_q = [&](int n) {
+        return __all_sync(0xffffffffu, mbar_wait(qd_full(n % C::NSQ), (n / C::NSQ) & 1, wc));
+      };
       if (ok && count > 0) {
-        if ((ok = __all_sync(0xffffffffu, mbar_wait(qd_full(0), 0, wc)))) {
+        if ((ok = wait_q(0))) {
           tc_fence_after();
           issue_s(0);
-          issue_dp(0);
+          if (count > 1 && (ok = wait_q(1))) {
+            tc_fence_after();
+            issue_s(1);
+          }
+          if (ok) issue_dp(0);
         }
       }
       for (int n = 0; n < count && ok; ++n) {
@@ -305,35 +321,32 @@ __global__ void __launch_bounds__(448, 1)
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(p_ready, n & 1, wc)))) break;
         tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < 4; ++k)  // dV += P^T dO_i  (K over the 64 queries)
-          mma_ts_e(tmem + C::T_DV, tmem + C::T_S + 32 * (k >> 1) + 8 * (k & 1), sdesc_add(dO_mn, so + k * 2048),
-                   C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
-        const bool more = n + 1 < count;
-        if (more) {
-          if (!(ok = __all_sync(0xffffffffu,
-                                mbar_wait(qd_full((n + 1) % C::NSQ), ((n + 1) / C::NSQ) & 1, wc))))
-            break;
-          tc_fence_after();
-          issue_s(n + 1);
-        }
+        for (int k = 0; k < 4; ++k)  // dV += P^T dO_i  (K over the 64 queries; A = P^T from TMEM)
+          mma_ts_e(tmem + C::T_DV, tmem + C::T_S + 64 * b + 32 * (k >> 1) + 8 * (k & 1),
+                   sdesc_add(dO_mn, so + k * 2048), C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(ds_ready, n & 1, wc)))) break;
         tc_fence_after();
+        if (n + 1 < count) issue_dp(n + 1);  // Q/dO_{n+1} landed before S_{n+1} was issued
 #pragma unroll
-        for (int k = 0; k < 4; ++k)  // dK += dS^T Q_i
-          mma_ts_e(tmem + C::T_DK, tmem + C::T_DP + 32 * (k >> 1) + 8 * (k & 1), sdesc_add(dQ_mn, so + k * 2048),
+        for (int k = 0; k < 4; ++k)  // dK += dS^T Q_i  (K over the 64 queries; A = dS^T in smem)
+          mma_ss_e(tmem + C::T_DK, sdesc_add(dS_k, b * C::DS_BYTES + 32 * k), sdesc_add(dQ_mn, so + k * 2048),
                    C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
         if (WITH_DQ) {
-          if (!(ok = __all_sync(0xffffffffu, mbar_wait(dq_free(b), ((n >> 1) & 1) ^ 1, wc)))) break;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(dq_free, (n & 1) ^ 1, wc)))) break;
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 8; ++k)  // dQ_i^T = K_j^T dS^T  (K over the 128 keys)
-            mma_ss_e(tmem + C::T_DQ + 64 * b, sdesc_add(dK_mn, k * 2048),
-                     sdesc_add(dS_mn, b * C::DS_BYTES + k * 2048), C::IDESC_Q, k > 0);
-          mma_commit_e(dq_full(b));
-          mma_commit_e(ds_free(b));
+            mma_ss_e(tmem + C::T_DQ, sdesc_add(dK_mn, k * 2048), sdesc_add(dS_mn, b * C::DS_BYTES + k * 2048),
+                     C::IDESC_Q, k > 0);
+          mma_commit_e(dq_full);
         }
+        mma_commit_e(ds_free(b));
         mma_commit_e(qd_empty(s));
-        if (more) issue_dp(n + 1);
+        if (n + 2 < count) {
+          if (!(ok = wait_q(n + 2))) break;
+          tc_fence_after();
+          issue_s(n + 2);
+        }
       }
       mma_commit_e(kv_done);
       if (!ok) mbar_wait_drain(kv_done, 0);
@@ -347,7 +360,7 @@ __global__ void __launch_bounds__(448, 1)
     const int key = 128 * j + r;
     const bool key_ok = key < a.N;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::T_S + 32 * g;
+    const uint32_t tS0 = tmem + lane_off + C::T_S + 32 * g;  // + 64 for odd query tiles
     const uint32_t tDP = tmem + lane_off + C::T_DP + 32 * g;
     const float cs = a.scale_log2;
     bool ok = !*abort_flag;
@@ -356,9 +369,10 @@ __global__ void __launch_bounds__(448, 1)
       const int i = i0 + n;
       const int b = n & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(qd_full(s), (n / C::NSQ) & 1, wc) &&
-                                       mbar_wait(s_full, n & 1, wc));
+                                       mbar_wait(s_full(b), (n >> 1) & 1, wc));
       if (!ok) break;
       tc_fence_after();
+      const uint32_t tS = tS0 + 64 * b;
       uint32_t sr[32];
       tmem_ld32(tS, sr);
       const float* ldp = reinterpret_cast<const float*>(gb + C::LD_OFF + s * C::LDB) + 32 * g;
@@ -407,22 +421,19 @@ __global__ void __launch_bounds__(448, 1)
       }
 #pragma unroll
       for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(p[2 * c], p[2 * c + 1]);
-      tmem_st16(tDP, pk);
-      if (WITH_DQ) {
-        // dS^T row r, query columns [32 g, 32 g + 32), into the shared buffer read by the dQ MMA
-        ok = __all_sync(0xffffffffu, mbar_wait(ds_free(b), ((n >> 1) & 1) ^ 1, wc));
-        if (!ok) break;
-        uint8_t* dsrow = gb + C::DS_OFF + b * C::DS_BYTES + r * 128;
+      // dS^T row r, query columns [32 g, 32 g + 32), into the shared buffer read by the dK and
+      // dQ MMAs (128-byte rows, 16-byte chunks swizzled by the row index)
+      ok = __all_sync(0xffffffffu, mbar_wait(ds_free(b), ((n >> 1) & 1) ^ 1, wc));
+      if (!ok) break;
+      uint8_t* dsrow = gb + C::DS_OFF + b * C::DS_BYTES + r * 128;
 #pragma unroll
-        for (int c16 = 0; c16 < 4; ++c16) {
-          const int chunk = 4 * g + c16;
-          *reinterpret_cast<uint4*>(dsrow + ((chunk ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
-        }
-        fence_proxy_async_smem();
+      for (int c16 = 0; c16 < 4; ++c16) {
+        const int chunk = 4 * g + c16;
+        *reinterpret_cast<uint4*>(dsrow + ((chunk ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
       }
-      tmem_wait_st();
-      tc_fence_before();
+      fence_proxy_async_smem();
+      tc_fence_before();  // the tcgen05.ld of dP^T is complete before dP_{n+1} may overwrite it
       mbar_arrive(ds_ready);
     }
   } else {
@@ -433,18 +444,17 @@ __global__ void __launch_bounds__(448, 1)
     const uint32_t stage_s = sb + C::DQS_OFF + wq * C::DQS_WARP;
     bool ok = !*abort_flag;
     for (int n = 0; n < (WITH_DQ ? count : 0) && ok; ++n) {
-      const int b = n & 1;
       const int i = i0 + n;
-      ok = __all_sync(0xffffffffu, mbar_wait(dq_full(b), (n >> 1) & 1, wc));
+      ok = __all_sync(0xffffffffu, mbar_wait(dq_full, n & 1, wc));
       if (!ok) break;
       tc_fence_after();
       uint32_t v[64];
-      tmem_ld32(tmem + lane_off + C::T_DQ + 64 * b, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_ld32(tmem + lane_off + C::T_DQ + 64 * b + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      tmem_ld32(tmem + lane_off + C::T_DQ, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_ld32(tmem + lane_off + C::T_DQ + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
       tmem_wait_ld();
       reg_fence(v);
       tc_fence_before();
-      mbar_arrive(dq_free(b));
+      mbar_arrive(dq_free);  // one dQ^T buffer: the next dQ MMA may overwrite it now
       // Split between two paths that use different resources: the first kBwdDqRedRows query
       // rows are added with fp32 reductions straight from registers (lane = d, so each row is
       // one coalesced 128-byte request), the rest are staged as a [rows][32 d] fp32 slice in
