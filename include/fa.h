@@ -87,6 +87,12 @@ fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* 
  *   workspace       : device scratch, 256-byte aligned, at least
  *                     fa_fwd_splitkv_workspace_bytes(B,H,N,d,splits) bytes for the number of
  *                     splits used (not needed, may be NULL, when that number is 1).
+ *
+ * fa_fwd_splitkv_default_splits returns the split count (1-4) that the library would choose:
+ * it simulates the grid's makespan on the current device's SMs (CTAs in launch order to the
+ * first free SM) for 1-4 splits and splits only when that predicts a gain of at least 1.25
+ * (the partial outputs and the merge cost the rest), which in practice means causal, long
+ * sequences over few heads.  Host-only; without a CUDA device it assumes 148 SMs.
  */
 int fa_fwd_splitkv_default_splits(int B, int H, int N, int d, int causal);
 size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int N, int d, int num_splits);

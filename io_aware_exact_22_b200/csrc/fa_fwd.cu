@@ -26,8 +26,11 @@ namespace fa {
 
 using namespace ptx;
 
-// Column pairs (out of every 8 pairs) whose exponential is evaluated on the FMA pipe.
-constexpr int kPolyPairsOf8 = 3;
+// Column pairs (out of every 8 pairs) whose exponential is evaluated on the FMA pipe.  Per
+// element and warp, MUFU ex2 occupies its pipe ~8 cycles and the polynomial the FMA pipe
+// ~9.3, on top of ~3.6 FMA-pipe cycles of scaling, row sum and packing; the two pipes balance
+// at a polynomial share of about 1/4.
+constexpr int kPolyPairsOf8 = 2;
 
 // FP8: Q, K, V are E4M3 (one byte per element) and both tile GEMMs run as kind::f8f6f4; P is
 // quantised to E4M3 for the PV GEMM.  Softmax, accumulators and the output are as for bf16.

@@ -93,3 +93,16 @@ def test_one_split_is_the_plain_forward(cuda_ok):
     o2, l2 = fa.forward(q, k, v, False, w.scale)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("B,H,N,causal,want", [
+    (1, 2, 16384, 1, 2), (1, 4, 16384, 1, 2), (1, 1, 32768, 1, 2),   # causal, few heads: split
+    (1, 2, 16384, 0, 1), (1, 8, 4096, 0, 1),                          # balanced rows: no gain
+    (1, 16, 4096, 1, 1), (1, 32, 16384, 1, 1), (4, 16, 1024, 0, 1),   # enough work to fill the SMs
+    (1, 1, 256, 0, 1)])
+def test_default_split_choice(B, H, N, causal, want):
+    # Host-side choice (a makespan simulation); the cases are those where a sweep of 1-8 splits
+    # on a B200 showed splitting to pay (1.2-1.9x) or to cost (up to 1.4x).
+    if torch.cuda.is_available() and torch.cuda.get_device_properties(0).multi_processor_count != 148:
+        pytest.skip("choices calibrated for 148 SMs")
+    assert fa.fa_fwd_splitkv_default_splits(B, H, N, 128, causal) == want
