@@ -160,10 +160,12 @@ def run_gpu(args):
     sp = stream.cuda_stream
     scale = w.scale
 
+    bwd_fn = fa.fa_bwd_deterministic if args.deterministic else fa.fa_bwd
+
     def step():
         rc = fa.fa_fwd(qd, kd, vd, o, lse, B, H, N, d, scale, w.causal, sp)
-        rc |= fa.fa_bwd(qd, kd, vd, o, dod, lse, dq, dk, dv, ws, ws_bytes, B, H, N, d, scale,
-                        w.causal, sp)
+        rc |= bwd_fn(qd, kd, vd, o, dod, lse, dq, dk, dv, ws, ws_bytes, B, H, N, d, scale,
+                     w.causal, sp)
         if rc:
             raise RuntimeError(f"fa call failed: {rc}")
 
@@ -186,8 +188,8 @@ def run_gpu(args):
         ev[i][0].record(stream)
         rc = fa.fa_fwd(qd, kd, vd, o, lse, B, H, N, d, scale, w.causal, sp)
         ev[i][1].record(stream)
-        rc |= fa.fa_bwd(qd, kd, vd, o, dod, lse, dq, dk, dv, ws, ws_bytes, B, H, N, d, scale,
-                        w.causal, sp)
+        rc |= bwd_fn(qd, kd, vd, o, dod, lse, dq, dk, dv, ws, ws_bytes, B, H, N, d, scale,
+                     w.causal, sp)
         ev[i][2].record(stream)
         if rc:
             raise RuntimeError(f"fa call failed: {rc}")
@@ -244,8 +246,8 @@ def run_gpu(args):
             if i >= 2:
                 stream.wait_event(ev_down[b])  # step i-2's results have left these buffers
             rc = fa.fa_fwd(qx, kx, vx, ox, lx, B, H, N, d, scale, w.causal, sp)
-            rc |= fa.fa_bwd(qx, kx, vx, ox, dx, lx, gq, gk, gv, ws, ws_bytes, B, H, N, d, scale,
-                            w.causal, sp)
+            rc |= bwd_fn(qx, kx, vx, ox, dx, lx, gq, gk, gv, ws, ws_bytes, B, H, N, d, scale,
+                         w.causal, sp)
             if rc:
                 raise RuntimeError(f"fa call failed: {rc}")
             ev_comp[b].record(stream)
@@ -309,7 +311,8 @@ def run_gpu(args):
         "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
-                   "step": "fa_fwd + fa_bwd", "per_rank": "same workload on every rank",
+                   "step": "fa_fwd + " + ("fa_bwd_deterministic" if args.deterministic else "fa_bwd"),
+                   "per_rank": "same workload on every rank",
                    "l2": "inputs larger than L2 (q,k,v,o,dO 134 MB each vs 126 MB L2), no flush"},
         "pct_of_peak": round(100 * value / world / peak, 2),
         "fwd": {"ms": round(fwd_ms, 4), "tflops": round(fwd_tflops, 1),
@@ -502,6 +505,8 @@ def main():
     ap.add_argument("--workload", type=int, default=4, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="run the step's backward through fa_bwd_deterministic")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the timing of the FP8, deterministic, split-KV and d=64 variants")
     args = ap.parse_args()

@@ -461,12 +461,13 @@ fa_status_t fa_bwd_deterministic(const void* q, const void* k, const void* v, co
   cudaStream_t s = (cudaStream_t)stream;
   // main kernel (dK, dV): Q/dO in 64-row boxes, K/V in 128-row boxes
   CUtensorMap tq64, tk128, tv128, tdo64, tdk, tdv;
-  // dQ kernel: Q/dO and K/V in 128-row boxes, dQ stored in 32-row boxes
-  CUtensorMap tq128, tdo128, tdq;
+  // dQ kernel: Q/dO in 128-row boxes, K/V in 64-row boxes, dQ stored in 32-row boxes
+  CUtensorMap tq128, tk64, tv64, tdo128, tdq;
   if (!make_tmap_bf16(&tq64, q, BH, N, d, 64) || !make_tmap_bf16(&tk128, k, BH, N, d, 128) ||
       !make_tmap_bf16(&tv128, v, BH, N, d, 128) || !make_tmap_bf16(&tdo64, dO, BH, N, d, 64) ||
       !make_tmap_bf16(&tdk, dk, BH, N, d, 32) || !make_tmap_bf16(&tdv, dv, BH, N, d, 32) ||
-      !make_tmap_bf16(&tq128, q, BH, N, d, 128) || !make_tmap_bf16(&tdo128, dO, BH, N, d, 128) ||
+      !make_tmap_bf16(&tq128, q, BH, N, d, 128) || !make_tmap_bf16(&tk64, k, BH, N, d, 64) ||
+      !make_tmap_bf16(&tv64, v, BH, N, d, 64) || !make_tmap_bf16(&tdo128, dO, BH, N, d, 128) ||
       !make_tmap_bf16(&tdq, dq, BH, N, d, 32))
     return FA_ERR_CUDA;
   BwdArgs a;
@@ -481,7 +482,7 @@ fa_status_t fa_bwd_deterministic(const void* q, const void* k, const void* v, co
   a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   if (launch_bwd_pre(o, dO, lse, ld, nullptr, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
   if (launch_bwd_main(d, tq64, tk128, tv128, tdo64, tdk, tdv, tdk, a, s, false) != cudaSuccess) return FA_ERR_CUDA;
-  if (launch_bwd_dq(d, tq128, tk128, tv128, tdo128, tdq, a, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (launch_bwd_dq(d, tq128, tk64, tv64, tdo128, tdq, a, s) != cudaSuccess) return FA_ERR_CUDA;
   return FA_OK;
 }
 

@@ -2,7 +2,7 @@
 //
 // dQ = scale * dS K with dS = P o (dP - D), P = exp(S - LSE), S = scale Q K^T, dP = dO V^T
 // (the recomputation backward of "xinc.fun archive 235", section 7).  Here one CTA owns 128
-// query rows and walks the key blocks of 128 keys in order, accumulating dQ in TMEM, so dQ is
+// query rows and walks the key blocks of 64 keys in order, accumulating dQ in TMEM, so dQ is
 // written once per row with a fixed summation order: no atomics, bitwise reproducible.  It
 // recomputes S and dP (the main backward kernel, run in its dK/dV-only mode, recomputes them
 // too); the pair replaces the main kernel's atomic dQ path when determinism is asked for, and
@@ -10,9 +10,8 @@
 //
 // Roles (192 threads): warps 0-3 compute P and dS (one query row per thread, its LSE2 and D in
 // registers), warp 4 issues MMAs, warp 5 issues TMA loads.
-// TMEM columns: S_b [128 b, 128 b + 128) for key blocks j with b = j & 1 (dS_j, bf16,
-// overwrites the first 64 columns of S_b), dP [256, 384), dQ [384, 384 + d).  Blocks of 128
-// keys keep every MMA at N = 128 (a tcgen05.mma costs about as much at N = 64).
+// TMEM columns: S_b [64 b, 64 b + 64) and dP_b [128 + 64 b, + 64) for key blocks j with
+// b = j & 1 (dS_j, bf16, overwrites the first 32 columns of S_b), dQ [256, 256 + d).
 #include "fa_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -28,25 +27,25 @@ template <int D>
 struct DqCfg {
   static constexpr int NBOX = D / 64;
   static constexpr int QT = 128 * D * 2;      // Q_i or dO_i (128 rows)
-  static constexpr int KT = 128 * D * 2;      // K_j or V_j (128 keys)
-  static constexpr int NS = (D == 128) ? 2 : 3;  // K/V ring stages, each [K_j | V_j]
+  static constexpr int KT = 64 * D * 2;       // K_j or V_j (64 keys)
+  static constexpr int NS = 3;                // K/V ring stages, each [K_j | V_j]
   static constexpr int Q_OFF = 0;
   static constexpr int DO_OFF = QT;
   static constexpr int KV_OFF = 2 * QT;
   static constexpr int ST_BYTES = 2 * KT;
   static constexpr int BAR_OFF = KV_OFF + NS * ST_BYTES;
-  // q_full, kv_full[NS], kv_empty[NS], s_full[2], dp_full, ds_ready, dq_done
-  static constexpr int NBAR = 1 + 2 * NS + 2 + 1 + 1 + 1;
+  // q_full, kv_full[NS], kv_empty[NS], s_full[2], ds_ready[2], dq_done
+  static constexpr int NBAR = 1 + 2 * NS + 2 + 2 + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   // Launched with at least 116 KB so that two CTAs never share an SM: both would ask for all
-  // 512 TMEM columns and the second would stall in tcgen05.alloc.
+  // 512 TMEM columns and the second would stall in tcgen05.alloc (d = 64 needs only ~83 KB).
   static constexpr int SMEM_USED = MISC_OFF + 16 + 1024;
   static constexpr int SMEM = SMEM_USED < 116 * 1024 ? 116 * 1024 : SMEM_USED;
   static constexpr int THREADS = 192;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t T_S = 0, T_DP = 256, T_DQ = 384;  // S_b at 128 b; dS_b over its first 64
-  static constexpr uint32_t IDESC_SP = idesc_bf16(128, 128, false, false);  // S, dP (N = 128 keys)
-  static constexpr uint32_t IDESC_DQ = idesc_bf16(128, D, false, true);     // dQ (N = d)
+  static constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 256;
+  static constexpr uint32_t IDESC_SP = idesc_bf16(128, 64, false, false);  // S, dP (N = 64 keys)
+  static constexpr uint32_t IDESC_DQ = idesc_bf16(128, D, false, true);    // dQ (N = d)
 };
 
 template <int D>
@@ -67,16 +66,15 @@ __global__ void __launch_bounds__(192, 1)
   const int bh = blockIdx.x / Tq128;
   const int it = Tq128 - 1 - (blockIdx.x % Tq128);
   const int q0 = 128 * it;
-  const int Tk = (a.N + 127) >> 7;
-  const int nblk = a.causal ? min(Tk, it + 1) : Tk;  // 128-key blocks with a visible key
+  const int Tk64 = (a.N + 63) >> 6;
+  const int nblk = a.causal ? min(Tk64, 2 * it + 2) : Tk64;  // 64-key blocks with a visible key
 
   const uint32_t bar = sb + C::BAR_OFF;
   const uint32_t q_full = bar;
   auto kv_full = [&](int s) { return bar + 8u * (1 + s); };
   auto kv_empty = [&](int s) { return bar + 8u * (1 + C::NS + s); };
   auto s_full = [&](int b) { return bar + 8u * (1 + 2 * C::NS + b); };
-  const uint32_t dp_full = bar + 8u * (3 + 2 * C::NS);
-  const uint32_t ds_ready = bar + 8u * (4 + 2 * C::NS);
+  auto ds_ready = [&](int b) { return bar + 8u * (3 + 2 * C::NS + b); };
   const uint32_t dq_done = bar + 8u * (5 + 2 * C::NS);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gb + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + C::MISC_OFF + 4);
@@ -88,9 +86,10 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(kv_full(s), 1);
       mbar_init(kv_empty(s), 1);
     }
-    for (int b = 0; b < 2; ++b) mbar_init(s_full(b), 1);
-    mbar_init(dp_full, 1);
-    mbar_init(ds_ready, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(s_full(b), 1);
+      mbar_init(ds_ready(b), 128);
+    }
     mbar_init(dq_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -125,8 +124,8 @@ __global__ void __launch_bounds__(192, 1)
         mbar_arrive_expect_tx_e(kv_full(s), C::ST_BYTES);
         const uint32_t st = sb + C::KV_OFF + s * C::ST_BYTES;
         for (int b = 0; b < C::NBOX; ++b) {
-          tma_load_3d_e(st + b * 16384, &tmK, kv_full(s), 64 * b, 128 * j, bh, keep);
-          tma_load_3d_e(st + C::KT + b * 16384, &tmV, kv_full(s), 64 * b, 128 * j, bh, keep);
+          tma_load_3d_e(st + b * 8192, &tmK, kv_full(s), 64 * b, 64 * j, bh, keep);
+          tma_load_3d_e(st + C::KT + b * 8192, &tmV, kv_full(s), 64 * b, 64 * j, bh, keep);
         }
       }
       if (j < nblk) {  // aborted: let issued copies land before the CTA exits
@@ -138,61 +137,52 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   } else if (warp == 4) {
     // ------------------------------------------------------------ MMA issuer (whole warp)
-    // Order:  S_0, dP_0 | S_{j+1}, [dS_j ready] dQ += dS_j K_j, dP_{j+1} | ...
-    // S is double-buffered, so S_{j+1} goes ahead of dS_j; S_{j+1} overwrites the buffer of
-    // dS_{j-1}, whose dQ product was issued before it (tcgen05 MMAs issued by one thread
-    // execute in order); dP_{j+1} follows the compute warps' read of dP_j (ds_ready).
+    // S_{j+1} and dP_{j+1} are issued before waiting for dS_j, so the tensor core works on the
+    // next key block while the compute warps turn block j into dS_j.
     if (!*abort_flag && nblk > 0) {
       const uint64_t dQ_k = sdesc_sw128(sb + C::Q_OFF, 16, 1024);
       const uint64_t dO_k = sdesc_sw128(sb + C::DO_OFF, 16, 1024);
       const uint64_t dK_k = sdesc_sw128(sb + C::KV_OFF, 16, 1024);
       const uint64_t dV_k = sdesc_sw128(sb + C::KV_OFF + C::KT, 16, 1024);
-      const uint64_t dK_mn = sdesc_sw128(sb + C::KV_OFF, 16384, 1024);
-      auto issue_s = [&](int j) {  // S_j = Q K_j^T  (K over d), into buffer j & 1
+      const uint64_t dK_mn = sdesc_sw128(sb + C::KV_OFF, 8192, 1024);
+      auto issue_sp = [&](int j) {  // S_j = Q K_j^T, dP_j = dO V_j^T  (K over d)
         const uint32_t so = (uint32_t)((j % C::NS) * C::ST_BYTES);
+        const uint32_t b = (uint32_t)(j & 1);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-          mma_ss_e(tmem + C::T_S + 128 * (j & 1), sdesc_add(dQ_k, off), sdesc_add(dK_k, so + off), C::IDESC_SP,
-                   k > 0);
+          const uint32_t qo = (k >> 2) * 16384 + (k & 3) * 32, ko = (k >> 2) * 8192 + (k & 3) * 32;
+          mma_ss_e(tmem + C::T_S + 64 * b, sdesc_add(dQ_k, qo), sdesc_add(dK_k, so + ko), C::IDESC_SP, k > 0);
         }
-        mma_commit_e(s_full(j & 1));
-      };
-      auto issue_dp = [&](int j) {  // dP_j = dO V_j^T
-        const uint32_t so = (uint32_t)((j % C::NS) * C::ST_BYTES);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-          mma_ss_e(tmem + C::T_DP, sdesc_add(dO_k, off), sdesc_add(dV_k, so + off), C::IDESC_SP, k > 0);
+          const uint32_t qo = (k >> 2) * 16384 + (k & 3) * 32, ko = (k >> 2) * 8192 + (k & 3) * 32;
+          mma_ss_e(tmem + C::T_DP + 64 * b, sdesc_add(dO_k, qo), sdesc_add(dV_k, so + ko), C::IDESC_SP, k > 0);
         }
-        mma_commit_e(dp_full);
-      };
-      auto wait_kv = [&](int j) {
-        return __all_sync(0xffffffffu, mbar_wait(kv_full(j % C::NS), (j / C::NS) & 1, wc));
+        mma_commit_e(s_full(b));
       };
       bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, wc));
-      if (ok) ok = wait_kv(0);
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(kv_full(0), 0, wc));
       if (ok) {
         tc_fence_after();
-        issue_s(0);
-        issue_dp(0);
+        issue_sp(0);
       }
       for (int j = 0; j < nblk && ok; ++j) {
         const int b = j & 1;
         if (j + 1 < nblk) {
-          if (!(ok = wait_kv(j + 1))) break;
+          // S/dP buffer b^1 was last read by the compute warps before they released dS_{j-1}
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(kv_full((j + 1) % C::NS), ((j + 1) / C::NS) & 1, wc))))
+            break;
           tc_fence_after();
-          issue_s(j + 1);
+          issue_sp(j + 1);
         }
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(ds_ready, j & 1, wc)))) break;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(ds_ready(b), (j >> 1) & 1, wc)))) break;
         tc_fence_after();
         const uint32_t so = (uint32_t)((j % C::NS) * C::ST_BYTES);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)  // dQ += dS_j K_j  (K over the 128 keys; A = dS_j from TMEM)
-          mma_ts_e(tmem + C::T_DQ, tmem + C::T_S + 128 * b + 8 * k, sdesc_add(dK_mn, so + k * 2048), C::IDESC_DQ,
+        for (int k = 0; k < 4; ++k)  // dQ += dS_j K_j  (K over the 64 keys)
+          mma_ts_e(tmem + C::T_DQ, tmem + C::T_S + 64 * b + 8 * k, sdesc_add(dK_mn, so + k * 2048), C::IDESC_DQ,
                    (j > 0 || k > 0) ? 1u : 0u);
         mma_commit_e(kv_empty(j % C::NS));
-        if (j + 1 < nblk) issue_dp(j + 1);
       }
       mma_commit_e(dq_done);
       if (!ok) mbar_wait_drain(dq_done, 0);
@@ -213,41 +203,33 @@ __global__ void __launch_bounds__(192, 1)
     bool ok = !*abort_flag;
     for (int j = 0; j < nblk && ok; ++j) {
       const int b = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full(b), (j >> 1) & 1, wc) && mbar_wait(dp_full, j & 1, wc));
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full(b), (j >> 1) & 1, wc));
       if (!ok) break;
       tc_fence_after();
-      // keys 128 j + c: visible iff below N and (causal) not after this query
-      int lim = a.N - 1 - 128 * j;
-      if (a.causal) lim = min(lim, qrow - 128 * j);
-      const uint32_t tS = tmem + lane_off + C::T_S + 128 * b;
-      const uint32_t tDP = tmem + lane_off + C::T_DP;
-      // 64 keys at a time (four TMEM loads in flight per wait); dS (bf16, packed) of chunk c
-      // goes to columns [32c, 32c + 32) of the same buffer, which this thread has already read
+      uint32_t x[64], y[64];
+      tmem_ld32(tmem + lane_off + C::T_S + 64 * b, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
+      tmem_ld32(tmem + lane_off + C::T_S + 64 * b + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
+      tmem_ld32(tmem + lane_off + C::T_DP + 64 * b, *reinterpret_cast<uint32_t(*)[32]>(&y[0]));
+      tmem_ld32(tmem + lane_off + C::T_DP + 64 * b + 32, *reinterpret_cast<uint32_t(*)[32]>(&y[32]));
+      tmem_wait_ld();
+      reg_fence(x);
+      reg_fence(y);
+      // keys 64 j + c: visible iff below N and (causal) not after this query
+      int lim = a.N - 1 - 64 * j;
+      if (a.causal) lim = min(lim, qrow - 64 * j);
+      uint32_t pk[32];
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t x[64], y[64];
-        tmem_ld32(tS + 64 * ch, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
-        tmem_ld32(tS + 64 * ch + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
-        tmem_ld32(tDP + 64 * ch, *reinterpret_cast<uint32_t(*)[32]>(&y[0]));
-        tmem_ld32(tDP + 64 * ch + 32, *reinterpret_cast<uint32_t(*)[32]>(&y[32]));
-        tmem_wait_ld();
-        reg_fence(x);
-        reg_fence(y);
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const int kc = 64 * ch + c;
-          float p0 = ex2(fmaf(__uint_as_float(x[c]), cs, -l2));
-          float p1 = ex2(fmaf(__uint_as_float(x[c + 1]), cs, -l2));
-          p0 = (kc > lim) ? 0.f : p0 * (__uint_as_float(y[c]) - dd);
-          p1 = (kc + 1 > lim) ? 0.f : p1 * (__uint_as_float(y[c + 1]) - dd);
-          pk[c >> 1] = pack_bf16(p0, p1);
-        }
-        tmem_st32(tS + 32 * ch, pk);
+      for (int c = 0; c < 64; c += 2) {
+        float p0 = ex2(fmaf(__uint_as_float(x[c]), cs, -l2));
+        float p1 = ex2(fmaf(__uint_as_float(x[c + 1]), cs, -l2));
+        p0 = (c > lim) ? 0.f : p0 * (__uint_as_float(y[c]) - dd);
+        p1 = (c + 1 > lim) ? 0.f : p1 * (__uint_as_float(y[c + 1]) - dd);
+        pk[c >> 1] = pack_bf16(p0, p1);
       }
+      tmem_st32(tmem + lane_off + C::T_S + 64 * b, pk);  // dS_j (bf16) over the first 32 columns
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(ds_ready);
+      mbar_arrive(ds_ready(b));
     }
     // ---------------------------------------------------------------- epilogue: dQ
     if (ok && nblk > 0) ok = __all_sync(0xffffffffu, mbar_wait(dq_done, 0, wc));

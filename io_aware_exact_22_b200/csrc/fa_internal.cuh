@@ -80,7 +80,7 @@ cudaError_t launch_bwd_main(int d, const CUtensorMap& tq, const CUtensorMap& tk,
                             const CUtensorMap& tdq, const BwdArgs& a, cudaStream_t stream,
                             bool with_dq = true);
 // Deterministic dQ (query-tile-outer, accumulated in TMEM, written once): tq/tdo with 128-row
-// boxes, tk/tv with 128-row boxes, tdq the bf16 dQ with 32-row boxes; needs a.ld filled.
+// boxes, tk/tv with 64-row boxes, tdq the bf16 dQ with 32-row boxes; needs a.ld filled.
 cudaError_t launch_bwd_dq(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a,
                           cudaStream_t stream);
