@@ -56,6 +56,23 @@ def dist_env():
     return world, rank, local
 
 
+def max_over_ranks(vals, device=None):
+    """Each value's maximum over all ranks of the default process group (the values unchanged
+    without one).  Timings are reported as the slowest rank's."""
+    import torch.distributed as dist
+    vals = [float(x) for x in vals]
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return vals
+    t = torch.tensor(vals, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_tflops(flops_per_rank_step: float, world: int, ms_per_step: float) -> float:
+    """Aggregate throughput: the work of all ranks over the slowest rank's time per step."""
+    return flops_per_rank_step * world / (ms_per_step * 1e-3) / 1e12
+
+
 def step_workload(wid: int):
     w = WORKLOADS[wid]
     # the step is forward + backward at this shape; dO ~ N(0,1) is drawn after q, k, v
@@ -202,13 +219,10 @@ def run_gpu(args):
     total_ms = t0.elapsed_time(t1)
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
-    if world > 1:
-        t = torch.tensor([total_ms, fwd_ms, bwd_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms, fwd_ms, bwd_ms = t.tolist()
+    total_ms, fwd_ms, bwd_ms = max_over_ranks([total_ms, fwd_ms, bwd_ms], dev)
     ms_per_step = total_ms / args.steps
     flops_step = w.fwd_flops() + w.bwd_flops()
-    value = flops_step * world / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_tflops(flops_step, world, ms_per_step)
 
     # ------------------------------------------------------------ end-to-end (host buffers)
     # Every step copies its inputs from pinned host memory and its results back, through the
@@ -273,12 +287,8 @@ def run_gpu(args):
         stream.wait_event(ev_down[(k_e2e - 1) & 1])
         a1.record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = a0.elapsed_time(a1) / k_e2e
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e_ms = t.item()
-        e2e = {"value": flops_step * world / (e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+        e_ms = max_over_ranks([a0.elapsed_time(a1) / k_e2e], dev)[0]
+        e2e = {"value": whole_job_tflops(flops_step, world, e_ms), "unit": "TFLOPS",
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": k_e2e, "pipelined": "3 streams, double-buffered device tensors",
                "api": "io_aware_exact_22_b200.fa.fa_fwd/fa_bwd from pinned host"}
