@@ -544,8 +544,12 @@ cudaError_t launch_fwd_fp8(int d, const CUtensorMap& tq, const CUtensorMap& tk, 
 // of "Flash Attention" (special-jiahao.github.io), section 增量求解 softmax, applied to nsplit
 // blocks: with M = max_s LSE_s and weights w_s = e^{LSE_s - M} (each block's sum rescaled to
 // the common max), O = sum_s w_s O_s / sum_s w_s and LSE = M + ln sum_s w_s.  Splits with
-// LSE_s = -inf hold no visible key and are skipped.  One warp per row; lane holds D/32 columns.
-template <int D>
+// LSE_s = -inf hold no visible key and contribute nothing; their partial rows are never
+// written.  One warp per row; lane holds D/32 columns.  S > 0: exactly S splits, with every
+// load of the row issued before any is used (the empty splits' rows are read, inside the
+// workspace, and their terms dropped by a select, so stale values never reach the sum);
+// S = 0: any number of splits, the empty ones skipped by a branch.
+template <int D, int S>
 __global__ void __launch_bounds__(256) fa_fwd_merge_kernel(const float* __restrict__ o_part,
                                                            const float* __restrict__ lse_part,
                                                            __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
@@ -553,6 +557,52 @@ __global__ void __launch_bounds__(256) fa_fwd_merge_kernel(const float* __restri
   constexpr int V = D / 32;
   const int lane = threadIdx.x & 31;
   const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  if constexpr (S > 0) {
+    for (long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < rows; row += nw) {
+      float L[S];
+      float x[S][V];
+#pragma unroll
+      for (int sp = 0; sp < S; ++sp) L[sp] = lse_part[sp * rows + row];
+#pragma unroll
+      for (int sp = 0; sp < S; ++sp) {
+        const float* src = o_part + ((size_t)sp * rows + row) * D + lane * V;
+        if (V == 4) {
+          const float4 t = *reinterpret_cast<const float4*>(src);
+          x[sp][0] = t.x, x[sp][1] = t.y, x[sp][2 % V] = t.z, x[sp][3 % V] = t.w;
+        } else {
+          const float2 t = *reinterpret_cast<const float2*>(src);
+          x[sp][0] = t.x, x[sp][1] = t.y;
+        }
+      }
+      float m = L[0];
+#pragma unroll
+      for (int sp = 1; sp < S; ++sp) m = fmaxf(m, L[sp]);
+      float acc[V];
+#pragma unroll
+      for (int e = 0; e < V; ++e) acc[e] = 0.f;
+      float wsum = 0.f;
+#pragma unroll
+      for (int sp = 0; sp < S; ++sp) {
+        const bool live = (L[sp] != -INFINITY);
+        const float w = live ? expf(L[sp] - m) : 0.f;
+        wsum += w;
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[e] = live ? fmaf(w, x[sp][e], acc[e]) : acc[e];
+      }
+      const float inv = (wsum > 0.f) ? 1.f / wsum : 0.f;
+      __nv_bfloat16* dst = o + (size_t)row * D + lane * V;
+      if (V == 4) {
+        uint2 u;
+        u.x = pack_bf16(acc[0] * inv, acc[1] * inv);
+        u.y = pack_bf16(acc[2 % V] * inv, acc[3 % V] * inv);
+        *reinterpret_cast<uint2*>(dst) = u;
+      } else {
+        *reinterpret_cast<uint32_t*>(dst) = pack_bf16(acc[0] * inv, acc[1] * inv);
+      }
+      if (lane == 0) lse[row] = (wsum > 0.f) ? m + logf(wsum) : -INFINITY;
+    }
+    return;
+  }
   for (long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < rows; row += nw) {
     float m = -INFINITY;
     for (int sp = 0; sp < nsplit; ++sp) m = fmaxf(m, lse_part[sp * rows + row]);
@@ -596,10 +646,24 @@ cudaError_t launch_fwd_merge(const float* o_part, const float* lse_part, void* o
   if (blocks > 148LL * 16) blocks = 148LL * 16;
   if (blocks < 1) blocks = 1;
   auto* out = reinterpret_cast<__nv_bfloat16*>(o);
-  if (d == 64)
-    fa_fwd_merge_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(o_part, lse_part, out, lse, nsplit, rows);
-  else
-    fa_fwd_merge_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(o_part, lse_part, out, lse, nsplit, rows);
+  const unsigned g = (unsigned)blocks;
+#define FA_MERGE(DD, SS) fa_fwd_merge_kernel<DD, SS><<<g, 256, 0, stream>>>(o_part, lse_part, out, lse, nsplit, rows)
+  if (d == 64) {
+    switch (nsplit) {
+      case 2: FA_MERGE(64, 2); break;
+      case 3: FA_MERGE(64, 3); break;
+      case 4: FA_MERGE(64, 4); break;
+      default: FA_MERGE(64, 0);
+    }
+  } else {
+    switch (nsplit) {
+      case 2: FA_MERGE(128, 2); break;
+      case 3: FA_MERGE(128, 3); break;
+      case 4: FA_MERGE(128, 4); break;
+      default: FA_MERGE(128, 0);
+    }
+  }
+#undef FA_MERGE
   return cudaGetLastError();
 }
 
