@@ -601,42 +601,42 @@ __global__ void __launch_bounds__(256) fa_fwd_merge_kernel(const float* __restri
       }
       if (lane == 0) lse[row] = (wsum > 0.f) ? m + logf(wsum) : -INFINITY;
     }
-    return;
-  }
-  for (long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < rows; row += nw) {
-    float m = -INFINITY;
-    for (int sp = 0; sp < nsplit; ++sp) m = fmaxf(m, lse_part[sp * rows + row]);
-    float acc[V];
-#pragma unroll
-    for (int e = 0; e < V; ++e) acc[e] = 0.f;
-    float wsum = 0.f;
-    if (m != -INFINITY) {
-      for (int sp = 0; sp < nsplit; ++sp) {
-        const float L = lse_part[sp * rows + row];
-        if (L == -INFINITY) continue;
-        const float w = expf(L - m);
-        wsum += w;
-        const float* src = o_part + ((size_t)sp * rows + row) * D + lane * V;
-        if (V == 4) {
-          const float4 x = *reinterpret_cast<const float4*>(src);
-          acc[0] += w * x.x; acc[1] += w * x.y; acc[2] += w * x.z; acc[3] += w * x.w;
-        } else {
-          const float2 x = *reinterpret_cast<const float2*>(src);
-          acc[0] += w * x.x; acc[1] += w * x.y;
+  } else {
+    for (long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < rows; row += nw) {
+      float m = -INFINITY;
+      for (int sp = 0; sp < nsplit; ++sp) m = fmaxf(m, lse_part[sp * rows + row]);
+      float acc[V];
+  #pragma unroll
+      for (int e = 0; e < V; ++e) acc[e] = 0.f;
+      float wsum = 0.f;
+      if (m != -INFINITY) {
+        for (int sp = 0; sp < nsplit; ++sp) {
+          const float L = lse_part[sp * rows + row];
+          if (L == -INFINITY) continue;
+          const float w = expf(L - m);
+          wsum += w;
+          const float* src = o_part + ((size_t)sp * rows + row) * D + lane * V;
+          if (V == 4) {
+            const float4 x = *reinterpret_cast<const float4*>(src);
+            acc[0] += w * x.x; acc[1] += w * x.y; acc[2] += w * x.z; acc[3] += w * x.w;
+          } else {
+            const float2 x = *reinterpret_cast<const float2*>(src);
+            acc[0] += w * x.x; acc[1] += w * x.y;
+          }
         }
       }
+      const float inv = (wsum > 0.f) ? 1.f / wsum : 0.f;
+      __nv_bfloat16* dst = o + (size_t)row * D + lane * V;
+      if (V == 4) {
+        uint2 u;
+        u.x = pack_bf16(acc[0] * inv, acc[1] * inv);
+        u.y = pack_bf16(acc[2] * inv, acc[3] * inv);
+        *reinterpret_cast<uint2*>(dst) = u;
+      } else {
+        *reinterpret_cast<uint32_t*>(dst) = pack_bf16(acc[0] * inv, acc[1] * inv);
+      }
+      if (lane == 0) lse[row] = (wsum > 0.f) ? m + logf(wsum) : -INFINITY;
     }
-    const float inv = (wsum > 0.f) ? 1.f / wsum : 0.f;
-    __nv_bfloat16* dst = o + (size_t)row * D + lane * V;
-    if (V == 4) {
-      uint2 u;
-      u.x = pack_bf16(acc[0] * inv, acc[1] * inv);
-      u.y = pack_bf16(acc[2] * inv, acc[3] * inv);
-      *reinterpret_cast<uint2*>(dst) = u;
-    } else {
-      *reinterpret_cast<uint32_t*>(dst) = pack_bf16(acc[0] * inv, acc[1] * inv);
-    }
-    if (lane == 0) lse[row] = (wsum > 0.f) ? m + logf(wsum) : -INFINITY;
   }
 }
 
