@@ -437,6 +437,22 @@ def measure_variants(w, dev, stream, qd, kd, vd, o, lse, dod, dq, dk, dv, ws, ws
     out["bwd_d64"] = {"kernels": "fa_bwd_main_kernel<64, no dQ> + fa_bwd_dq_kernel<64>",
                       "shape": "B=4 H=16 N=1024 d=64", "ms": round(ms, 4), "tflops": round(tf, 1),
                       "peak": peak, "frac": round(tf / peak, 4)}
+    # sequence sharded into 4 pieces (ring schedule), every rank's pieces on this GPU in turn:
+    # the partial-result and merge overhead of sharding, without the exchange
+    from io_aware_exact_22_b200 import ring
+    W = 4
+    if N % W == 0:
+        n = N // W
+        shard = lambda t: [t[:, :, r * n:(r + 1) * n].contiguous() for r in range(W)]  # noqa: E731
+        qs, ks, vs = shard(qd), shard(kd), shard(vd)
+        ms = _time_ms(lambda: ring.ring_attention_forward_local(qs, ks, vs, w.causal, w.scale), stream,
+                      iters=5)
+        tf = w.fwd_flops() / (ms * 1e-3) / 1e12
+        out["fwd_ring_sharded_on_one_gpu"] = {
+            "kernels": "fa_fwd_kernel<128, partial> per (rank, visible shard) + fa_fwd_merge_kernel<128>",
+            "shape": f"{w.name}, {W} shards of {n}", "ms": round(ms, 4), "tflops": round(tf, 1),
+            "peak": peak, "frac": round(tf / peak, 4)}
+        del qs, ks, vs
     if fa.fa_get_device_status(sp) != 0:
         raise RuntimeError("device-side timeout while timing the variants")
     return out

@@ -121,6 +121,33 @@ fa_status_t fa_fwd_fp8(const void* q, const void* k, const void* v, const float*
                        int B, int H, int N, int d, float scale, int causal, void* stream);
 
 /*
+ * The two halves of the split-KV forward, for callers that hold the keys in pieces (for
+ * instance one piece per GPU of a sequence sharded across GPUs).
+ *
+ * fa_fwd_partial: attention of q over one set of keys k, v (all [B,H,N,d] bf16, the same N),
+ * returned as that key set's normalised partial result:
+ *   o_part   : out, fp32 [B,H,N,d]  O_s = softmax over these keys of scale * Q K^T, times V
+ *   lse_part : out, fp32 [B,H,N]    LSE_s, natural log (-inf for a row with no visible key)
+ * causal != 0 masks key j for query i when j > i within this key set (the diagonal piece);
+ * causal == 0 sees every key (a piece that lies entirely before the queries).  Alignment as
+ * fa_fwd, o_part 16 bytes.
+ *
+ * fa_merge_partials: combines nparts such results of the same queries with the two-block
+ * softmax merge of "Flash Attention" (special-jiahao.github.io, section 增量求解 softmax)
+ * extended to nparts blocks (M = max_s LSE_s, w_s = exp(LSE_s - M), O = sum_s w_s O_s / sum_s
+ * w_s, LSE = M + ln sum_s w_s; parts with LSE_s = -inf contribute nothing):
+ *   o_parts   : in, fp32 [nparts,B,H,N,d] contiguous (16-byte aligned)
+ *   lse_parts : in, fp32 [nparts,B,H,N]
+ *   o, lse    : out, bf16 [B,H,N,d] (16-byte aligned) and fp32 [B,H,N]
+ *   nparts    : 1 .. 1024.  d in {64, 128}.
+ */
+fa_status_t fa_fwd_partial(const void* q, const void* k, const void* v, float* o_part,
+                           float* lse_part, int B, int H, int N, int d, float scale, int causal,
+                           void* stream);
+fa_status_t fa_merge_partials(const float* o_parts, const float* lse_parts, int nparts, void* o,
+                              float* lse, int B, int H, int N, int d, void* stream);
+
+/*
  * Bytes of device workspace that fa_bwd needs: per 64-row query tile, the fp32 base-2 LSE and
  * row term D_i of its 64 rows (B*H*ceil(N/64)*128 floats, rounded up to 256 bytes), followed
  * by the fp32 dQ accumulator [B*H*N*d].  Returns 0 for an empty or invalid shape.

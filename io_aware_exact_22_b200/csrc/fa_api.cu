@@ -389,6 +389,49 @@ fa_status_t fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o,
   return FA_OK;
 }
 
+fa_status_t fa_fwd_partial(const void* q, const void* k, const void* v, float* o_part, float* lse_part,
+                           int B, int H, int N, int d, float scale, int causal, void* stream) {
+  bool empty = false;
+  fa_status_t st = check_shape(B, H, N, d, scale, causal, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!q || !k || !v || !o_part || !lse_part) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o_part, 16) || !aligned(lse_part, 4))
+    return FA_ERR_INVALID_ARG;
+  if ((st = check_device()) != FA_OK) return st;
+  const int BH = B * H;
+  if ((long long)BH * ((N + 255) / 256) > INT_MAX) return FA_ERR_INVALID_ARG;
+  CUtensorMap tq, tk, tv, to;
+  if (!make_tmap_bf16(&tq, q, BH, N, d, 128) || !make_tmap_bf16(&tk, k, BH, N, d, 128) ||
+      !make_tmap_bf16(&tv, v, BH, N, d, 128) || !make_tmap_f32(&to, o_part, BH, N, d, 32, 32, true))
+    return FA_ERR_CUDA;
+  FwdArgs a;
+  if (!(a.status = device_status_word())) return FA_ERR_CUDA;
+  a.lse = lse_part;
+  a.N = N;
+  a.BH = BH;
+  a.nqb = (N + 255) / 256;
+  a.causal = causal;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  a.nsplit = 1;
+  return launch_fwd_partial(d, tq, tk, tv, to, a, (cudaStream_t)stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status_t fa_merge_partials(const float* o_parts, const float* lse_parts, int nparts, void* o, float* lse,
+                              int B, int H, int N, int d, void* stream) {
+  bool empty = false;
+  fa_status_t st = check_shape(B, H, N, d, 1.0f, 0, &empty);
+  if (st != FA_OK || empty) return st;
+  if (nparts < 1 || nparts > 1024) return FA_ERR_INVALID_ARG;
+  if (!o_parts || !lse_parts || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned(o_parts, 16) || !aligned(lse_parts, 4) || !aligned(o, 16) || !aligned(lse, 4))
+    return FA_ERR_INVALID_ARG;
+  if ((st = check_device()) != FA_OK) return st;
+  const long long rows = (long long)B * H * N;
+  return launch_fwd_merge(o_parts, lse_parts, o, lse, nparts, rows, d, (cudaStream_t)stream) == cudaSuccess
+             ? FA_OK
+             : FA_ERR_CUDA;
+}
+
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
   const long long rows = (long long)B * H * N;

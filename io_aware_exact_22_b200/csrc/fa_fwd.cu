@@ -534,6 +534,12 @@ cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, cons
   return launch_fwd_t<128, false>(tq, tk, tv, to, a, stream);
 }
 
+cudaError_t launch_fwd_partial(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                               const CUtensorMap& to, const FwdArgs& a, cudaStream_t stream) {
+  if (d == 64) return launch_fwd_t<64, true>(tq, tk, tv, to, a, stream);
+  return launch_fwd_t<128, true>(tq, tk, tv, to, a, stream);
+}
+
 cudaError_t launch_fwd_fp8(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            const CUtensorMap& to, const FwdArgs& a, cudaStream_t stream) {
   if (d != 128 || a.nsplit != 1) return cudaErrorNotSupported;

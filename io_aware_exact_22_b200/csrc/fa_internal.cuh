@@ -60,6 +60,10 @@ bool encode_tmap_f32(CUtensorMap* m, const void* ptr, int BH, int N, int d, int 
 // outputs [nsplit * BH, N, d] (box 32 x 32, 128-byte swizzle) and a.lse the partial LSEs.
 cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& to, const FwdArgs& a, cudaStream_t stream);
+// Partial outputs (fp32 O / l and LSE) for a.nsplit >= 1 key ranges, whatever a.nsplit is; `to`
+// maps the fp32 partials [a.nsplit * BH, N, d].
+cudaError_t launch_fwd_partial(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                               const CUtensorMap& to, const FwdArgs& a, cudaStream_t stream);
 // FP8 (E4M3) inputs, d = 128, whole key range; Q/K/V maps from make_tmap_e4m3 (128-row boxes)
 cudaError_t launch_fwd_fp8(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            const CUtensorMap& to, const FwdArgs& a, cudaStream_t stream);

@@ -24,7 +24,7 @@ STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_E
 EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_device_status",
            "fa_status_string", "fa_version", "fa_bwd_noalloc", "fa_selftest_wait_timeout",
            "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_default_splits",
-           "fa_bwd_deterministic", "fa_fwd_fp8")
+           "fa_bwd_deterministic", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials")
 # Size of the library's built-in scratch used by fa_bwd_noalloc (include/fa.h).
 NOALLOC_MAX_SCRATCH_BYTES = 64 << 20
 
@@ -50,6 +50,10 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd.restype = i
         L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
         L.fa_fwd_fp8.restype = i
+        L.fa_fwd_partial.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+        L.fa_fwd_partial.restype = i
+        L.fa_merge_partials.argtypes = [vp, vp, i, vp, vp, i, i, i, i, vp]
+        L.fa_merge_partials.restype = i
         L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, vp]
         L.fa_bwd.restype = i
         L.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
@@ -103,6 +107,16 @@ def fa_fwd_fp8(q, k, v, descale_q, descale_k, descale_v, o, lse, B, H, N, d, sca
     return lib().fa_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(descale_q), _ptr(descale_k),
                             _ptr(descale_v), _ptr(o), _ptr(lse), B, H, N, d, float(scale),
                             int(causal), _stream(stream))
+
+
+def fa_fwd_partial(q, k, v, o_part, lse_part, B, H, N, d, scale, causal, stream=None) -> int:
+    return lib().fa_fwd_partial(_ptr(q), _ptr(k), _ptr(v), _ptr(o_part), _ptr(lse_part), B, H, N, d,
+                                float(scale), int(causal), _stream(stream))
+
+
+def fa_merge_partials(o_parts, lse_parts, nparts, o, lse, B, H, N, d, stream=None) -> int:
+    return lib().fa_merge_partials(_ptr(o_parts), _ptr(lse_parts), int(nparts), _ptr(o), _ptr(lse), B, H,
+                                   N, d, _stream(stream))
 
 
 def fa_fwd_splitkv(q, k, v, o, lse, B, H, N, d, scale, causal, num_splits, workspace,

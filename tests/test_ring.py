@@ -1,0 +1,125 @@
+"""Sequence-sharded forward (io_aware_exact_22_b200.ring): K/V shards passed around a ring of
+ranks, partial results merged by the softmax merge of "Flash Attention" (special-jiahao.github.io,
+section 增量求解 softmax).
+
+On CPU: the ring exchange itself on spawned gloo ranks (every rank sees every shard, in ring
+order, with the right contents), the choice of pieces under the causal mask, and the C ABI's
+argument checks.  On one GPU: the whole schedule for W virtual ranks, one after the other,
+against the fp64 oracle over the full sequence (the multi-GPU run differs only in where the
+shards come from)."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle
+from io_aware_exact_22_b200 import fa, ring
+from io_aware_exact_22_b200.inputs import custom, make_inputs, to_f64
+from tests._helpers import check_lse, check_o, f64
+
+OK, INVALID, UNSUPPORTED = 0, 1, 2
+A16 = 0x10000
+
+
+def test_visible_shards():
+    assert ring.visible_shards(2, 4, False) == {0: False, 1: False, 2: False, 3: False}
+    assert ring.visible_shards(0, 4, True) == {0: True}
+    assert ring.visible_shards(3, 4, True) == {0: False, 1: False, 2: False, 3: True}
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        k = torch.full((2, 3), float(rank))
+        v = torch.full((2, 3), 100.0 + rank)
+        seen = [(src, float(ks[0, 0]), float(vs[1, 2])) for src, ks, vs in ring.ring_shards(k, v)]
+        q.put((rank, seen))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3, 4])
+def test_ring_exchange_on_gloo_ranks(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = dict(q.get(timeout=10) for _ in range(world))
+    for r in range(world):
+        want = [((r - s) % world, float((r - s) % world), 100.0 + (r - s) % world) for s in range(world)]
+        assert res[r] == want
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), INVALID), (dict(o=0), INVALID), (dict(o=A16 + 8), INVALID), (dict(lse=0), INVALID),
+    (dict(d=80), UNSUPPORTED), (dict(scale=-1.0), INVALID), (dict(causal=5), INVALID)])
+def test_partial_rejects_bad_arguments(kw, code):
+    a = dict(q=A16, k=A16, v=A16, o=A16, lse=A16, B=1, H=2, N=256, d=128, scale=0.1, causal=0)
+    a.update(kw)
+    assert fa.fa_fwd_partial(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["N"], a["d"],
+                             a["scale"], a["causal"], 0) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n=0), INVALID), (dict(n=2000), INVALID), (dict(op=0), INVALID), (dict(op=A16 + 4), INVALID),
+    (dict(o=A16 + 8), INVALID), (dict(d=96), UNSUPPORTED)])
+def test_merge_rejects_bad_arguments(kw, code):
+    a = dict(op=A16, lp=A16, n=2, o=A16, lse=A16, B=1, H=2, N=256, d=128)
+    a.update(kw)
+    assert fa.fa_merge_partials(a["op"], a["lp"], a["n"], a["o"], a["lse"], a["B"], a["H"], a["N"],
+                                a["d"], 0) == code
+
+
+def test_empty_problems_are_no_ops():
+    assert fa.fa_fwd_partial(A16, A16, A16, A16, A16, 1, 0, 64, 128, 0.1, 0, 0) == OK
+    assert fa.fa_merge_partials(A16, A16, 3, A16, A16, 1, 2, 0, 64, 0) == OK
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("W,n,d", [(2, 128, 128), (3, 200, 128), (4, 384, 64), (2, 1, 128), (5, 129, 64)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_ring_schedule_on_one_gpu(cuda_ok, W, n, d, causal):
+    w = custom(1, 2, W * n, d, causal, seed=W * 1000 + n)
+    q, k, v = make_inputs(w, with_grad=False)
+    shard = lambda t: [t[:, :, r * n:(r + 1) * n].contiguous().cuda() for r in range(W)]  # noqa: E731
+    outs = ring.ring_attention_forward_local(shard(q), shard(k), shard(v), causal, w.scale)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status() == 0
+    o_ref, lse_ref = oracle.attention_forward(to_f64(q), to_f64(k), to_f64(v), w.scale, causal)
+    o = np.concatenate([f64(x[0]) for x in outs], axis=2)
+    lse = np.concatenate([f64(x[1]) for x in outs], axis=2)
+    check_o(o, o_ref)
+    check_lse(lse, lse_ref)
+
+
+@pytest.mark.gpu
+def test_one_part_is_the_forward(cuda_ok):
+    w = custom(2, 3, 700, 128, True, seed=4)
+    q, k, v = (t.cuda() for t in make_inputs(w, with_grad=False))
+    B, H, N, d = w.shape
+    po = torch.empty((1, B, H, N, d), device="cuda")
+    pl = torch.empty((1, B, H, N), device="cuda")
+    assert fa.fa_fwd_partial(q, k, v, po, pl, B, H, N, d, w.scale, 1) == OK
+    o, lse = torch.empty_like(q), torch.empty((B, H, N), device="cuda")
+    assert fa.fa_merge_partials(po, pl, 1, o, lse, B, H, N, d) == OK
+    o2, l2 = fa.forward(q, k, v, True, w.scale)
+    torch.cuda.synchronize()
+    assert (o.float() - o2.float()).abs().max().item() <= 8e-3
+    assert (lse - l2).abs().max().item() <= 1e-5
+    assert torch.equal(lse, pl[0])
