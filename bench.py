@@ -452,6 +452,19 @@ def measure_variants(w, dev, stream, qd, kd, vd, o, lse, dod, dq, dk, dv, ws, ws
             "kernels": "fa_fwd_kernel<128, partial> per (rank, visible shard) + fa_fwd_merge_kernel<128>",
             "shape": f"{w.name}, {W} shards of {n}", "ms": round(ms, 4), "tflops": round(tf, 1),
             "peak": peak, "frac": round(tf / peak, 4)}
+        if d == 128:
+            fw = ring.ring_attention_forward_local(qs, ks, vs, w.causal, w.scale)
+            os_, ls_ = [x[0] for x in fw], [x[1] for x in fw]
+            dos = shard(dod)
+            ms = _time_ms(lambda: ring.ring_attention_backward_local(qs, ks, vs, os_, dos, ls_, w.causal, w.scale),
+                          stream, warmup=3, iters=3)
+            tf = w.bwd_flops() / (ms * 1e-3) / 1e12
+            out["bwd_ring_sharded_on_one_gpu"] = {
+                "kernels": "fa_bwd_pre_kernel per rank + fa_bwd_main_kernel<128> (accumulate) per (rank, "
+                           "visible shard) + fa_bwd_post_kernel x 3 per rank",
+                "shape": f"{w.name}, {W} shards of {n}", "ms": round(ms, 4), "tflops": round(tf, 1),
+                "peak": peak, "frac": round(tf / peak, 4)}
+            del fw, os_, ls_, dos
         del qs, ks, vs
     if fa.fa_get_device_status(sp) != 0:
         raise RuntimeError("device-side timeout while timing the variants")

@@ -211,6 +211,31 @@ fa_status_t fa_bwd_deterministic(const void* q, const void* k, const void* v, co
                                  int B, int H, int N, int d, float scale, int causal, void* stream);
 
 /*
+ * The backward in three steps, for callers that hold the keys in pieces (the sequence-sharded
+ * backward: every key set's contribution is added in turn).  d == 128.  The workspace has
+ * fa_bwd's layout and size; dk_acc, dv_acc are caller-owned fp32 [B,H,N,d] accumulators
+ * (16-byte aligned) for the keys of one piece, zeroed by the caller before the first addition.
+ *   fa_bwd_prepare    : from this rank's o, dO (bf16) and lse (fp32), the per-row statistics
+ *                       (LSE * log2 e, D_i = rowsum(dO o O)) into the workspace, and its fp32
+ *                       dQ accumulator zeroed.
+ *   fa_bwd_accumulate : the contribution of one key set k, v (same N) to the gradients of these
+ *                       queries: dQ added into the workspace's accumulator (fp32 reductions),
+ *                       scale * dK and dV added into dk_acc and dv_acc.  causal != 0 applies the
+ *                       mask within the key set (the diagonal piece); 0 sees every key.
+ *   fa_bwd_finish     : dq = scale * accumulator, dk = dk_acc, dv = dv_acc, rounded to bf16.
+ * Summed over all key sets, the results are fa_bwd's (up to summation order).
+ */
+fa_status_t fa_bwd_prepare(const void* o, const void* dO, const float* lse, void* workspace,
+                           size_t workspace_bytes, int B, int H, int N, int d, void* stream);
+fa_status_t fa_bwd_accumulate(const void* q, const void* k, const void* v, const void* dO,
+                              void* workspace, size_t workspace_bytes, float* dk_acc,
+                              float* dv_acc, int B, int H, int N, int d, float scale, int causal,
+                              void* stream);
+fa_status_t fa_bwd_finish(const void* workspace, size_t workspace_bytes, const float* dk_acc,
+                          const float* dv_acc, void* dq, void* dk, void* dv,
+                          int B, int H, int N, int d, float scale, void* stream);
+
+/*
  * Synchronises `stream`, reads and clears the device status word of the current device.
  * Returns FA_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call,
  * FA_ERR_CUDA if the synchronisation itself failed, FA_OK otherwise.

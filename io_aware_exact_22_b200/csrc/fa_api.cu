@@ -486,6 +486,83 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
   return FA_OK;
 }
 
+fa_status_t fa_bwd_prepare(const void* o, const void* dO, const float* lse, void* workspace, size_t workspace_bytes,
+                           int B, int H, int N, int d, void* stream) {
+  bool empty = false;
+  fa_status_t st = check_shape(B, H, N, d, 1.0f, 0, &empty);
+  if (st != FA_OK || empty) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (!o || !dO || !lse || !workspace) return FA_ERR_INVALID_ARG;
+  if (!aligned(o, 16) || !aligned(dO, 16) || !aligned(lse, 4) || !aligned(workspace, 256)) return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  if ((st = check_device()) != FA_OK) return st;
+  const int BH = B * H;
+  float* ld = reinterpret_cast<float*>(workspace);
+  float* dq_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + ld_bytes(BH, N));
+  return launch_bwd_pre(o, dO, lse, ld, dq_acc, BH, N, d, (cudaStream_t)stream) == cudaSuccess ? FA_OK
+                                                                                                : FA_ERR_CUDA;
+}
+
+fa_status_t fa_bwd_accumulate(const void* q, const void* k, const void* v, const void* dO, void* workspace,
+                              size_t workspace_bytes, float* dk_acc, float* dv_acc, int B, int H, int N, int d,
+                              float scale, int causal, void* stream) {
+  bool empty = false;
+  fa_status_t st = check_shape(B, H, N, d, scale, causal, &empty);
+  if (st != FA_OK || empty) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !dO || !workspace || !dk_acc || !dv_acc) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dO, 16) || !aligned(workspace, 256) ||
+      !aligned(dk_acc, 16) || !aligned(dv_acc, 16))
+    return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  if ((st = check_device()) != FA_OK) return st;
+  const int BH = B * H;
+  float* ld = reinterpret_cast<float*>(workspace);
+  float* dq_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + ld_bytes(BH, N));
+  CUtensorMap tq, tk, tv, tdo, tdq;
+  if (!make_tmap_bf16(&tq, q, BH, N, d, 64) || !make_tmap_bf16(&tk, k, BH, N, d, 128) ||
+      !make_tmap_bf16(&tv, v, BH, N, d, 128) || !make_tmap_bf16(&tdo, dO, BH, N, d, 64) ||
+      !make_tmap_f32(&tdq, dq_acc, BH, N, d, 32, 64 - kBwdDqRedRows))
+    return FA_ERR_CUDA;
+  BwdArgs a;
+  if (!(a.status = device_status_word())) return FA_ERR_CUDA;
+  a.lse = nullptr;
+  a.ld = ld;
+  a.dq_acc = dq_acc;
+  a.dk_acc = dk_acc;
+  a.dv_acc = dv_acc;
+  a.N = N;
+  a.BH = BH;
+  a.causal = causal;
+  a.scale = scale;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  // the dK/dV store maps are not used in accumulate mode; any valid map fills the parameters
+  return launch_bwd_main(d, tq, tk, tv, tdo, tk, tv, tdq, a, (cudaStream_t)stream) == cudaSuccess ? FA_OK
+                                                                                                  : FA_ERR_CUDA;
+}
+
+fa_status_t fa_bwd_finish(const void* workspace, size_t workspace_bytes, const float* dk_acc, const float* dv_acc,
+                          void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, void* stream) {
+  bool empty = false;
+  fa_status_t st = check_shape(B, H, N, d, scale, 0, &empty);
+  if (st != FA_OK || empty) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (!workspace || !dk_acc || !dv_acc || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256) || !aligned(dk_acc, 16) || !aligned(dv_acc, 16) || !aligned(dq, 16) ||
+      !aligned(dk, 16) || !aligned(dv, 16))
+    return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  if ((st = check_device()) != FA_OK) return st;
+  const long long elems = (long long)B * H * N * d;
+  const float* dq_acc =
+      reinterpret_cast<const float*>(reinterpret_cast<const char*>(workspace) + ld_bytes((long long)B * H, N));
+  cudaStream_t s = (cudaStream_t)stream;
+  if (launch_bwd_post(dq_acc, dq, elems, scale, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (launch_bwd_post(dk_acc, dk, elems, 1.0f, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (launch_bwd_post(dv_acc, dv, elems, 1.0f, s) != cudaSuccess) return FA_ERR_CUDA;
+  return FA_OK;
+}
+
 fa_status_t fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o, const void* dO,
                                  const float* lse, void* dq, void* dk, void* dv, void* workspace,
                                  size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,

@@ -490,7 +490,34 @@ __global__ void __launch_bounds__(448, 1)
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     bool ok = !*abort_flag;
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(kv_done, 0, wc));
-    if (ok) {
+    if (ok && a.dk_acc != nullptr) {
+      // accumulate mode: add this key row's scale * dK (or dV) into the fp32 accumulator row;
+      // this CTA is the only one touching these rows in this call
+      tc_fence_after();
+      const float mul = is_dk ? a.scale : 1.f;
+      const uint32_t src = tmem + lane_off + (is_dk ? C::T_DK : C::T_DV);
+      const int key = 128 * j + r;
+      float* accrow = (is_dk ? a.dk_acc : a.dv_acc) + ((size_t)bh * a.N + key) * C::D;
+#pragma unroll 1
+      for (int c32 = 0; c32 < C::D; c32 += 32) {
+        uint32_t o[32];
+        tmem_ld32(src + c32, o);
+        tmem_wait_ld();
+        reg_fence(o);
+        if (key < a.N && count > 0) {
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            float4* pa = reinterpret_cast<float4*>(accrow + c32 + 4 * cc);
+            float4 g = *pa;
+            g.x += __uint_as_float(o[4 * cc + 0]) * mul;
+            g.y += __uint_as_float(o[4 * cc + 1]) * mul;
+            g.z += __uint_as_float(o[4 * cc + 2]) * mul;
+            g.w += __uint_as_float(o[4 * cc + 3]) * mul;
+            *pa = g;
+          }
+        }
+      }
+    } else if (ok) {
       tc_fence_after();
       const float mul = is_dk ? a.scale : 1.f;
       const uint32_t src = tmem + lane_off + (is_dk ? C::T_DK : C::T_DV);

@@ -33,6 +33,10 @@ struct BwdArgs {
   int causal;
   float scale;       // softmax scale
   float scale_log2;  // scale * log2(e)
+  // When set (d = 128, with the dQ path): scale * dK and dV of this call are added into these
+  // fp32 [BH, N, d] accumulators instead of being stored as bf16 (the sequence-sharded backward)
+  float* dk_acc = nullptr;
+  float* dv_acc = nullptr;
 };
 
 // Backward dQ accumulation: of each 64-row query tile, the first kBwdDqRedRows rows are added

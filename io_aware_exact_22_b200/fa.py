@@ -24,7 +24,8 @@ STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_E
 EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_device_status",
            "fa_status_string", "fa_version", "fa_bwd_noalloc", "fa_selftest_wait_timeout",
            "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_default_splits",
-           "fa_bwd_deterministic", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials")
+           "fa_bwd_deterministic", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials",
+           "fa_bwd_prepare", "fa_bwd_accumulate", "fa_bwd_finish")
 # Size of the library's built-in scratch used by fa_bwd_noalloc (include/fa.h).
 NOALLOC_MAX_SCRATCH_BYTES = 64 << 20
 
@@ -54,6 +55,12 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd_partial.restype = i
         L.fa_merge_partials.argtypes = [vp, vp, i, vp, vp, i, i, i, i, vp]
         L.fa_merge_partials.restype = i
+        L.fa_bwd_prepare.argtypes = [vp, vp, vp, vp, sz, i, i, i, i, vp]
+        L.fa_bwd_prepare.restype = i
+        L.fa_bwd_accumulate.argtypes = [vp, vp, vp, vp, vp, sz, vp, vp, i, i, i, i, f, i, vp]
+        L.fa_bwd_accumulate.restype = i
+        L.fa_bwd_finish.argtypes = [vp, sz, vp, vp, vp, vp, vp, i, i, i, i, f, vp]
+        L.fa_bwd_finish.restype = i
         L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, vp]
         L.fa_bwd.restype = i
         L.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
@@ -117,6 +124,24 @@ def fa_fwd_partial(q, k, v, o_part, lse_part, B, H, N, d, scale, causal, stream=
 def fa_merge_partials(o_parts, lse_parts, nparts, o, lse, B, H, N, d, stream=None) -> int:
     return lib().fa_merge_partials(_ptr(o_parts), _ptr(lse_parts), int(nparts), _ptr(o), _ptr(lse), B, H,
                                    N, d, _stream(stream))
+
+
+def fa_bwd_prepare(o, dO, lse, workspace, workspace_bytes, B, H, N, d, stream=None) -> int:
+    return lib().fa_bwd_prepare(_ptr(o), _ptr(dO), _ptr(lse), _ptr(workspace), int(workspace_bytes), B, H,
+                                N, d, _stream(stream))
+
+
+def fa_bwd_accumulate(q, k, v, dO, workspace, workspace_bytes, dk_acc, dv_acc, B, H, N, d, scale,
+                      causal, stream=None) -> int:
+    return lib().fa_bwd_accumulate(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(workspace),
+                                   int(workspace_bytes), _ptr(dk_acc), _ptr(dv_acc), B, H, N, d,
+                                   float(scale), int(causal), _stream(stream))
+
+
+def fa_bwd_finish(workspace, workspace_bytes, dk_acc, dv_acc, dq, dk, dv, B, H, N, d, scale,
+                  stream=None) -> int:
+    return lib().fa_bwd_finish(_ptr(workspace), int(workspace_bytes), _ptr(dk_acc), _ptr(dv_acc),
+                               _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale), _stream(stream))
 
 
 def fa_fwd_splitkv(q, k, v, o, lse, B, H, N, d, scale, causal, num_splits, workspace,

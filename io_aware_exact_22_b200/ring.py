@@ -1,4 +1,4 @@
-"""Sequence-sharded exact attention, forward: K/V shards passed around a ring of ranks.
+"""Sequence-sharded exact attention: K/V shards passed around a ring of ranks.
 
 Rank r of W holds the r-th contiguous shard of the sequence of q, k and v (each [B, H, n, d],
 global positions [r n, r n + n)).  The K/V shards travel around the ring (rank r sends to
@@ -9,6 +9,11 @@ its queries, with the causal mask for its own shard, skipped for shards after it
 fa_merge_partials then combines the partial results by the softmax merge of "Flash Attention"
 (special-jiahao.github.io, section 增量求解 softmax), which is what makes the pieces add up to
 exact attention over the whole sequence.
+
+The backward passes each K/V shard round the ring together with fp32 accumulators for its
+dK and dV: every rank adds its queries' contribution (fa_bwd_accumulate, which also adds into
+the rank's own dQ accumulator) before handing the shard on, and one more hop brings every
+shard's accumulators back to its owner, which rounds them to bf16 (fa_bwd_finish).
 
 The exchange has no multicast and no library kernel touches another GPU's memory: each shard
 is received into this rank's own buffers before it is read.  Causal sharding by contiguous
@@ -115,3 +120,97 @@ def ring_attention_forward_local(q_shards, k_shards, v_shards, causal: bool,
         order = [((r - step) % W, k_shards[(r - step) % W], v_shards[(r - step) % W]) for step in range(W)]
         outs.append(_accumulate(q_shards[r], iter(order), r, W, causal, sc, o, l))
     return outs
+
+
+# ------------------------------------------------------------------------------ backward
+def ring_round(tensors, group=None):
+    """Passes a list of tensors (a K/V shard and its gradient accumulators) round the ring.
+    Yields (step, src, held) for step 0 .. W-1, held being the list of rank src = r - step (its
+    own first); after each yield, when the caller has added into the held accumulators, the held
+    list is sent on to rank r+1 and the next one received from rank r-1.  After the last step
+    the list held is this rank's own again; it is yielded once more with step == W."""
+    W = dist.get_world_size(group)
+    r = dist.get_rank(group)
+    nxt, prv = _peer(group, (r + 1) % W), _peer(group, (r - 1) % W)
+    cur = list(tensors)
+    bufs = [[torch.empty_like(t) for t in cur] for _ in range(2)] if W > 1 else []
+    for step in range(W):
+        yield step, (r - step) % W, cur
+        if W > 1:
+            nb = bufs[step % 2]
+            ops = [dist.P2POp(dist.isend, t, nxt, group) for t in cur]
+            ops += [dist.P2POp(dist.irecv, t, prv, group) for t in nb]
+            for rq in dist.batch_isend_irecv(ops):
+                rq.wait()
+            cur = nb
+    yield W, r, cur
+
+
+def _check_bwd(*ts):
+    for t in ts:
+        if not (t.is_cuda and t.is_contiguous() and t.dim() == 4 and t.shape[-1] == 128):
+            raise ValueError("the sharded backward takes contiguous CUDA tensors [B,H,n,128]")
+
+
+def ring_attention_backward(q, k, v, o, do, lse, causal: bool, scale: float | None = None,
+                            group=None, dq=None, dk=None, dv=None):
+    """dQ, dK, dV of this rank's shards.  q, k, v, o, do: this rank's bf16 [B, H, n, 128]
+    shards; lse: its fp32 [B, H, n] from ring_attention_forward.  Collective over `group`."""
+    _check_bwd(q, k, v, o, do)
+    B, H, n, d = q.shape
+    scale = d ** -0.5 if scale is None else scale
+    W, r = dist.get_world_size(group), dist.get_rank(group)
+    wsb = fa.fa_bwd_workspace_bytes(B, H, n, d)
+    ws = torch.empty(wsb, device=q.device, dtype=torch.uint8)
+    _ok(fa.fa_bwd_prepare(o, do, lse, ws, wsb, B, H, n, d), "fa_bwd_prepare")
+    acc = [torch.zeros(q.shape, device=q.device, dtype=torch.float32) for _ in range(2)]
+    vis = visible_shards(r, W, causal)
+    home = None
+    for step, src, (ks, vs, dka, dva) in ring_round([k, v, acc[0], acc[1]], group):
+        if step == W:
+            home = (dka, dva)
+            break
+        if src in vis:
+            _ok(fa.fa_bwd_accumulate(q, ks, vs, do, ws, wsb, dka, dva, B, H, n, d, scale, vis[src]),
+                "fa_bwd_accumulate")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    _ok(fa.fa_bwd_finish(ws, wsb, home[0], home[1], dq, dk, dv, B, H, n, d, scale), "fa_bwd_finish")
+    return dq, dk, dv
+
+
+def ring_attention_backward_local(q_shards, k_shards, v_shards, o_shards, do_shards, lse_shards,
+                                  causal: bool, scale: float | None = None):
+    """The same computation for all W shards on one device: every rank's contributions in its
+    ring order, each shard's accumulators shared instead of passed on.  Returns
+    [(dQ_r, dK_r, dV_r)]."""
+    W = len(q_shards)
+    _check_bwd(*q_shards, *k_shards, *v_shards, *o_shards, *do_shards)
+    B, H, n, d = q_shards[0].shape
+    scale = d ** -0.5 if scale is None else scale
+    wsb = fa.fa_bwd_workspace_bytes(B, H, n, d)
+    wss = [torch.empty(wsb, device=q_shards[0].device, dtype=torch.uint8) for _ in range(W)]
+    dka = [torch.zeros(q_shards[0].shape, device=q_shards[0].device, dtype=torch.float32) for _ in range(W)]
+    dva = [torch.zeros_like(t) for t in dka]
+    for r in range(W):
+        _ok(fa.fa_bwd_prepare(o_shards[r], do_shards[r], lse_shards[r], wss[r], wsb, B, H, n, d),
+            "fa_bwd_prepare")
+    for r in range(W):
+        vis = visible_shards(r, W, causal)
+        for step in range(W):
+            src = (r - step) % W
+            if src in vis:
+                _ok(fa.fa_bwd_accumulate(q_shards[r], k_shards[src], v_shards[src], do_shards[r], wss[r], wsb,
+                                         dka[src], dva[src], B, H, n, d, scale, vis[src]), "fa_bwd_accumulate")
+    outs = []
+    for r in range(W):
+        g = [torch.empty_like(q_shards[r]) for _ in range(3)]
+        _ok(fa.fa_bwd_finish(wss[r], wsb, dka[r], dva[r], *g, B, H, n, d, scale), "fa_bwd_finish")
+        outs.append(tuple(g))
+    return outs
+
+
+def _ok(rc, name):
+    if rc:
+        raise fa.FAError(rc, name)

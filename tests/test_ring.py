@@ -19,7 +19,7 @@ import torch.multiprocessing as mp
 import oracle
 from io_aware_exact_22_b200 import fa, ring
 from io_aware_exact_22_b200.inputs import custom, make_inputs, to_f64
-from tests._helpers import check_lse, check_o, f64
+from tests._helpers import check_grad, check_lse, check_o, f64
 
 OK, INVALID, UNSUPPORTED = 0, 1, 2
 A16 = 0x10000
@@ -123,3 +123,78 @@ def test_one_part_is_the_forward(cuda_ok):
     assert (o.float() - o2.float()).abs().max().item() <= 8e-3
     assert (lse - l2).abs().max().item() <= 1e-5
     assert torch.equal(lse, pl[0])
+
+
+# ---------------------------------------------------------------- backward
+def _round_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        own = [torch.full((2, 3), float(rank)), torch.zeros(2, 3)]
+        seen, home = [], None
+        for step, src, held in ring.ring_round(own):
+            if step == world:
+                home = (float(held[0][0, 0]), float(held[1][1, 1]))
+                break
+            seen.append((src, float(held[0][0, 0])))
+            held[1] += rank + 1  # this rank's contribution to shard src's accumulator
+        q.put((rank, seen, home))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_ring_round_trip_on_gloo_ranks(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_round_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = {r: (seen, home) for r, seen, home in (q.get(timeout=10) for _ in range(world))}
+    for r in range(world):
+        seen, home = res[r]
+        assert seen == [((r - s) % world, float((r - s) % world)) for s in range(world)]
+        # back home: this rank's own shard, with every rank's contribution added
+        assert home == (float(r), float(world * (world + 1) // 2))
+
+
+@pytest.mark.parametrize("fn", ["prepare", "accumulate", "finish"])
+def test_backward_pieces_reject_d64_and_null(fn):
+    a = A16
+    if fn == "prepare":
+        assert fa.fa_bwd_prepare(a, a, a, a, 1 << 30, 1, 2, 256, 64, 0) == UNSUPPORTED
+        assert fa.fa_bwd_prepare(0, a, a, a, 1 << 30, 1, 2, 256, 128, 0) == INVALID
+        assert fa.fa_bwd_prepare(a, a, a, a, 10, 1, 2, 256, 128, 0) == INVALID
+    elif fn == "accumulate":
+        assert fa.fa_bwd_accumulate(a, a, a, a, a, 1 << 30, a, a, 1, 2, 256, 64, 0.1, 0, 0) == UNSUPPORTED
+        assert fa.fa_bwd_accumulate(a, a, a, a, a, 1 << 30, 0, a, 1, 2, 256, 128, 0.1, 0, 0) == INVALID
+        assert fa.fa_bwd_accumulate(a, a, a, a, a, 1 << 30, a + 4, a, 1, 2, 256, 128, 0.1, 0, 0) == INVALID
+    else:
+        assert fa.fa_bwd_finish(a, 1 << 30, a, a, a, a, a, 1, 2, 256, 64, 0.1, 0) == UNSUPPORTED
+        assert fa.fa_bwd_finish(a, 1 << 30, a, a, 0, a, a, 1, 2, 256, 128, 0.1, 0) == INVALID
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("W,n", [(2, 128), (3, 200), (4, 129)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_ring_backward_on_one_gpu(cuda_ok, W, n, causal):
+    w = custom(1, 2, W * n, 128, causal, seed=W * 100 + n, backward=True)
+    q, k, v, do = make_inputs(w)
+    shard = lambda t: [t[:, :, r * n:(r + 1) * n].contiguous().cuda() for r in range(W)]  # noqa: E731
+    qs, ks, vs, dos = shard(q), shard(k), shard(v), shard(do)
+    fwd = ring.ring_attention_forward_local(qs, ks, vs, causal, w.scale)
+    grads = ring.ring_attention_backward_local(qs, ks, vs, [x[0] for x in fwd], dos, [x[1] for x in fwd],
+                                               causal, w.scale)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status() == 0
+    gq, gk, gv = (np.concatenate([f64(g[i]) for g in grads], axis=2) for i in range(3))
+    for h in range(w.H):
+        rq, rk, rv, _ = oracle.attention_backward_head(to_f64(q[0, h]), to_f64(k[0, h]), to_f64(v[0, h]),
+                                                       to_f64(do[0, h]), w.scale, causal)
+        check_grad(gq[0, h], rq, f"dQ[{h}]")
+        check_grad(gk[0, h], rk, f"dK[{h}]")
+        check_grad(gv[0, h], rv, f"dV[{h}]")
