@@ -1,10 +1,11 @@
 """ctypes binding over libfa.so (C ABI in include/fa.h).
 
-The functions ``fa_fwd``, ``fa_bwd``, ``fa_bwd_workspace_bytes``, ``fa_get_device_status``,
-``fa_status_string`` and ``fa_version`` carry the C names and only marshal arguments: torch
-tensors supply device pointers and the current CUDA stream, and every step of the attention
-path runs in the library's kernels.  ``forward`` / ``backward`` additionally allocate the
-output tensors with torch (memory plumbing only).
+Every name in ``EXPORTS`` (``fa_fwd``, ``fa_bwd``, the split-KV, FP8, deterministic,
+allocation-free and sharded-pieces entry points, the status and self-test calls) has a
+function here with the C name that only marshals arguments: torch tensors supply device
+pointers and the current CUDA stream, and every step of the attention path runs in the
+library's kernels.  ``forward``, ``forward_splitkv``, ``forward_fp8`` and ``backward``
+additionally allocate the output tensors with torch (memory plumbing only).
 
 Loading fails loudly (``RuntimeError``) when the shared library is missing: there is no
 fallback implementation.

@@ -148,8 +148,16 @@ def ring_round(tensors, group=None):
 
 def _check_bwd(*ts):
     for t in ts:
-        if not (t.is_cuda and t.is_contiguous() and t.dim() == 4 and t.shape[-1] == 128):
-            raise ValueError("the sharded backward takes contiguous CUDA tensors [B,H,n,128]")
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and t.dim() == 4
+                and t.shape[-1] == 128 and t.shape == ts[0].shape):
+            raise ValueError("the sharded backward takes contiguous CUDA bf16 tensors [B,H,n,128] "
+                             "of one shape")
+
+
+def _check_lse(lse, q):
+    if not (lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous()
+            and tuple(lse.shape) == tuple(q.shape[:3])):
+        raise ValueError("lse must be a contiguous CUDA fp32 tensor [B,H,n]")
 
 
 def ring_attention_backward(q, k, v, o, do, lse, causal: bool, scale: float | None = None,
@@ -157,6 +165,7 @@ def ring_attention_backward(q, k, v, o, do, lse, causal: bool, scale: float | No
     """dQ, dK, dV of this rank's shards.  q, k, v, o, do: this rank's bf16 [B, H, n, 128]
     shards; lse: its fp32 [B, H, n] from ring_attention_forward.  Collective over `group`."""
     _check_bwd(q, k, v, o, do)
+    _check_lse(lse, q)
     B, H, n, d = q.shape
     scale = d ** -0.5 if scale is None else scale
     W, r = dist.get_world_size(group), dist.get_rank(group)
@@ -187,6 +196,8 @@ def ring_attention_backward_local(q_shards, k_shards, v_shards, o_shards, do_sha
     [(dQ_r, dK_r, dV_r)]."""
     W = len(q_shards)
     _check_bwd(*q_shards, *k_shards, *v_shards, *o_shards, *do_shards)
+    for lse, q in zip(lse_shards, q_shards):
+        _check_lse(lse, q)
     B, H, n, d = q_shards[0].shape
     scale = d ** -0.5 if scale is None else scale
     wsb = fa.fa_bwd_workspace_bytes(B, H, n, d)
