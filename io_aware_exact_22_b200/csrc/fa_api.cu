@@ -84,6 +84,18 @@ fa_status_t check_shape(int B, int H, int N, int d, float scale, int causal, boo
 }
 
 // Per-query-tile statistics of the backward: [BH][ceil(N/64)][128] fp32, rounded to 256 bytes.
+// Work order of the attention grids.  Under the causal mask a head's query blocks (forward) or
+// key tiles (backward) differ in length; launching every head's heaviest block first gives the
+// shortest tail, but spreads the blocks in flight over all heads, whose streamed operand pair
+// (K, V in the forward; Q, dO in the backward) must then stay in L2 together.  Measured on
+// B200 (126 MB L2): block-major gains up to 21 % (forward) and 8 % (backward) when that pair
+// spans at most ~67 MB for all heads, and loses 5-13 % at 134 MB and beyond.
+int block_major_order(long long BH, int N, int d, int elem_bytes, int causal) {
+  if (!causal) return 0;
+  const double pair_bytes = 2.0 * (double)BH * N * d * elem_bytes;
+  return pair_bytes <= 80.0 * 1024 * 1024 ? 1 : 0;
+}
+
 size_t ld_bytes(long long bh, int N) {
   const long long tiles = bh * ((N + 63) / 64);
   return ((size_t)tiles * 128 * 4 + 255) & ~(size_t)255;
@@ -248,6 +260,7 @@ fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* 
   a.causal = causal;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   a.nsplit = 1;
+  a.block_major = block_major_order(BH, N, d, 2, causal);
   if ((long long)a.BH * a.nqb > INT_MAX) return FA_ERR_INVALID_ARG;
   return launch_fwd(d, tq, tk, tv, to, a, (cudaStream_t)stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -278,6 +291,7 @@ fa_status_t fa_fwd_fp8(const void* q, const void* k, const void* v, const float*
   a.causal = causal;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   a.nsplit = 1;
+  a.block_major = block_major_order(BH, N, d, 1, causal);
   a.descale_q = descale_q;
   a.descale_k = descale_k;
   a.descale_v = descale_v;
@@ -383,6 +397,7 @@ fa_status_t fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o,
   a.causal = causal;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   a.nsplit = sp;
+  a.block_major = block_major_order(BH, N, d, 2, causal);
   cudaStream_t s = (cudaStream_t)stream;
   if (launch_fwd(d, tq, tk, tv, to, a, s) != cudaSuccess) return FA_ERR_CUDA;
   if (launch_fwd_merge(o_part, lse_part, o, lse, sp, rows, d, s) != cudaSuccess) return FA_ERR_CUDA;
@@ -413,6 +428,7 @@ fa_status_t fa_fwd_partial(const void* q, const void* k, const void* v, float* o
   a.causal = causal;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   a.nsplit = 1;
+  a.block_major = block_major_order(BH, N, d, 2, causal);
   return launch_fwd_partial(d, tq, tk, tv, to, a, (cudaStream_t)stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -478,6 +494,7 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
   a.causal = causal;
   a.scale = scale;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  a.block_major = block_major_order(BH, N, d, 2, causal);
   if (launch_bwd_pre(o, dO, lse, ld, dq_acc, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
   cudaError_t e = launch_bwd_main(d, tq, tk, tv, tdo, tdk, tdv, tdq, a, s);
   if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
@@ -536,6 +553,7 @@ fa_status_t fa_bwd_accumulate(const void* q, const void* k, const void* v, const
   a.causal = causal;
   a.scale = scale;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  a.block_major = block_major_order(BH, N, d, 2, causal);
   // the dK/dV store maps are not used in accumulate mode; any valid map fills the parameters
   return launch_bwd_main(d, tq, tk, tv, tdo, tk, tv, tdq, a, (cudaStream_t)stream) == cudaSuccess ? FA_OK
                                                                                                   : FA_ERR_CUDA;
@@ -600,6 +618,7 @@ fa_status_t fa_bwd_deterministic(const void* q, const void* k, const void* v, co
   a.causal = causal;
   a.scale = scale;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  a.block_major = block_major_order(BH, N, d, 2, causal);
   if (launch_bwd_pre(o, dO, lse, ld, nullptr, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
   if (launch_bwd_main(d, tq64, tk128, tv128, tdo64, tdk, tdv, tdk, a, s, false) != cudaSuccess) return FA_ERR_CUDA;
   if (launch_bwd_dq(d, tq128, tk64, tv64, tdo128, tdq, a, s) != cudaSuccess) return FA_ERR_CUDA;

@@ -172,8 +172,10 @@ __global__ void __launch_bounds__(448, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int bh = blockIdx.x / Tk;
-  const int j = blockIdx.x % Tk;               // key tile: keys [128 j, 128 j + 128)
+  // head-major (a head's key tiles together, heaviest first) or tile-major (every head's
+  // heaviest key tile first); see fa_fwd_kernel for the trade-off
+  const int bh = a.block_major ? (int)(blockIdx.x % a.BH) : (int)(blockIdx.x / Tk);
+  const int j = a.block_major ? (int)(blockIdx.x / a.BH) : (int)(blockIdx.x % Tk);  // keys [128 j, +128)
   const int i0 = a.causal ? 2 * j : 0;         // first query tile with a visible pair
   const int count = max(0, Tq - i0);
 

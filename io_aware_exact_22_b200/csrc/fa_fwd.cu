@@ -85,8 +85,10 @@ __global__ void __launch_bounds__(320, 1)
   // ---- work item: (head bh, block of 256 query rows, key split); heavier causal blocks first
   const int split = blockIdx.x % a.nsplit;
   const int item = blockIdx.x / a.nsplit;
-  const int bh = item / a.nqb;
-  const int qb = a.nqb - 1 - (item % a.nqb);
+  // head-major (a head's query blocks together, heaviest first: its K/V stays in L2) or
+  // block-major (every head's heaviest block first: the shortest tail under the causal mask)
+  const int bh = a.block_major ? item % a.BH : item / a.nqb;
+  const int qb = a.nqb - 1 - (a.block_major ? item / a.BH : item % a.nqb);
   const int q0 = qb * 256;
   const int Tk = (a.N + 127) >> 7;
   const bool has1 = (q0 + 128) < a.N;
