@@ -13,10 +13,12 @@
 //   warps 0-3  softmax warpgroup for query tile 0   (one thread per query row)
 //   warps 4-7  softmax warpgroup for query tile 1
 //   warp  8    MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j on the tensor core
-//   warp  9    TMA producer (one thread): Q tiles once, then K_j, V_j into the ring
+//   warp  9    TMA producer (one thread): Q tiles once, then K_0, and K_{j+1} ahead of V_j
 // TMEM (512 columns x 128 lanes, fp32): S_0 [0,128), S_1 [128,256), O_0 [256,256+d),
-// O_1 [256+d, 256+2d).  P_t (bf16, two per column) overwrites the first 64 columns of S_t.
-// While softmax warpgroup 0 works on S_0, the tensor core runs tile 1's MMAs and vice versa.
+// O_1 [256+d, 256+2d).  P_t goes to shared memory (bf16 or E4M3, the K-major 128-byte-swizzled
+// layout of an MMA A operand), so S_t is free as soon as its softmax warpgroup has loaded it
+// into registers: S_t for block j+1 is computed while the softmax of block j runs, and each
+// tile's chain per block is its softmax alone rather than S MMA + softmax + PV MMA.
 #include "fa_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -40,17 +42,20 @@ struct FwdCfg {
   static constexpr int BOXW = 128 / EB;            // elements per 128-byte swizzle box row
   static constexpr int NBOX = D / BOXW;            // swizzle boxes per row
   static constexpr int TILE = 128 * D * EB;        // bytes of one 128-row input tile
-  static constexpr int NS = (TILE == 32768) ? 4 : 8;  // K/V ring stages (one K or one V each)
+  // K/V ring stages (one K or one V tile each).  K_{j+1} is loaded ahead of V_j, so with three
+  // stages K_{j+2} reuses V_{j-1}'s stage and V_{j+1} reuses K_{j+1}'s.
+  static constexpr int NS = (TILE == 32768) ? 3 : 8;
   static constexpr int KSTEP = 32 / EB;            // elements of K per MMA (32 bytes)
-  static constexpr int P_COLS = 128 * EB / 4;      // TMEM columns of packed P for 128 keys
+  static constexpr int PTILE = 128 * 128 * EB;     // bytes of one P tile (128 rows x 128 keys)
   static constexpr int OTILE = 128 * D * 2;        // bytes of one 128-row bf16 output tile
   // O staging: the dead Q tiles (bf16) or the idle K/V ring (FP8: Q tiles are half as large)
   static constexpr int OST_OFF = FP8 ? 2 * TILE : 0;
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = 2 * TILE;
-  static constexpr int BAR_OFF = KV_OFF + NS * TILE;
-  // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_full
-  static constexpr int NBAR = 1 + 2 * NS + 2 + 2 + 1;
+  static constexpr int P_OFF = KV_OFF + NS * TILE;  // ring and P tiles together stage partial outputs
+  static constexpr int BAR_OFF = P_OFF + 2 * PTILE;
+  // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], s_free[2], p_full[2], pv_done[2], o_full
+  static constexpr int NBAR = 1 + 2 * NS + 8 + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM = MISC_OFF + 16 + 1024;  // + slack to align the base to 1024
   static constexpr int THREADS = 320;
@@ -59,10 +64,10 @@ struct FwdCfg {
   static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_O0 = 256, T_O1 = 256 + D;
   static constexpr uint32_t IDESC_QK = FP8 ? idesc_e4m3(128, 128, false, false) : idesc_bf16(128, 128, false, false);
   static constexpr uint32_t IDESC_PV = FP8 ? idesc_e4m3(128, D, false, true) : idesc_bf16(128, D, false, true);
-  // P is computed as 2^(s c - m + P_OFF) and the reference m moves once a block's max exceeds
+  // P is computed as 2^(s c - m + P_SHIFT) and the reference m moves once a block's max exceeds
   // it by more than MOVE (both base 2).  bf16: P <= 2^8.  FP8: P <= 2^8.75 < 448 (the largest
   // E4M3 value) and values down to 2^-17 of the reference term stay representable.
-  static constexpr float P_OFF = FP8 ? 8.0f : 0.0f;
+  static constexpr float P_SHIFT = FP8 ? 8.0f : 0.0f;
   static constexpr float MOVE = FP8 ? 0.75f : 8.0f;
 };
 
@@ -107,9 +112,11 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t q_full = bar;
   auto kv_full = [&](int s) { return bar + 8u * (1 + s); };
   auto kv_empty = [&](int s) { return bar + 8u * (1 + C::NS + s); };
-  auto s_full = [&](int t) { return bar + 8u * (1 + 2 * C::NS + t); };
-  auto p_full = [&](int t) { return bar + 8u * (3 + 2 * C::NS + t); };
-  const uint32_t o_full = bar + 8u * (5 + 2 * C::NS);
+  auto s_full = [&](int t) { return bar + 8u * (1 + 2 * C::NS + t); };   // S_t computed
+  auto s_free = [&](int t) { return bar + 8u * (3 + 2 * C::NS + t); };   // S_t loaded by its softmax
+  auto p_full = [&](int t) { return bar + 8u * (5 + 2 * C::NS + t); };   // P_t written
+  auto pv_done = [&](int t) { return bar + 8u * (7 + 2 * C::NS + t); };  // P_t V_j added into O_t
+  const uint32_t o_full = bar + 8u * (9 + 2 * C::NS);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gb + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + C::MISC_OFF + 4);
   const WaitCtx wc{abort_flag, a.status};
@@ -122,7 +129,9 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(s_full(t), 1);
+      mbar_init(s_free(t), 128);
       mbar_init(p_full(t), 128);
+      mbar_init(pv_done(t), 1);
     }
     mbar_init(o_full, 1);
     *abort_flag = 0;
@@ -157,19 +166,23 @@ __global__ void __launch_bounds__(320, 1)
         for (int b = 0; b < C::NBOX; ++b)
           tma_load_3d_e(sb + C::Q_OFF + t * C::TILE + b * 16384, &tmQ, q_full, C::BOXW * b, q0 + 128 * t,
                         bh, keep);
+      // ring order: K_0, then K_{j+1} (when there is one) before V_j
       int it = 0;
       bool ok = true;
+      auto load = [&](const CUtensorMap* m, int j) {
+        const int s = it % C::NS;
+        const uint32_t ph = (it / C::NS) & 1;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(kv_empty(s), ph ^ 1, wc)))) return;
+        mbar_arrive_expect_tx_e(kv_full(s), C::TILE);
+        for (int b = 0; b < C::NBOX; ++b)
+          tma_load_3d_e(sb + C::KV_OFF + s * C::TILE + b * 16384, m, kv_full(s), C::BOXW * b, 128 * (kb0 + j),
+                        bh, keep);
+        ++it;
+      };
+      load(&tmK, 0);
       for (int j = 0; j < nmax && ok; ++j) {
-        for (int kv = 0; kv < 2; ++kv, ++it) {
-          const int s = it % C::NS;
-          const uint32_t ph = (it / C::NS) & 1;
-          if (!(ok = __all_sync(0xffffffffu, mbar_wait(kv_empty(s), ph ^ 1, wc)))) break;
-          mbar_arrive_expect_tx_e(kv_full(s), C::TILE);
-          const CUtensorMap* m = kv ? &tmV : &tmK;
-          for (int b = 0; b < C::NBOX; ++b)
-            tma_load_3d_e(sb + C::KV_OFF + s * C::TILE + b * 16384, m, kv_full(s), C::BOXW * b, 128 * (kb0 + j),
-                          bh, keep);
-        }
+        if (j + 1 < nmax) load(&tmK, j + 1);
+        if (ok) load(&tmV, j);
       }
       if (!ok) {  // let copies already issued land before the CTA exits
         mbar_wait_drain(q_full, 0);
@@ -198,57 +211,68 @@ __global__ void __launch_bounds__(320, 1)
             mma_ss_e(dst, sdesc_add(dQ_k, qoff + off), sdesc_add(dK_k, koff + off), C::IDESC_QK, k > 0);
         }
       };
-      auto issue_pv = [&](uint32_t dst, uint32_t ptm, uint32_t voff, bool acc) {
+      const uint64_t dP_k = sdesc_sw128(sb + C::P_OFF, 16, 1024);       // P tiles, K-major
+      auto issue_pv = [&](uint32_t dst, uint32_t poff, uint32_t voff, bool acc) {
 #pragma unroll
-        for (int k = 0; k < 128 / C::KSTEP; ++k) {  // KSTEP keys per MMA: 8 TMEM columns of P
+        for (int k = 0; k < 128 / C::KSTEP; ++k) {  // KSTEP keys (32 bytes of P) per MMA
+          const uint32_t po = poff + (k >> 2) * 16384 + (k & 3) * 32;
           const uint32_t vo = voff + k * C::KSTEP * 128;
           if constexpr (FP8)
-            mma_ts_e8(dst, ptm + 8 * k, sdesc_add(dV_mn, vo), C::IDESC_PV, (acc || k > 0) ? 1u : 0u);
+            mma_ss_e8(dst, sdesc_add(dP_k, po), sdesc_add(dV_mn, vo), C::IDESC_PV, (acc || k > 0) ? 1u : 0u);
           else
-            mma_ts_e(dst, ptm + 8 * k, sdesc_add(dV_mn, vo), C::IDESC_PV, (acc || k > 0) ? 1u : 0u);
+            mma_ss_e(dst, sdesc_add(dP_k, po), sdesc_add(dV_mn, vo), C::IDESC_PV, (acc || k > 0) ? 1u : 0u);
         }
       };
+      // ring positions: K_0 first, then K_{j+1} (when there is one) before V_j
+      auto pos_k = [&](int j) { return j == 0 ? 0 : 2 * j - 1; };
+      auto pos_v = [&](int j) { return j + 1 < nmax ? 2 * j + 2 : 2 * j + 1; };
       auto stage_addr = [&](int it) { return (uint32_t)((it % C::NS) * C::TILE); };
       auto stage_par = [&](int it) { return (uint32_t)((it / C::NS) & 1); };
+      auto wait_stage = [&](int it) {
+        return __all_sync(0xffffffffu, mbar_wait(kv_full(it % C::NS), stage_par(it), wc));
+      };
       bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, wc));
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(kv_full(0), 0, wc));
+      if (ok) ok = wait_stage(0);
       if (ok) {
         tc_fence_after();
-        if (n0 > 0) {
-          issue_qk(C::T_S0, 0u, stage_addr(0));
-          mma_commit_e(s_full(0));
-        }
-        if (n1 > 0) {
-          issue_qk(C::T_S1, (uint32_t)C::TILE, stage_addr(0));
-          mma_commit_e(s_full(1));
+        for (int t = 0; t < 2; ++t) {
+          if (nt[t] == 0) continue;
+          issue_qk(t ? C::T_S1 : C::T_S0, (uint32_t)(t * C::TILE), stage_addr(0));
+          mma_commit_e(s_full(t));
         }
         mma_commit_e(kv_empty(0));
       }
       for (int j = 0; j < nmax && ok; ++j) {
-        const int itK = 2 * (j + 1), itV = 2 * j + 1;  // ring positions of K_{j+1} and V_j
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(kv_full(itV % C::NS), stage_par(itV), wc)))) break;
+        // S_t for block j+1, each as soon as tile t's softmax has loaded S_t for block j
+        if (j + 1 < nmax) {
+          const int itK = pos_k(j + 1);
+          if (!(ok = wait_stage(itK))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (j + 1 >= nt[t]) continue;
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(s_free(t), j & 1, wc)))) break;
+            tc_fence_after();
+            issue_qk(t ? C::T_S1 : C::T_S0, (uint32_t)(t * C::TILE), stage_addr(itK));
+            mma_commit_e(s_full(t));
+          }
+          if (!ok) break;
+          mma_commit_e(kv_empty(itK % C::NS));
+        }
+        // O_t += P_t V_j, each as soon as tile t's softmax has written P_t
+        const int itV = pos_v(j);
+        if (!(ok = wait_stage(itV))) break;
         tc_fence_after();
-        bool k_ready = false;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           if (j >= nt[t]) continue;
           if (!(ok = __all_sync(0xffffffffu, mbar_wait(p_full(t), j & 1, wc)))) break;
           tc_fence_after();
-          issue_pv(t ? C::T_O1 : C::T_O0, t ? C::T_S1 : C::T_S0, stage_addr(itV), j > 0);
-          if (j + 1 < nt[t]) {
-            if (!k_ready) {
-              if (!(ok = __all_sync(0xffffffffu, mbar_wait(kv_full(itK % C::NS), stage_par(itK), wc))))
-                break;
-              tc_fence_after();
-              k_ready = true;
-            }
-            issue_qk(t ? C::T_S1 : C::T_S0, (uint32_t)(t * C::TILE), stage_addr(itK));
-            mma_commit_e(s_full(t));
-          }
+          issue_pv(t ? C::T_O1 : C::T_O0, (uint32_t)(t * C::PTILE), stage_addr(itV), j > 0);
+          mma_commit_e(pv_done(t));
         }
         if (!ok) break;
         mma_commit_e(kv_empty(itV % C::NS));
-        if (k_ready) mma_commit_e(kv_empty(itK % C::NS));
       }
       mma_commit_e(o_full);
       if (!ok) mbar_wait_drain(o_full, 0);  // every issued MMA has completed before TMEM is freed
@@ -287,12 +311,26 @@ __global__ void __launch_bounds__(320, 1)
       tmem_ld32(tSrow + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
       tmem_wait_ld();
       reg_fence(sr);
+      tc_fence_before();
+      mbar_arrive(s_free(t));  // S_t may now be overwritten by the next block's scores
       float x[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
       const int jg = kb0 + j;                 // key block index in the whole key range
       const bool edge = (jg == ntile_g - 1);  // the only block that can hold the diagonal or the tail
-      uint32_t pk[64];
+      // P_t row r in shared memory: 16-byte chunks g of the 128-byte-swizzled K-major layout (64
+      // bf16 or 128 E4M3 keys per 128-byte box row), each stored as soon as its four 32-bit
+      // words are packed (word indices are compile-time constants in the unrolled loops)
+      uint8_t* prow = gb + C::P_OFF + t * C::PTILE + r * 128;
+      uint32_t cw[4];
+      auto put_word = [&](int w, uint32_t v) {
+        cw[w & 3] = v;
+        if ((w & 3) == 3) {
+          const int g = w >> 2;
+          *reinterpret_cast<uint4*>(prow + (g >> 3) * 16384 + (((g & 7) ^ (r & 7)) << 4)) =
+              make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        }
+      };
 
       // Exponentials of a full (unmasked) block against reference -mneg: y = s * cs - m for a
       // pair of columns in one f32x2 FMA; kPolyPairsOf8 of every 8 pairs take the FMA-pipe
@@ -320,11 +358,11 @@ __global__ void __launch_bounds__(320, 1)
             sa = f2_add(sa, f2_pack(p0, p1));
           if constexpr (FP8) {
             if ((c >> 1) & 1)
-              pk[c >> 2] = pack_e4m3x4(q0p, q1p, p0, p1);
+              put_word(c >> 2, pack_e4m3x4(q0p, q1p, p0, p1));
             else
               q0p = p0, q1p = p1;
           } else {
-            pk[c >> 1] = pack_bf16(p0, p1);
+            put_word(c >> 1, pack_bf16(p0, p1));
           }
         }
         float s0, s1, s2, s3;
@@ -360,22 +398,14 @@ __global__ void __launch_bounds__(320, 1)
         alpha = ex2(m_ref - mblk);  // 0 when m_ref is still -inf
         m_ref = mblk;
       }
-      if (__any_sync(0xffffffffu, move && j > 0)) {
-        // O_t holds sum_{j' < j} of P V relative to the old reference: rescale by alpha.
-#pragma unroll 1
-        for (int cc = 0; cc < D; cc += 32) {
-          uint32_t o[32];
-          tmem_ld32(tOrow + cc, o);
-          tmem_wait_ld();
-          reg_fence(o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tOrow + cc, o);
-        }
-      }
       l *= alpha;
+      // P_t V_{j-1} must have been added into O_t before P_t is rewritten or O_t rescaled
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(pv_done(t), (j - 1) & 1, wc));
+        if (!ok) break;
+      }
       float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
-      if constexpr (FP8) mneg += C::P_OFF;
+      if constexpr (FP8) mneg += C::P_SHIFT;
       float rsum;
       if (!edge) {
         rsum = exp_full(mneg);
@@ -393,7 +423,7 @@ __global__ void __launch_bounds__(320, 1)
             rs1 += p1;
             rs0 += p2;
             rs1 += p3;
-            pk[c >> 2] = pack_e4m3x4(p0, p1, p2, p3);
+            put_word(c >> 2, pack_e4m3x4(p0, p1, p2, p3));
           }
         } else {
 #pragma unroll
@@ -402,15 +432,28 @@ __global__ void __launch_bounds__(320, 1)
             const float p1 = (c + 1 > lim) ? 0.f : ex2(fmaf(x[c + 1], cs, mneg));
             rs0 += p0;
             rs1 += p1;
-            pk[c >> 1] = pack_bf16(p0, p1);
+            put_word(c >> 1, pack_bf16(p0, p1));
           }
         }
         rsum = rs0 + rs1;
       }
       l += rsum;
-      tmem_st32(tSrow + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      if constexpr (!FP8) tmem_st32(tSrow + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-      tmem_wait_st();
+      if (j > 0 && __any_sync(0xffffffffu, move)) {
+        // O_t holds sum_{j' < j} of P V relative to the old reference: rescale by alpha.
+        tc_fence_after();
+#pragma unroll 1
+        for (int cc = 0; cc < D; cc += 32) {
+          uint32_t o[32];
+          tmem_ld32(tOrow + cc, o);
+          tmem_wait_ld();
+          reg_fence(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tOrow + cc, o);
+        }
+        tmem_wait_st();
+      }
+      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(p_full(t));
     }
@@ -459,9 +502,9 @@ __global__ void __launch_bounds__(320, 1)
           __syncwarp();
           if (qrow < a.N)
             a.lse[(size_t)bh * a.N + qrow] =
-                (l > 0.f) ? (m_ref - C::P_OFF + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+                (l > 0.f) ? (m_ref - C::P_SHIFT + log2f(l)) * 0.69314718055994530942f : -INFINITY;
         } else {
-          // fp32 partial O_s = O / l of this split, staged in the (now idle) K/V ring as
+          // fp32 partial O_s = O / l of this split, staged in the (now idle) K/V ring and P tiles as
           // 32-column, 128-byte-swizzled boxes and written by TMA; then LSE_s.
           constexpr int PBOX = D / 32;
           const uint32_t pstage = C::KV_OFF + t * (128 * D * 4);
@@ -510,7 +553,7 @@ static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, co
   using C = FwdCfg<D, FP8>;
   static_assert(C::SMEM <= 232448, "shared memory budget");
   static_assert(C::SMEM > 116 * 1024, "one CTA per SM: each allocates all 512 TMEM columns");
-  static_assert(2 * 128 * D * 4 <= C::NS * C::TILE, "partial-output staging must fit the K/V ring");
+  static_assert(2 * 128 * D * 4 <= C::NS * C::TILE + 2 * C::PTILE, "partial-output staging must fit the ring and P");
   static_assert(C::OST_OFF + 2 * C::OTILE <= C::BAR_OFF, "output staging must fit");
   static bool attr_set[64];  // per device: the attribute outlives the call
   int dev = 0;
