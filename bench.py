@@ -131,6 +131,14 @@ class ClockSampler:
                                     if r[3].replace(".", "").isdigit()), default=None)}
 
 
+def l2_note(tensor_bytes: int) -> str:
+    """How the timed steps stand to the 126 MB L2 (no flush between steps either way)."""
+    mb = tensor_bytes / 1e6
+    if tensor_bytes > 126 * 1024 * 1024:
+        return f"inputs larger than L2 (q,k,v,o,dO {mb:.0f} MB each vs 126 MB L2), no flush"
+    return f"inputs fit in L2 (q,k,v,o,dO {mb:.1f} MB each), no flush: L2-warm figures"
+
+
 # ---------------------------------------------------------------------- traffic
 def kernel_traffic(name: str):
     """DRAM bytes per launch from the committed ncu summary, or None once the kernel's sources
@@ -328,7 +336,7 @@ def run_gpu(args):
         "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
                    "step": "fa_fwd + " + ("fa_bwd_deterministic" if args.deterministic else "fa_bwd"),
                    "per_rank": "same workload on every rank",
-                   "l2": "inputs larger than L2 (q,k,v,o,dO 134 MB each vs 126 MB L2), no flush"},
+                   "l2": l2_note(B * H * N * d * 2)},
         "pct_of_peak": round(100 * value / world / peak, 2),
         "fwd": {"ms": round(fwd_ms, 4), "tflops": round(fwd_tflops, 1),
                 "pct_of_peak": round(100 * fwd_tflops / peak, 2)},
