@@ -17,7 +17,8 @@ shard's accumulators back to its owner, which rounds them to bf16 (fa_bwd_finish
 
 The exchange has no multicast and no library kernel touches another GPU's memory: each shard
 is received into this rank's own buffers before it is read.  Causal sharding by contiguous
-shards leaves rank W - 1 with W pieces of work and rank 0 with one.
+shards leaves rank W - 1 with W pieces of work and rank 0 with one; the zig-zag layout at the
+end of this module (rank r holds chunks r and 2W-1-r of 2W) gives every rank 2W+1.
 """
 from __future__ import annotations
 
@@ -31,29 +32,34 @@ def _peer(group, rank: int) -> int:
     return rank if group is None else dist.get_global_rank(group, rank)
 
 
-def ring_shards(k: torch.Tensor, v: torch.Tensor, group=None):
-    """Yields (src, k_src, v_src) for the K/V shards of all W ranks: this rank's own first, then
-    rank r-1's, r-2's, ... around the ring.  The transfer of the next shard (send the current
-    one to rank r+1, receive from rank r-1) is in flight while the caller uses the current one;
-    two receive buffers alternate.  Every rank must run the generator to the end."""
+def ring_pass(tensors, group=None):
+    """Yields (src, held) for the tensor lists of all W ranks: this rank's own first, then rank
+    r-1's, r-2's, ... around the ring.  The transfer of the next list (send the current one to
+    rank r+1, receive from rank r-1) is in flight while the caller uses the current one; two
+    sets of receive buffers alternate.  Every rank must run the generator to the end."""
     W = dist.get_world_size(group)
     r = dist.get_rank(group)
     nxt, prv = _peer(group, (r + 1) % W), _peer(group, (r - 1) % W)
-    cur = (k, v)
-    bufs = [(torch.empty_like(k), torch.empty_like(v)) for _ in range(2 if W > 2 else 1)]
+    cur = list(tensors)
+    bufs = [[torch.empty_like(t) for t in cur] for _ in range(2 if W > 2 else 1)]
     for step in range(W):
         reqs = []
         if step < W - 1:
             nb = bufs[step % len(bufs)]
-            reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, cur[0], nxt, group),
-                                           dist.P2POp(dist.isend, cur[1], nxt, group),
-                                           dist.P2POp(dist.irecv, nb[0], prv, group),
-                                           dist.P2POp(dist.irecv, nb[1], prv, group)])
-        yield (r - step) % W, cur[0], cur[1]
+            ops = [dist.P2POp(dist.isend, t, nxt, group) for t in cur]
+            ops += [dist.P2POp(dist.irecv, t, prv, group) for t in nb]
+            reqs = dist.batch_isend_irecv(ops)
+        yield (r - step) % W, cur
         for rq in reqs:
             rq.wait()
         if step < W - 1:
             cur = nb
+
+
+def ring_shards(k: torch.Tensor, v: torch.Tensor, group=None):
+    """Yields (src, k_src, v_src) for the K/V shards of all W ranks, as ring_pass does."""
+    for src, (ks, vs) in ring_pass([k, v], group):
+        yield src, ks, vs
 
 
 def visible_shards(r: int, W: int, causal: bool):
@@ -225,3 +231,194 @@ def ring_attention_backward_local(q_shards, k_shards, v_shards, o_shards, do_sha
 def _ok(rc, name):
     if rc:
         raise fa.FAError(rc, name)
+
+
+# ------------------------------------------------------------------------ zig-zag layout
+# With contiguous shards, causal attention gives rank W-1 W pieces of work and rank 0 one.  In
+# the zig-zag layout the sequence is cut into 2W chunks and rank r holds chunks r and 2W-1-r
+# (one early, one late), so every rank computes 2W+1 pieces (W(2W+1) = the 2W(2W+1)/2 visible
+# chunk pairs spread evenly).  Each rank passes a list of two chunks of q, k, v (and so on) of
+# equal shape [B, H, n, d]; the pieces are the same partial-result, merge and accumulate calls
+# as for contiguous shards.
+
+def zigzag_chunks(r: int, W: int):
+    """Sequence chunks (of 2W) held by rank r: (r, 2W-1-r)."""
+    return (r, 2 * W - 1 - r)
+
+
+def zigzag_pieces(r: int, W: int, src: int, causal: bool):
+    """The pieces rank r computes with rank src's key chunks: (query slot, key slot, masked)
+    for every pair of r's query chunk a and src's key chunk b with b <= a (every pair when not
+    causal); the causal mask applies inside the piece when a == b."""
+    out = []
+    for iq, a in enumerate(zigzag_chunks(r, W)):
+        for ik, b in enumerate(zigzag_chunks(src, W)):
+            if causal and b > a:
+                continue
+            out.append((iq, ik, causal and a == b))
+    return out
+
+
+def _check_chunks(ts, bwd: bool):
+    """Chunks of one rank: contiguous CUDA bf16 [B, H, n, d] of one shape (d = 128 for the
+    backward)."""
+    shape = ts[0].shape
+    for t in ts:
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.dim() == 4 and t.is_contiguous()
+                and t.shape == shape and (not bwd or t.shape[-1] == 128)):
+            raise ValueError("zig-zag chunks must be contiguous CUDA bf16 tensors [B,H,n,d] of one "
+                             "shape" + (" with d = 128" if bwd else ""))
+
+
+def _zigzag_forward(q2, shard_iter, r, W, causal, scale, out2, lse2):
+    """O and LSE of rank r's two query chunks from the key/value chunks of every rank
+    (shard_iter yields (src, [k_a, k_b, v_a, v_b]) of rank src's chunks)."""
+    B, H, n, d = q2[0].shape
+    chunks = zigzag_chunks(r, W)
+    parts = []
+    for a in chunks:
+        m = a + 1 if causal else 2 * W  # key chunks visible to query chunk a
+        parts.append((torch.empty((m, B, H, n, d), device=q2[0].device, dtype=torch.float32),
+                      torch.empty((m, B, H, n), device=q2[0].device, dtype=torch.float32)))
+    used = [0, 0]
+    for src, held in shard_iter:
+        for iq, ik, masked in zigzag_pieces(r, W, src, causal):
+            po, pl = parts[iq]
+            _ok(fa.fa_fwd_partial(q2[iq], held[ik], held[2 + ik], po[used[iq]], pl[used[iq]], B, H, n, d,
+                                  scale, masked), "fa_fwd_partial")
+            used[iq] += 1
+    for iq in range(2):
+        _ok(fa.fa_merge_partials(parts[iq][0], parts[iq][1], used[iq], out2[iq], lse2[iq], B, H, n, d),
+            "fa_merge_partials")
+    return out2, lse2
+
+
+def ring_attention_forward_zigzag(q2, k2, v2, causal: bool, scale: float | None = None, group=None):
+    """O and LSE of this rank's two zig-zag query chunks (chunks r and 2W-1-r of the sequence),
+    attending over the whole sharded sequence.  q2, k2, v2: lists of this rank's two chunks,
+    contiguous bf16 [B, H, n, d].  Returns ([O_a, O_b], [LSE_a, LSE_b]).  Collective over
+    `group`; the key/value chunks travel round the ring while the held ones are used."""
+    _check_chunks([*q2, *k2, *v2], bwd=False)
+    B, H, n, d = q2[0].shape
+    scale = d ** -0.5 if scale is None else scale
+    W, r = dist.get_world_size(group), dist.get_rank(group)
+    out2 = [torch.empty_like(q2[0]), torch.empty_like(q2[1])]
+    lse2 = [torch.empty((B, H, n), device=q2[0].device, dtype=torch.float32) for _ in range(2)]
+    return _zigzag_forward(q2, ring_pass([k2[0], k2[1], v2[0], v2[1]], group), r, W, causal, scale,
+                           out2, lse2)
+
+
+def _zigzag_split(t, W):
+    n = t.shape[2] // (2 * W)
+    return [t[:, :, c * n:(c + 1) * n].contiguous() for c in range(2 * W)]
+
+
+def ring_attention_forward_zigzag_local(q, k, v, W: int, causal: bool, scale: float | None = None):
+    """The zig-zag forward of W ranks on this device, one after the other, for whole-sequence
+    q, k, v [B, H, N, d] (N a multiple of 2W): each rank's chunks are cut out, its pieces
+    computed in its ring order, and O [B, H, N, d], LSE [B, H, N] returned in sequence order."""
+    B, H, N, d = q.shape
+    if N % (2 * W):
+        raise ValueError("N must be a multiple of 2W")
+    cq, ck, cv = _zigzag_split(q, W), _zigzag_split(k, W), _zigzag_split(v, W)
+    _check_chunks(cq + ck + cv, bwd=False)
+    scale = d ** -0.5 if scale is None else scale
+    n = N // (2 * W)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+    for r in range(W):
+        a = zigzag_chunks(r, W)
+        order = []
+        for step in range(W):
+            src = (r - step) % W
+            s0, s1 = zigzag_chunks(src, W)
+            order.append((src, [ck[s0], ck[s1], cv[s0], cv[s1]]))
+        out2 = [torch.empty_like(cq[a[0]]), torch.empty_like(cq[a[1]])]
+        lse2 = [torch.empty((B, H, n), device=q.device, dtype=torch.float32) for _ in range(2)]
+        _zigzag_forward([cq[a[0]], cq[a[1]]], iter(order), r, W, causal, scale, out2, lse2)
+        for i in range(2):
+            o[:, :, a[i] * n:(a[i] + 1) * n] = out2[i]
+            lse[:, :, a[i] * n:(a[i] + 1) * n] = lse2[i]
+    return o, lse
+
+
+def _zigzag_backward(q2, do2, ws2, wsb, round_iter, r, W, causal, scale):
+    """Adds rank r's contributions into every key chunk's dK/dV accumulators as they come round
+    (round_iter yields (step, src, [k_a, k_b, v_a, v_b, dk_a, dk_b, dv_a, dv_b]) and, at
+    step W, this rank's own list back); returns this rank's own [dk_a, dk_b, dv_a, dv_b]."""
+    B, H, n, d = q2[0].shape
+    for step, src, held in round_iter:
+        if step == W:
+            return held[4:]
+        for iq, ik, masked in zigzag_pieces(r, W, src, causal):
+            _ok(fa.fa_bwd_accumulate(q2[iq], held[ik], held[2 + ik], do2[iq], ws2[iq], wsb, held[4 + ik],
+                                     held[6 + ik], B, H, n, d, scale, masked), "fa_bwd_accumulate")
+    raise RuntimeError("the ring ended before the accumulators came home")
+
+
+def ring_attention_backward_zigzag(q2, k2, v2, o2, do2, lse2, causal: bool, scale: float | None = None,
+                                   group=None):
+    """dQ, dK, dV of this rank's two zig-zag chunks.  q2, k2, v2, o2, do2: lists of its two bf16
+    [B, H, n, 128] chunks; lse2: the two fp32 [B, H, n] LSEs from ring_attention_forward_zigzag.
+    Each rank's key chunks go round the ring with fp32 dK/dV accumulators and come home after
+    one more hop.  Returns ([dQ_a, dQ_b], [dK_a, dK_b], [dV_a, dV_b]).  Collective over `group`."""
+    _check_chunks([*q2, *k2, *v2, *o2, *do2], bwd=True)
+    for lse, q in zip(lse2, q2):
+        _check_lse(lse, q)
+    B, H, n, d = q2[0].shape
+    scale = d ** -0.5 if scale is None else scale
+    W, r = dist.get_world_size(group), dist.get_rank(group)
+    wsb = fa.fa_bwd_workspace_bytes(B, H, n, d)
+    ws2 = [torch.empty(wsb, device=q2[0].device, dtype=torch.uint8) for _ in range(2)]
+    for i in range(2):
+        _ok(fa.fa_bwd_prepare(o2[i], do2[i], lse2[i], ws2[i], wsb, B, H, n, d), "fa_bwd_prepare")
+    acc = [torch.zeros(q2[0].shape, device=q2[0].device, dtype=torch.float32) for _ in range(4)]
+    home = _zigzag_backward(q2, do2, ws2, wsb, ring_round([k2[0], k2[1], v2[0], v2[1], *acc], group), r, W,
+                            causal, scale)
+    dq2, dk2, dv2 = [], [], []
+    for i in range(2):
+        g = [torch.empty_like(q2[i]) for _ in range(3)]
+        _ok(fa.fa_bwd_finish(ws2[i], wsb, home[i], home[2 + i], *g, B, H, n, d, scale), "fa_bwd_finish")
+        dq2.append(g[0])
+        dk2.append(g[1])
+        dv2.append(g[2])
+    return dq2, dk2, dv2
+
+
+def ring_attention_backward_zigzag_local(q, k, v, o, do, lse, W: int, causal: bool,
+                                         scale: float | None = None):
+    """The zig-zag backward of W ranks on this device for whole-sequence tensors (N a multiple
+    of 2W): every rank's pieces in its ring order, each chunk's accumulators shared instead of
+    passed on.  Returns dQ, dK, dV [B, H, N, d] in sequence order."""
+    B, H, N, d = q.shape
+    if N % (2 * W):
+        raise ValueError("N must be a multiple of 2W")
+    cq, ck, cv, co, cdo = (_zigzag_split(t, W) for t in (q, k, v, o, do))
+    _check_chunks(cq + ck + cv + co + cdo, bwd=True)
+    n = N // (2 * W)
+    clse = [lse[:, :, c * n:(c + 1) * n].contiguous() for c in range(2 * W)]
+    for lc, qc in zip(clse, cq):
+        _check_lse(lc, qc)
+    scale = d ** -0.5 if scale is None else scale
+    wsb = fa.fa_bwd_workspace_bytes(B, H, n, d)
+    ws = [torch.empty(wsb, device=q.device, dtype=torch.uint8) for _ in range(2 * W)]
+    for c in range(2 * W):
+        _ok(fa.fa_bwd_prepare(co[c], cdo[c], clse[c], ws[c], wsb, B, H, n, d), "fa_bwd_prepare")
+    dka = [torch.zeros(cq[0].shape, device=q.device, dtype=torch.float32) for _ in range(2 * W)]
+    dva = [torch.zeros_like(t) for t in dka]
+    for r in range(W):
+        a = zigzag_chunks(r, W)
+        for step in range(W):
+            src = (r - step) % W
+            b = zigzag_chunks(src, W)
+            for iq, ik, masked in zigzag_pieces(r, W, src, causal):
+                _ok(fa.fa_bwd_accumulate(cq[a[iq]], ck[b[ik]], cv[b[ik]], cdo[a[iq]], ws[a[iq]], wsb, dka[b[ik]],
+                                         dva[b[ik]], B, H, n, d, scale, masked), "fa_bwd_accumulate")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    for c in range(2 * W):
+        g = [torch.empty_like(cq[c]) for _ in range(3)]
+        _ok(fa.fa_bwd_finish(ws[c], wsb, dka[c], dva[c], *g, B, H, n, d, scale), "fa_bwd_finish")
+        dq[:, :, c * n:(c + 1) * n] = g[0]
+        dk[:, :, c * n:(c + 1) * n] = g[1]
+        dv[:, :, c * n:(c + 1) * n] = g[2]
+    return dq, dk, dv
