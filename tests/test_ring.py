@@ -3,8 +3,9 @@ ranks, partial results merged by the softmax merge of "Flash Attention" (special
 section 增量求解 softmax).
 
 On CPU: the ring exchange itself on spawned gloo ranks (every rank sees every shard, in ring
-order, with the right contents), the choice of pieces under the causal mask, and the C ABI's
-argument checks.  On one GPU: the whole schedule for W virtual ranks, one after the other,
+order, with the right contents), the choice of pieces under the causal mask, the C ABI's
+argument checks, and the whole forward and backward schedule (on one process and on gloo
+ranks) with the piece calls replaced by fp64 stand-ins, against autograd.  On one GPU: the whole schedule for W virtual ranks, one after the other,
 against the fp64 oracle over the full sequence (the multi-GPU run differs only in where the
 shards come from)."""
 import os
@@ -19,6 +20,9 @@ import torch.multiprocessing as mp
 import oracle
 from io_aware_exact_22_b200 import fa, ring
 from io_aware_exact_22_b200.inputs import custom, make_inputs, to_f64
+from tests._fakes import data as fake_data
+from tests._fakes import reference as fake_reference
+from tests._fakes import use_fakes
 from tests._helpers import check_grad, check_lse, check_o, f64
 
 OK, INVALID, UNSUPPORTED = 0, 1, 2
@@ -198,3 +202,58 @@ def test_ring_backward_on_one_gpu(cuda_ok, W, n, causal):
         check_grad(gq[0, h], rq, f"dQ[{h}]")
         check_grad(gk[0, h], rk, f"dK[{h}]")
         check_grad(gv[0, h], rv, f"dV[{h}]")
+
+
+# ------------------------------------------------------------ the schedule with fp64 pieces (CPU)
+@pytest.mark.parametrize("W,n", [(1, 5), (2, 4), (3, 3), (4, 2)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_contiguous_schedule_with_fp64_pieces(monkeypatch, W, n, causal):
+    # the piece calls are replaced by fp64 stand-ins (tests/_fakes.py): this checks the ring's
+    # bookkeeping, the pieces each rank takes and the accumulators shared between ranks
+    use_fakes(monkeypatch.setattr)
+    q, k, v, do = fake_data(2, 3, W * n, 8, seed=W * 10 + n)
+    scale = 8 ** -0.5
+    shard = lambda t: [t[:, :, r * n:(r + 1) * n].contiguous() for r in range(W)]  # noqa: E731
+    fwd = ring.ring_attention_forward_local(shard(q), shard(k), shard(v), causal, scale)
+    o_ref, lse_ref, gq_ref, gk_ref, gv_ref = fake_reference(q, k, v, do, scale, causal)
+    assert torch.allclose(torch.cat([x[0] for x in fwd], 2), o_ref, atol=1e-5)
+    assert torch.allclose(torch.cat([x[1] for x in fwd], 2).double(), lse_ref, atol=1e-5)
+    grads = ring.ring_attention_backward_local(shard(q), shard(k), shard(v), [x[0] for x in fwd], shard(do),
+                                               [x[1] for x in fwd], causal, scale)
+    for i, ref in enumerate((gq_ref, gk_ref, gv_ref)):
+        assert torch.allclose(torch.cat([g[i] for g in grads], 2), ref, atol=1e-5)
+
+
+def _sharded_main(rank, world, port, n, causal, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        use_fakes()
+        q, k, v, do = fake_data(1, 2, world * n, 8, seed=11)
+        scale = 8 ** -0.5
+        cut = lambda t: t[:, :, rank * n:(rank + 1) * n].contiguous()  # noqa: E731
+        o, lse = ring.ring_attention_forward(cut(q), cut(k), cut(v), causal, scale)
+        dq, dk, dv = ring.ring_attention_backward(cut(q), cut(k), cut(v), o, cut(do), lse, causal, scale)
+        o_ref, lse_ref, gq, gk, gv = fake_reference(q, k, v, do, scale, causal)
+        ok = torch.allclose(lse.double(), cut(lse_ref[..., None])[..., 0], atol=1e-5)
+        for got, ref in ((o, o_ref), (dq, gq), (dk, gk), (dv, gv)):
+            ok &= torch.allclose(got, cut(ref), atol=1e-5)
+        out.put((rank, bool(ok)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("causal", [True, False])
+def test_sharded_forward_and_backward_on_gloo_ranks(world, causal):
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_sharded_main, args=(r, world, port, 3, causal, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = dict(out.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res == {r: True for r in range(world)}
