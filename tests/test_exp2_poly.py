@@ -10,7 +10,6 @@ import subprocess
 import sys
 
 import numpy as np
-import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "io_aware_exact_22_b200", "csrc", "sm100_ptx.cuh")

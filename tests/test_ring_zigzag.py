@@ -13,7 +13,6 @@ On one GPU: the same schedule through the library against the fp64 oracle."""
 import os
 import socket
 
-import numpy as np
 import pytest
 import torch
 import torch.distributed as dist

@@ -3,7 +3,6 @@ softmax merge ("Flash Attention", special-jiahao.github.io, section 增量求解
 against the fp64 oracle and against the unsplit forward."""
 import math
 
-import numpy as np
 import pytest
 import torch
 

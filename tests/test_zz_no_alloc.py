@@ -8,7 +8,6 @@ returns, on two calls in a row (the second call runs on scratch the first one le
 and that problems too large for the built-in scratch are refused.  It sits in its own file,
 collected last, so that a failure here never hides the other tests.
 """
-import numpy as np
 import pytest
 import torch
 
