@@ -37,6 +37,8 @@ from io_aware_exact_22_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
 
 METRIC = "attention TFLOPS (fwd/bwd, causal halved) and % of B200 BF16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DATASHEET_BF16_TFLOPS = 2250.0  # B200 dense bf16, NVIDIA's figure (without 2:4 sparsity)
+DATASHEET_HBM_GBS = 8000.0
 
 
 def load_peaks():
@@ -186,38 +188,47 @@ def run_gpu(args):
     scale = w.scale
 
     bwd_fn = fa.fa_bwd_deterministic if args.deterministic else fa.fa_bwd
+    # The timed step launches fa_bwd's three kernels through their own entry points
+    # (fa_bwd_prepare, fa_bwd_main, fa_bwd_dq_post: together exactly fa_bwd), so that CUDA
+    # events between them time the dominant key-tile kernel on its own.
+    split_bwd = not args.deterministic and d == 128
 
-    def step():
+    def launch_step(ev=None):
+        rec = (lambda idx: ev[idx].record(stream)) if ev is not None else (lambda idx: None)
+        rec(0)
         rc = fa.fa_fwd(qd, kd, vd, o, lse, B, H, N, d, scale, w.causal, sp)
-        rc |= bwd_fn(qd, kd, vd, o, dod, lse, dq, dk, dv, ws, ws_bytes, B, H, N, d, scale,
-                     w.causal, sp)
+        rec(1)
+        if split_bwd:
+            rc |= fa.fa_bwd_prepare(o, dod, lse, ws, ws_bytes, B, H, N, d, sp)
+            rec(2)
+            rc |= fa.fa_bwd_main(qd, kd, vd, dod, ws, ws_bytes, dk, dv, B, H, N, d, scale, w.causal, sp)
+            rec(3)
+            rc |= fa.fa_bwd_dq_post(ws, ws_bytes, dq, B, H, N, d, scale, sp)
+        else:
+            rc |= bwd_fn(qd, kd, vd, o, dod, lse, dq, dk, dv, ws, ws_bytes, B, H, N, d, scale,
+                         w.causal, sp)
+            rec(2)
+            rec(3)
+        rec(4)
         if rc:
             raise RuntimeError(f"fa call failed: {rc}")
 
     for _ in range(args.warmup):
-        step()
+        launch_step()
     torch.cuda.synchronize(dev)
     if fa.fa_get_device_status(sp) != 0:
         raise RuntimeError("device-side timeout during warm-up")
 
     clocks = ClockSampler(local)
     clocks.start()
-    n_ev = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_ev)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     t0.record(stream)
     for i in range(args.steps):
-        ev[i][0].record(stream)
-        rc = fa.fa_fwd(qd, kd, vd, o, lse, B, H, N, d, scale, w.causal, sp)
-        ev[i][1].record(stream)
-        rc |= bwd_fn(qd, kd, vd, o, dod, lse, dq, dk, dv, ws, ws_bytes, B, H, N, d, scale,
-                     w.causal, sp)
-        ev[i][2].record(stream)
-        if rc:
-            raise RuntimeError(f"fa call failed: {rc}")
+        launch_step(ev[i])
     t1.record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
@@ -225,9 +236,13 @@ def run_gpu(args):
     clk = clocks.stop()
     status = fa.fa_get_device_status(sp)
     total_ms = t0.elapsed_time(t1)
-    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
-    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
-    total_ms, fwd_ms, bwd_ms = max_over_ranks([total_ms, fwd_ms, bwd_ms], dev)
+
+    def seg(a, b):
+        return statistics.mean(e[a].elapsed_time(e[b]) for e in ev)
+
+    fwd_ms, bwd_ms = seg(0, 1), seg(1, 4)
+    pre_ms, main_ms, post_ms = seg(1, 2), seg(2, 3), seg(3, 4)
+    total_ms, fwd_ms, bwd_ms, main_ms = max_over_ranks([total_ms, fwd_ms, bwd_ms, main_ms], dev)
     ms_per_step = total_ms / args.steps
     flops_step = w.fwd_flops() + w.bwd_flops()
     value = whole_job_tflops(flops_step, world, ms_per_step)
@@ -313,12 +328,19 @@ def run_gpu(args):
         return None
 
     peaks, peak_src = load_peaks()
-    # The step loop keeps the GPU busy for the whole timed region (under the power cap), so the
-    # sustained cuBLAS figure is the denominator; the burst-based fraction is reported too.
-    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    peak_burst = peaks["bf16_tflops"]
+    # The timed region is well under a second of back-to-back steps at the maximum SM clock, so
+    # the denominator is the burst cuBLAS figure; the sustained one (seconds-long loop under
+    # the power cap) and the datasheet's 2250 dense bf16 TFLOP/s are reported beside it.
+    peak = peaks["bf16_tflops"]
+    peak_sus = peaks.get("bf16_tflops_sustained", peak)
     bwd_tflops = w.bwd_flops() / (bwd_ms * 1e-3) / 1e12
     fwd_tflops = w.fwd_flops() / (fwd_ms * 1e-3) / 1e12
+    main_tflops = w.bwd_flops() / (main_ms * 1e-3) / 1e12 if split_bwd else bwd_tflops
+
+    def fracs(tf):
+        return {"frac": round(tf / peak, 4), "frac_of_datasheet": round(tf / DATASHEET_BF16_TFLOPS, 4),
+                "frac_of_sustained": round(tf / peak_sus, 4)}
+
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -333,28 +355,34 @@ def run_gpu(args):
         "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
-                   "step": "fa_fwd + " + ("fa_bwd_deterministic" if args.deterministic else "fa_bwd"),
+                   "step": ("fa_fwd + fa_bwd_prepare + fa_bwd_main + fa_bwd_dq_post (= fa_bwd)"
+                            if split_bwd else "fa_fwd + " + ("fa_bwd_deterministic" if args.deterministic
+                                                             else "fa_bwd")),
                    "per_rank": "same workload on every rank",
                    "l2": l2_note(B * H * N * d * 2)},
         "pct_of_peak": round(100 * value / world / peak, 2),
-        "fwd": {"ms": round(fwd_ms, 4), "tflops": round(fwd_tflops, 1),
-                "pct_of_peak": round(100 * fwd_tflops / peak, 2)},
-        "bwd": {"ms": round(bwd_ms, 4), "tflops": round(bwd_tflops, 1),
-                "pct_of_peak": round(100 * bwd_tflops / peak, 2)},
-        "roofline": {"kernel": "fa_bwd (main kernel + memory-bound pre/post, timed together)",
-                     "bound": "tensor", "achieved": round(bwd_tflops, 1), "peak": peak,
-                     "unit": "TFLOP/s", "frac": round(bwd_tflops / peak, 4),
+        "pct_of_datasheet": round(100 * value / world / DATASHEET_BF16_TFLOPS, 2),
+        "peak_tflops": {"burst": peak, "sustained": peak_sus, "datasheet": DATASHEET_BF16_TFLOPS,
+                        "source": peak_src},
+        "fwd": {"ms": round(fwd_ms, 4), "tflops": round(fwd_tflops, 1), **fracs(fwd_tflops)},
+        "bwd": {"ms": round(bwd_ms, 4), "tflops": round(bwd_tflops, 1), **fracs(bwd_tflops),
+                "kernels_ms": {"fa_bwd_pre_kernel": round(pre_ms, 4), "fa_bwd_main_kernel": round(main_ms, 4),
+                               "fa_bwd_post_kernel": round(post_ms, 4)} if split_bwd else None},
+        "roofline": {"kernel": "fa_bwd_main_kernel<128>" if split_bwd else "backward (all kernels)",
+                     "bound": "tensor", "achieved": round(main_tflops, 1), "peak": peak,
+                     "unit": "TFLOP/s", **fracs(main_tflops),
                      "traffic": kernel_traffic("fa_bwd_main_kernel"),
-                     "peak_source": f"{peak_src} bf16_tflops_sustained",
-                     "frac_of_burst_peak": round(bwd_tflops / peak_burst, 4),
-                     "algorithmic_flops_per_launch": w.bwd_flops()},
+                     "peak_source": f"{peak_src} bf16_tflops (burst)",
+                     "duration_ms": round(main_ms, 4),
+                     "algorithmic_flops_per_launch": w.bwd_flops(),
+                     "note": "the metric's backward FLOPs (2.5x the forward's), all done by this kernel; "
+                             "duration from CUDA events around its launch in every timed step"},
         "roofline_fwd": {"kernel": "fa_fwd_kernel<128>", "bound": "tensor",
                          "achieved": round(fwd_tflops, 1), "peak": peak, "unit": "TFLOP/s",
-                         "frac": round(fwd_tflops / peak, 4),
-                         "frac_of_burst_peak": round(fwd_tflops / peak_burst, 4),
-                         "traffic": kernel_traffic("fa_fwd_kernel"),
+                         **fracs(fwd_tflops), "traffic": kernel_traffic("fa_fwd_kernel"),
                          "algorithmic_flops_per_launch": w.fwd_flops()},
         "clocks": clk,
+        # per step: the forward kernel and the backward's pre, key-tile and dQ kernels
         "gpu_launches": 4 * args.steps,
         "device_status": status,
     }
@@ -363,6 +391,8 @@ def run_gpu(args):
     if not args.no_variants and world == 1:
         line["variants"] = measure_variants(w, dev, stream, qd, kd, vd, o, lse, dod, dq, dk, dv, ws,
                                             ws_bytes, peak)
+    if not args.no_configs and world == 1:
+        line["configs"] = measure_configs(dev, stream, peaks)
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(w, q, k, v, do)
     return line
@@ -483,6 +513,102 @@ def measure_variants(w, dev, stream, qd, kd, vd, o, lse, dod, dq, dk, dv, ws, ws
     return out
 
 
+# ---------------------------------------------------------------------- the other workloads
+L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
+
+
+def _time_flushed_us(fn, stream, flush, iters=20, warmup=3):
+    """Mean device time of fn() in microseconds, each launch timed alone with CUDA events on
+    the launching stream, the L2 flushed before it (a 256 MB buffer is rewritten, outside the
+    events), so that every launch reads its inputs from HBM."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    for i in range(iters):
+        flush.fill_(i & 0xff)
+        evs[i][0].record(stream)
+        fn()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    return 1e3 * statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+
+def _time_warm_us(fn, stream, iters=50, warmup=3):
+    """Mean device time of fn() in microseconds over back-to-back launches (inputs left in L2
+    by the previous launch: the serving case where a layer's inputs were just produced)."""
+    return 1e3 * _time_ms(fn, stream, iters=iters, warmup=warmup)
+
+
+def measure_configs(dev, stream, peaks):
+    """Workloads 1, 2, 3 (forward) and 5 (backward) of the benchmark table, each timed by CUDA
+    events with the L2 flushed before every launch: time, attention TFLOPS (same formulas as
+    the step) against the burst, datasheet and sustained bf16 peaks, and the algorithmic HBM
+    bytes (inputs read and outputs written once) over the time against the measured HBM copy
+    bandwidth, the view that matters for the small, memory-leaning shapes."""
+    from io_aware_exact_22_b200 import fa
+    sp = stream.cuda_stream
+    peak = peaks["bf16_tflops"]
+    peak_sus = peaks.get("bf16_tflops_sustained", peak)
+    hbm = peaks["hbm_gbs"]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    out = {}
+
+    def chk(rc, name):
+        if rc:
+            raise RuntimeError(f"{name} failed: {rc}")
+
+    def entry(w, us, warm_us, flops, nbytes, kernels):
+        tf = flops / (us * 1e-6) / 1e12
+        gbs = nbytes / (us * 1e-6) / 1e9
+        return {"workload": w.name, "kernels": kernels, "us": round(us, 2),
+                "us_l2_warm": round(warm_us, 2), "tflops": round(tf, 1),
+                "frac": round(tf / peak, 4), "frac_of_datasheet": round(tf / DATASHEET_BF16_TFLOPS, 4),
+                "frac_of_sustained": round(tf / peak_sus, 4),
+                "algorithmic_bytes": int(nbytes), "gbs": round(gbs, 1), "frac_of_hbm": round(gbs / hbm, 4),
+                "frac_of_datasheet_hbm": round(gbs / DATASHEET_HBM_GBS, 4),
+                "timing": "CUDA events per launch, L2 flushed (256 MB written) before each of 20 launches"}
+
+    for wid in (1, 2, 3):
+        w = WORKLOADS[wid]
+        B, H, N, d = w.shape
+        q, k, v = (t.to(dev) for t in make_inputs(w, with_grad=False))
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+        fn = lambda: chk(fa.fa_fwd(q, k, v, o, lse, B, H, N, d, w.scale, w.causal, sp), "fa_fwd")  # noqa: E731
+        us = _time_flushed_us(fn, stream, flush)
+        warm = _time_warm_us(fn, stream)
+        out[str(wid)] = entry(w, us, warm, w.fwd_flops(), w.fwd_bytes(), f"fa_fwd_kernel<{d}>")
+        del q, k, v, o, lse
+    w = WORKLOADS[5]
+    B, H, N, d = w.shape
+    q, k, v, do = (t.to(dev) for t in make_inputs(w, with_grad=True))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+    chk(fa.fa_fwd(q, k, v, o, lse, B, H, N, d, w.scale, w.causal, sp), "fa_fwd")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    wsb = fa.fa_bwd_workspace_bytes(B, H, N, d)
+    ws = torch.empty(wsb, device=dev, dtype=torch.uint8)
+    fn = lambda: chk(fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, wsb, B, H, N, d, w.scale, w.causal, sp),  # noqa: E731
+                     "fa_bwd")
+    us = _time_flushed_us(fn, stream, flush)
+    warm = _time_warm_us(fn, stream)
+    out["5"] = entry(w, us, warm, w.bwd_flops(), w.bwd_bytes(),
+                     "fa_bwd_pre_kernel + fa_bwd_main_kernel<128> + fa_bwd_post_kernel")
+    chk(fa.fa_bwd_prepare(o, do, lse, ws, wsb, B, H, N, d, sp), "fa_bwd_prepare")
+    fm = lambda: chk(fa.fa_bwd_main(q, k, v, do, ws, wsb, dk, dv, B, H, N, d, w.scale, w.causal, sp),  # noqa: E731
+                     "fa_bwd_main")
+    us_m = _time_flushed_us(fm, stream, flush)
+    tf = w.bwd_flops() / (us_m * 1e-6) / 1e12
+    out["5"]["main_kernel"] = {"kernel": "fa_bwd_main_kernel<128>", "us": round(us_m, 2), "tflops": round(tf, 1),
+                               "frac": round(tf / peak, 4),
+                               "frac_of_datasheet": round(tf / DATASHEET_BF16_TFLOPS, 4)}
+    del q, k, v, do, o, lse, dq, dk, dv, ws, flush
+    if fa.fa_get_device_status(sp) != 0:
+        raise RuntimeError("device-side timeout while timing the workloads")
+    return out
+
+
 # ---------------------------------------------------------------------- CPU (oracle) arms
 def _blas_threads():
     try:
@@ -558,6 +684,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--deterministic", action="store_true",
                     help="run the step's backward through fa_bwd_deterministic")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the timing of the other benchmark workloads (1, 2, 3, 5)")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the timing of the FP8, deterministic, split-KV and d=64 variants")
     args = ap.parse_args()

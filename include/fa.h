@@ -236,6 +236,23 @@ fa_status_t fa_bwd_finish(const void* workspace, size_t workspace_bytes, const f
                           int B, int H, int N, int d, float scale, void* stream);
 
 /*
+ * fa_bwd (d == 128) taken apart into its three kernels, so that each can be launched, and
+ * timed, on its own.  fa_bwd_prepare (above), then fa_bwd_main, then fa_bwd_dq_post, on one
+ * stream and one workspace, give exactly what fa_bwd gives.
+ *   fa_bwd_main    : the key-tile pass on prepared statistics: recomputes S and P tile by tile,
+ *                    stores dk = scale * dS^T Q and dv = P^T dO (bf16 [B,H,N,d], 16-byte
+ *                    aligned) and adds dS K into the workspace's fp32 dQ accumulator.
+ *                    q, k, v, dO as for fa_bwd.
+ *   fa_bwd_dq_post : dq = scale * accumulator, rounded to bf16 ([B,H,N,d], 16-byte aligned).
+ * Same error rules as fa_bwd; d != 128 returns FA_ERR_UNSUPPORTED.
+ */
+fa_status_t fa_bwd_main(const void* q, const void* k, const void* v, const void* dO,
+                        void* workspace, size_t workspace_bytes, void* dk, void* dv,
+                        int B, int H, int N, int d, float scale, int causal, void* stream);
+fa_status_t fa_bwd_dq_post(const void* workspace, size_t workspace_bytes, void* dq,
+                           int B, int H, int N, int d, float scale, void* stream);
+
+/*
  * Synchronises `stream`, reads and clears the device status word of the current device.
  * Returns FA_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call,
  * FA_ERR_CUDA if the synchronisation itself failed, FA_OK otherwise.

@@ -454,6 +454,46 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   return ld_bytes((long long)B * H, N) + (size_t)rows * d * 4;
 }
 
+// The key-tile kernel of fa_bwd on prepared statistics: bf16 dK, dV stored, dQ added into the
+// workspace's fp32 accumulator.  Arguments are checked by the callers.
+static fa_status_t bwd_main_d128(const void* q, const void* k, const void* v, const void* dO, void* workspace,
+                                 void* dk, void* dv, int BH, int N, float scale, int causal, cudaStream_t s) {
+  const int d = 128;
+  float* ld = reinterpret_cast<float*>(workspace);
+  float* dq_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + ld_bytes(BH, N));
+  CUtensorMap tq, tk, tv, tdo, tdk, tdv, tdq;
+  if (!make_tmap_bf16(&tq, q, BH, N, d, 64) || !make_tmap_bf16(&tk, k, BH, N, d, 128) ||
+      !make_tmap_bf16(&tv, v, BH, N, d, 128) || !make_tmap_bf16(&tdo, dO, BH, N, d, 64) ||
+      !make_tmap_bf16(&tdk, dk, BH, N, d, 32) || !make_tmap_bf16(&tdv, dv, BH, N, d, 32) ||
+      !make_tmap_f32(&tdq, dq_acc, BH, N, d, 32, 64 - kBwdDqRedRows))
+    return FA_ERR_CUDA;
+  BwdArgs a;
+  if (!(a.status = device_status_word())) return FA_ERR_CUDA;
+  a.lse = nullptr;
+  a.ld = ld;
+  a.dq_acc = dq_acc;
+  a.N = N;
+  a.BH = BH;
+  a.causal = causal;
+  a.scale = scale;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  a.block_major = block_major_order(BH, N, d, 2, causal);
+  cudaError_t e = launch_bwd_main(d, tq, tk, tv, tdo, tdk, tdv, tdq, a, s);
+  if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+static fa_status_t check_bwd_io(const void* q, const void* k, const void* v, const void* dO, const void* dk,
+                                const void* dv, const void* workspace, size_t workspace_bytes, int B, int H,
+                                int N, int d) {
+  if (!q || !k || !v || !dO || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dO, 16) || !aligned(dk, 16) ||
+      !aligned(dv, 16) || !aligned(workspace, 256))
+    return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
 fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                    const float* lse, void* dq, void* dk, void* dv, void* workspace,
                    size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
@@ -466,41 +506,45 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
     return fa_bwd_deterministic(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes, B, H, N, d, scale,
                                 causal, stream);
   if (d != 128) return FA_ERR_UNSUPPORTED;
-  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dO, 16) ||
-      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) ||
-      !aligned(workspace, 256))
-    return FA_ERR_INVALID_ARG;
-  if (workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  if ((st = check_bwd_io(q, k, v, dO, dk, dv, workspace, workspace_bytes, B, H, N, d)) != FA_OK) return st;
+  if (!o || !lse || !dq || !aligned(o, 16) || !aligned(dq, 16) || !aligned(lse, 4)) return FA_ERR_INVALID_ARG;
   if ((st = check_device()) != FA_OK) return st;
   const int BH = B * H;
   const long long rows = (long long)BH * N;
   float* ld = reinterpret_cast<float*>(workspace);
   float* dq_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + ld_bytes(BH, N));
   cudaStream_t s = (cudaStream_t)stream;
-  CUtensorMap tq, tk, tv, tdo, tdk, tdv, tdq;
-  if (!make_tmap_bf16(&tq, q, BH, N, d, 64) || !make_tmap_bf16(&tk, k, BH, N, d, 128) ||
-      !make_tmap_bf16(&tv, v, BH, N, d, 128) || !make_tmap_bf16(&tdo, dO, BH, N, d, 64) ||
-      !make_tmap_bf16(&tdk, dk, BH, N, d, 32) || !make_tmap_bf16(&tdv, dv, BH, N, d, 32) ||
-      !make_tmap_f32(&tdq, dq_acc, BH, N, d, 32, 64 - kBwdDqRedRows))
-    return FA_ERR_CUDA;
-  BwdArgs a;
-  if (!(a.status = device_status_word())) return FA_ERR_CUDA;
-  a.lse = lse;
-  a.ld = ld;
-  a.dq_acc = dq_acc;
-  a.N = N;
-  a.BH = BH;
-  a.causal = causal;
-  a.scale = scale;
-  a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
-  a.block_major = block_major_order(BH, N, d, 2, causal);
   if (launch_bwd_pre(o, dO, lse, ld, dq_acc, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
-  cudaError_t e = launch_bwd_main(d, tq, tk, tv, tdo, tdk, tdv, tdq, a, s);
-  if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
-  if (e != cudaSuccess) return FA_ERR_CUDA;
+  if ((st = bwd_main_d128(q, k, v, dO, workspace, dk, dv, BH, N, scale, causal, s)) != FA_OK) return st;
   if (launch_bwd_post(dq_acc, dq, rows * d, scale, s) != cudaSuccess) return FA_ERR_CUDA;
   return FA_OK;
+}
+
+fa_status_t fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* workspace,
+                        size_t workspace_bytes, void* dk, void* dv, int B, int H, int N, int d, float scale,
+                        int causal, void* stream) {
+  bool empty = false;
+  fa_status_t st = check_shape(B, H, N, d, scale, causal, &empty);
+  if (st != FA_OK || empty) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if ((st = check_bwd_io(q, k, v, dO, dk, dv, workspace, workspace_bytes, B, H, N, d)) != FA_OK) return st;
+  if ((st = check_device()) != FA_OK) return st;
+  return bwd_main_d128(q, k, v, dO, workspace, dk, dv, B * H, N, scale, causal, (cudaStream_t)stream);
+}
+
+fa_status_t fa_bwd_dq_post(const void* workspace, size_t workspace_bytes, void* dq, int B, int H, int N, int d,
+                           float scale, void* stream) {
+  bool empty = false;
+  fa_status_t st = check_shape(B, H, N, d, scale, 0, &empty);
+  if (st != FA_OK || empty) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (!workspace || !dq || !aligned(workspace, 256) || !aligned(dq, 16)) return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  if ((st = check_device()) != FA_OK) return st;
+  const long long rows = (long long)B * H * N;
+  const float* dq_acc =
+      reinterpret_cast<const float*>(reinterpret_cast<const char*>(workspace) + ld_bytes((long long)B * H, N));
+  return launch_bwd_post(dq_acc, dq, rows * d, scale, (cudaStream_t)stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 fa_status_t fa_bwd_prepare(const void* o, const void* dO, const float* lse, void* workspace, size_t workspace_bytes,

@@ -26,7 +26,7 @@ EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_device_status",
            "fa_status_string", "fa_version", "fa_bwd_noalloc", "fa_selftest_wait_timeout",
            "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_default_splits",
            "fa_bwd_deterministic", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials",
-           "fa_bwd_prepare", "fa_bwd_accumulate", "fa_bwd_finish")
+           "fa_bwd_prepare", "fa_bwd_accumulate", "fa_bwd_finish", "fa_bwd_main", "fa_bwd_dq_post")
 # Size of the library's built-in scratch used by fa_bwd_noalloc (include/fa.h).
 NOALLOC_MAX_SCRATCH_BYTES = 64 << 20
 
@@ -62,6 +62,10 @@ def lib() -> ctypes.CDLL:
         L.fa_bwd_accumulate.restype = i
         L.fa_bwd_finish.argtypes = [vp, sz, vp, vp, vp, vp, vp, i, i, i, i, f, vp]
         L.fa_bwd_finish.restype = i
+        L.fa_bwd_main.argtypes = [vp, vp, vp, vp, vp, sz, vp, vp, i, i, i, i, f, i, vp]
+        L.fa_bwd_main.restype = i
+        L.fa_bwd_dq_post.argtypes = [vp, sz, vp, i, i, i, i, f, vp]
+        L.fa_bwd_dq_post.restype = i
         L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, vp]
         L.fa_bwd.restype = i
         L.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
@@ -143,6 +147,17 @@ def fa_bwd_finish(workspace, workspace_bytes, dk_acc, dv_acc, dq, dk, dv, B, H, 
                   stream=None) -> int:
     return lib().fa_bwd_finish(_ptr(workspace), int(workspace_bytes), _ptr(dk_acc), _ptr(dv_acc),
                                _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale), _stream(stream))
+
+
+def fa_bwd_main(q, k, v, dO, workspace, workspace_bytes, dk, dv, B, H, N, d, scale, causal,
+                stream=None) -> int:
+    return lib().fa_bwd_main(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(workspace), int(workspace_bytes),
+                             _ptr(dk), _ptr(dv), B, H, N, d, float(scale), int(causal), _stream(stream))
+
+
+def fa_bwd_dq_post(workspace, workspace_bytes, dq, B, H, N, d, scale, stream=None) -> int:
+    return lib().fa_bwd_dq_post(_ptr(workspace), int(workspace_bytes), _ptr(dq), B, H, N, d, float(scale),
+                                _stream(stream))
 
 
 def fa_fwd_splitkv(q, k, v, o, lse, B, H, N, d, scale, causal, num_splits, workspace,

@@ -38,12 +38,13 @@ ZERO_RMS = 1e-9
 ZERO_MAX_ABS = 1e-4
 
 
-# Output rounding: a bf16 result is at best within half an ulp (2^-9 relative) of the exact
-# value, which exceeds the 5e-2 absolute budget once |value| > 25.6.  For shapes outside the
-# five benchmark workloads whose gradients grow that large (the long-sequence backward with
-# q, k ~ N(0, 3)), the bound is 5e-2 + 2^-8 |reference|: the absolute budget plus one bf16
-# ulp of the value.
+# Output rounding: a bf16 value in [2^e, 2^(e+1)) is rounded to a multiple of 2^(e-7), so half
+# an ulp is 2^(e-8): 0.0625 from |value| = 16 on, more than the whole 5e-2 budget.  Where a
+# reference gradient reaches |value| >= 16 (the long-sequence backward with q, k ~ N(0, 3)),
+# that element alone is held to 5e-2 + 2^-8 |reference| (the budget plus at most one bf16 ulp
+# of the value); every smaller element keeps the plain 5e-2.
 BF16_ULP_REL = 2.0 ** -8
+ULP_SLACK_FROM = 16.0
 
 
 def check_grad(g_gpu: np.ndarray, g_ref: np.ndarray, what: str, rel_tol: float = GRAD_REL_L2,
@@ -51,8 +52,12 @@ def check_grad(g_gpu: np.ndarray, g_ref: np.ndarray, what: str, rel_tol: float =
     assert np.isfinite(g_gpu).all(), f"{what}: non-finite values"
     err = np.abs(g_gpu - g_ref)
     if ulp_slack:
-        excess = err - (GRAD_MAX_ABS + BF16_ULP_REL * np.abs(g_ref))
-        assert excess.max() <= 0, f"{what}: error exceeds 5e-2 + 2^-8|ref| by {excess.max():.3e}"
+        big = np.abs(g_ref) >= ULP_SLACK_FROM
+        check_grad.slack_elements += int(big.sum())
+        small_err = err[~big].max() if (~big).any() else 0.0
+        assert small_err <= GRAD_MAX_ABS, f"{what}: max-abs {small_err:.3e} > {GRAD_MAX_ABS} where |ref| < 16"
+        excess = err[big] - (GRAD_MAX_ABS + BF16_ULP_REL * np.abs(g_ref[big]))
+        assert excess.size == 0 or excess.max() <= 0, f"{what}: error exceeds 5e-2 + 2^-8|ref| by {excess.max():.3e}"
     else:
         assert err.max() <= GRAD_MAX_ABS, f"{what}: max-abs {err.max():.3e} > {GRAD_MAX_ABS}"
     ref_norm = np.linalg.norm(g_ref)
@@ -62,3 +67,7 @@ def check_grad(g_gpu: np.ndarray, g_ref: np.ndarray, what: str, rel_tol: float =
     rel = np.linalg.norm(g_gpu - g_ref) / ref_norm
     assert rel <= rel_tol, f"{what}: rel-L2 {rel:.3e} > {rel_tol}"
     return err.max(), rel
+
+
+# number of elements checked under the ulp allowance (a test using it asserts that it is > 0)
+check_grad.slack_elements = 0

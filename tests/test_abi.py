@@ -124,3 +124,36 @@ def test_library_is_the_in_tree_build():
     path = fa.LIB_PATH
     assert os.path.dirname(os.path.abspath(path)) == os.path.join(ROOT, "io_aware_exact_22_b200")
     assert isinstance(fa.lib(), ctypes.CDLL)
+
+
+def _bwd_main(**kw):
+    args = dict(q=A16, k=A16, v=A16, dO=A16, ws=A16, wsb=1 << 40, dk=A16, dv=A16, B=1, H=1, N=128,
+                d=128, scale=0.125, causal=1, stream=0)
+    args.update(kw)
+    return fa.fa_bwd_main(args["q"], args["k"], args["v"], args["dO"], args["ws"], args["wsb"],
+                          args["dk"], args["dv"], args["B"], args["H"], args["N"], args["d"],
+                          args["scale"], args["causal"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), INVALID), (dict(dO=0), INVALID), (dict(ws=0), INVALID), (dict(dv=0), INVALID),
+    (dict(ws=A16 + 16), INVALID), (dict(dk=A16 + 8), INVALID), (dict(wsb=10), INVALID),
+    (dict(d=64), UNSUPPORTED), (dict(d=96), UNSUPPORTED), (dict(N=-1), INVALID),
+    (dict(scale=0.0), INVALID), (dict(causal=2), INVALID),
+])
+def test_backward_main_rejects_bad_arguments(kw, code):
+    assert _bwd_main(**kw) == code
+
+
+@pytest.mark.parametrize("args,code", [
+    ((0, 1 << 40, A16, 1, 1, 128, 128, 0.1), INVALID),
+    ((A16, 1 << 40, 0, 1, 1, 128, 128, 0.1), INVALID),
+    ((A16 + 16, 1 << 40, A16, 1, 1, 128, 128, 0.1), INVALID),
+    ((A16, 1 << 40, A16 + 4, 1, 1, 128, 128, 0.1), INVALID),
+    ((A16, 100, A16, 1, 1, 128, 128, 0.1), INVALID),
+    ((A16, 1 << 40, A16, 1, 1, 128, 64, 0.1), UNSUPPORTED),
+    ((A16, 1 << 40, A16, 1, 1, 128, 128, -1.0), INVALID),
+    ((A16, 1 << 40, A16, 1, 1, 0, 128, 0.1), OK),
+])
+def test_backward_dq_post_rejects_bad_arguments(args, code):
+    assert fa.fa_bwd_dq_post(*args, 0) == code

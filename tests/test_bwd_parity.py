@@ -65,17 +65,22 @@ def test_large_scores(cuda_ok):
 
 
 def test_backward_workload_full_size(cuda_ok):
-    # B=2, H=16, N=4096, d=128, causal: two heads checked element by element.
-    _check_heads(WORKLOADS[5], heads=[(0, 0), (1, 15)])
+    # B=2, H=16, N=4096, d=128, causal: eight heads checked element by element.
+    _check_heads(WORKLOADS[5], heads=[(0, 0), (0, 5), (0, 10), (0, 15), (1, 0), (1, 6), (1, 11), (1, 15)])
 
 
-def test_long_sequence_backward_sampled_head(cuda_ok):
-    # The benchmark's training step runs the backward at the long-sequence shape too.
+def test_long_sequence_backward_full_heads(cuda_ok):
+    # The benchmark's step runs the backward at the long-sequence shape (dO from seed 1, as
+    # bench.py draws it): four of the 32 heads, every element.  With q, k ~ N(0, 3) some
+    # gradients reach |g| >= 16, where half a bf16 ulp (0.0625) alone exceeds the 5e-2 budget;
+    # only those elements get the one-ulp allowance (and the test asserts that they occur).
     w = WORKLOADS[4]
     q, k, v = make_inputs(w, with_grad=False)
     g = torch.Generator("cpu").manual_seed(1)
     do = torch.randn(w.shape, generator=g).to(torch.bfloat16)
-    _check_heads(w, heads=[(0, 5)], inputs=(q, k, v, do), ulp_slack=True)
+    check_grad.slack_elements = 0
+    _check_heads(w, heads=[(0, 0), (0, 5), (0, 19), (0, 31)], inputs=(q, k, v, do), ulp_slack=True)
+    assert check_grad.slack_elements > 0, "no |ref| >= 16: the ulp allowance would not be needed"
 
 
 def test_zero_upstream_gradient(cuda_ok):
@@ -93,3 +98,22 @@ def test_repeatable_up_to_atomic_order(cuda_ok):
     # dK and dV are accumulated in a fixed order; dQ uses atomics whose order may vary.
     assert np.array_equal(dk1, dk2) and np.array_equal(dv1, dv2)
     assert np.abs(dq1 - dq2).max() <= 2e-2
+
+
+def test_three_step_backward_equals_fa_bwd(cuda_ok):
+    # fa_bwd_prepare, fa_bwd_main, fa_bwd_dq_post launch exactly fa_bwd's kernels
+    w = custom(2, 2, 777, 128, True, seed=17, backward=True)
+    q, k, v, do = (t.cuda() for t in make_inputs(w))
+    o, lse = fa.forward(q, k, v, True, w.scale)
+    ref = fa.backward(q, k, v, o, do, lse, True, w.scale)
+    B, H, N, d = w.shape
+    wsb = fa.fa_bwd_workspace_bytes(B, H, N, d)
+    ws = torch.empty(wsb, device="cuda", dtype=torch.uint8)
+    dq, dk, dv = (torch.full_like(q, float("nan")) for _ in range(3))
+    assert fa.fa_bwd_prepare(o, do, lse, ws, wsb, B, H, N, d) == 0
+    assert fa.fa_bwd_main(q, k, v, do, ws, wsb, dk, dv, B, H, N, d, w.scale, 1) == 0
+    assert fa.fa_bwd_dq_post(ws, wsb, dq, B, H, N, d, w.scale) == 0
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status() == 0
+    assert torch.equal(dk, ref[1]) and torch.equal(dv, ref[2])
+    check_grad(f64(dq), f64(ref[0]), "dQ (three steps vs fa_bwd)")

@@ -58,20 +58,29 @@ def test_large_scores_stress_rescale(cuda_ok):
     _full_check(custom(1, 2, 1024, 64, False, seed=4, qk_std=3.0))
 
 
-def test_causal_workload_sampled(cuda_ok):
+def test_causal_workload_full_heads(cuda_ok):
+    # B=2, H=16, N=4096, d=128, causal: 8 of the 32 heads element by element, sampled rows of
+    # the others.
     w = WORKLOADS[3]
-    _sampled_check(w, heads=[(0, 0), (1, 15)], rows_per_head=48)
+    (q, k, v), o, lse = _run(w)
+    o, lse = f64(o), f64(lse)
+    for b, h in [(0, 0), (0, 5), (0, 10), (0, 15), (1, 0), (1, 6), (1, 11), (1, 15)]:
+        o_ref, l_ref = oracle.attention_forward_head(to_f64(q[b, h]), to_f64(k[b, h]), to_f64(v[b, h]),
+                                                     w.scale, w.causal)
+        check_o(o[b, h], o_ref, f"O[{b},{h}]")
+        check_lse(lse[b, h], l_ref)
+    _sampled_rows_check(w, (q, k, v), o, lse, [(b, h) for b in range(2) for h in range(16)], 24)
 
 
 def test_long_sequence_workload_sampled(cuda_ok):
-    # Full size, in the launch configuration the benchmark times.
+    # Full size, in the launch configuration the benchmark times: sampled rows of all 32 heads.
     w = WORKLOADS[4]
-    _sampled_check(w, heads=[(0, 0), (0, 13), (0, 31)], rows_per_head=40)
-
-
-def _sampled_check(w, heads, rows_per_head):
     (q, k, v), o, lse = _run(w)
-    o, lse = f64(o), f64(lse)
+    _sampled_rows_check(w, (q, k, v), f64(o), f64(lse), [(0, h) for h in range(32)], 52)
+
+
+def _sampled_rows_check(w, inputs, o, lse, heads, rows_per_head):
+    q, k, v = inputs
     rng = np.random.default_rng(0)
     N = w.N
     fixed = np.array([0, 1, 127, 128, 129, 255, 256, N // 2, N - 129, N - 128, N - 2, N - 1])
