@@ -456,22 +456,33 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
 
 // The key-tile kernel of fa_bwd on prepared statistics: bf16 dK, dV stored, dQ added into the
 // workspace's fp32 accumulator.  Arguments are checked by the callers.
+// The key-tile kernel of fa_bwd on prepared statistics: bf16 dK, dV stored (or, with dk_acc set,
+// scale * dK and dV added into fp32 accumulators), dQ added into the workspace's fp32
+// accumulator.  Arguments are checked by the callers.
 static fa_status_t bwd_main_d128(const void* q, const void* k, const void* v, const void* dO, void* workspace,
-                                 void* dk, void* dv, int BH, int N, float scale, int causal, cudaStream_t s) {
+                                 void* dk, void* dv, int BH, int N, float scale, int causal, cudaStream_t s,
+                                 float* dk_acc = nullptr, float* dv_acc = nullptr) {
   const int d = 128;
   float* ld = reinterpret_cast<float*>(workspace);
   float* dq_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + ld_bytes(BH, N));
   CUtensorMap tq, tk, tv, tdo, tdk, tdv, tdq;
   if (!make_tmap_bf16(&tq, q, BH, N, d, 64) || !make_tmap_bf16(&tk, k, BH, N, d, 128) ||
       !make_tmap_bf16(&tv, v, BH, N, d, 128) || !make_tmap_bf16(&tdo, dO, BH, N, d, 64) ||
-      !make_tmap_bf16(&tdk, dk, BH, N, d, 32) || !make_tmap_bf16(&tdv, dv, BH, N, d, 32) ||
       !make_tmap_f32(&tdq, dq_acc, BH, N, d, 32, 64 - kBwdDqRedRows))
     return FA_ERR_CUDA;
+  if (dk_acc == nullptr) {
+    if (!make_tmap_bf16(&tdk, dk, BH, N, d, 32) || !make_tmap_bf16(&tdv, dv, BH, N, d, 32)) return FA_ERR_CUDA;
+  } else {
+    tdk = tk;  // accumulate mode: the bf16 store maps are not used; any valid map fills them
+    tdv = tv;
+  }
   BwdArgs a;
   if (!(a.status = device_status_word())) return FA_ERR_CUDA;
   a.lse = nullptr;
   a.ld = ld;
   a.dq_acc = dq_acc;
+  a.dk_acc = dk_acc;
+  a.dv_acc = dv_acc;
   a.N = N;
   a.BH = BH;
   a.causal = causal;
@@ -577,30 +588,8 @@ fa_status_t fa_bwd_accumulate(const void* q, const void* k, const void* v, const
     return FA_ERR_INVALID_ARG;
   if (workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
   if ((st = check_device()) != FA_OK) return st;
-  const int BH = B * H;
-  float* ld = reinterpret_cast<float*>(workspace);
-  float* dq_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + ld_bytes(BH, N));
-  CUtensorMap tq, tk, tv, tdo, tdq;
-  if (!make_tmap_bf16(&tq, q, BH, N, d, 64) || !make_tmap_bf16(&tk, k, BH, N, d, 128) ||
-      !make_tmap_bf16(&tv, v, BH, N, d, 128) || !make_tmap_bf16(&tdo, dO, BH, N, d, 64) ||
-      !make_tmap_f32(&tdq, dq_acc, BH, N, d, 32, 64 - kBwdDqRedRows))
-    return FA_ERR_CUDA;
-  BwdArgs a;
-  if (!(a.status = device_status_word())) return FA_ERR_CUDA;
-  a.lse = nullptr;
-  a.ld = ld;
-  a.dq_acc = dq_acc;
-  a.dk_acc = dk_acc;
-  a.dv_acc = dv_acc;
-  a.N = N;
-  a.BH = BH;
-  a.causal = causal;
-  a.scale = scale;
-  a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
-  a.block_major = block_major_order(BH, N, d, 2, causal);
-  // the dK/dV store maps are not used in accumulate mode; any valid map fills the parameters
-  return launch_bwd_main(d, tq, tk, tv, tdo, tk, tv, tdq, a, (cudaStream_t)stream) == cudaSuccess ? FA_OK
-                                                                                                  : FA_ERR_CUDA;
+  return bwd_main_d128(q, k, v, dO, workspace, nullptr, nullptr, B * H, N, scale, causal, (cudaStream_t)stream,
+                       dk_acc, dv_acc);
 }
 
 fa_status_t fa_bwd_finish(const void* workspace, size_t workspace_bytes, const float* dk_acc, const float* dv_acc,

@@ -66,10 +66,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Bounded wait for the phase with the given parity.  Returns false when the CTA-wide abort
 // flag is raised or the time limit runs out (then it raises the CTA flag and the device
-// status word), so that every waiter leaves its loop and the kernel exits.  The slow path is
-// kept out of line so that hot loops only carry the first probe.
-static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                            uint32_t* status) {
+// status word), so that every waiter leaves its loop and the kernel exits.
+__device__ __forceinline__ bool mbar_wait_loop(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                               uint32_t* status) {
   const uint64_t t0 = globaltimer();
   uint32_t it = 0;
   while (true) {
@@ -88,9 +87,20 @@ static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity
     }
   }
 }
+// The slow path is kept out of line so that hot loops only carry the first probe.
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                   uint32_t* status) {
+  return mbar_wait_loop(bar, parity, abort_flag, status);
+}
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& w) {
   if (mbar_try_wait(bar, parity)) return true;
   return mbar_wait_slow(bar, parity, w.abort_flag, w.status);
+}
+// The same wait with the slow path inlined, for kernels that rebalance registers with
+// setmaxnreg: code under a raised register budget cannot call out of line.
+__device__ __forceinline__ bool mbar_wait_inl(uint32_t bar, uint32_t parity, const WaitCtx& w) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_loop(bar, parity, w.abort_flag, w.status);
 }
 
 // Wait used only on the abort path, to let copies already in flight land before exit.

@@ -38,26 +38,57 @@ ZERO_RMS = 1e-9
 ZERO_MAX_ABS = 1e-4
 
 
-# Output rounding: a bf16 value in [2^e, 2^(e+1)) is rounded to a multiple of 2^(e-7), so half
-# an ulp is 2^(e-8): 0.0625 from |value| = 16 on, more than the whole 5e-2 budget.  Where a
-# reference gradient reaches |value| >= 16 (the long-sequence backward with q, k ~ N(0, 3)),
-# that element alone is held to 5e-2 + 2^-8 |reference| (the budget plus at most one bf16 ulp
-# of the value); every smaller element keeps the plain 5e-2.
-BF16_ULP_REL = 2.0 ** -8
-ULP_SLACK_FROM = 16.0
+# A tolerance for shapes outside the five benchmark workloads whose gradients are large and
+# cancelling (the long-sequence backward with q, k ~ N(0, 3)), derived from the arithmetic:
+#  * the kernel rounds dS (and P) to bf16 before the tensor-core products dK = scale dS^T Q,
+#    dQ = scale dS K, dV = P^T dO; bf16 has an 8-bit significand, so each product term moves
+#    by at most 2^-8 of its magnitude, and an element by at most 2^-8 T, T the sum of its
+#    terms' absolute values (the standard a-priori bound of a sum of rounded terms);
+#  * its output is rounded to bf16, which adds up to half an ulp of the value: 2^(e-8) for a
+#    value in [2^e, 2^(e+1)), 0.0625 from |value| = 16 on;
+#  * everything else (fp32 accumulation, the exponential, D from the bf16 O) stays within the
+#    stated 5e-2.
+# So each element is held to  5e-2 + 2^-8 T + halfulp_bf16(|ref| + 5e-2),  with T from
+# abs_term_sums (fp64, the oracle's own pinned score and softmax steps), and rel-L2 stays at
+# 1e-2.  The five benchmark workloads use the plain 5e-2.
+BF16_U = 2.0 ** -8
+
+
+def halfulp_bf16(x: np.ndarray) -> np.ndarray:
+    x = np.maximum(np.abs(x), 2.0 ** -126)
+    return np.exp2(np.floor(np.log2(x)) - 8.0)
+
+
+def abs_term_sums(q, k, v, do, scale: float, causal: bool, row_chunk: int = 2048):
+    """For one head (fp64 [N, d] arrays): the sums of absolute values of the terms of every
+    gradient element, T_Q = scale |dS| |K|, T_K = scale |dS|^T |Q|, T_V = |P|^T |dO|, with P and
+    dS = P o (dO V^T - D) formed by the oracle's score and softmax steps."""
+    import oracle
+    N = q.shape[0]
+    tq = np.zeros_like(q)
+    tk = np.zeros_like(k)
+    tv = np.zeros_like(v)
+    ak, aq, ado = np.abs(k), np.abs(q), np.abs(do)
+    for c0 in range(0, N, row_chunk):
+        r = np.arange(c0, min(N, c0 + row_chunk))
+        p, _, _ = oracle.softmax_rows(oracle.scaled_scores(q, k, scale, causal, r))
+        dp = do[r] @ v.T
+        ds = np.abs(p * (dp - (p * dp).sum(axis=-1, keepdims=True)))
+        tq[r] = scale * (ds @ ak)
+        tk += scale * (ds.T @ aq[r])
+        tv += p.T @ ado[r]
+    return tq, tk, tv
 
 
 def check_grad(g_gpu: np.ndarray, g_ref: np.ndarray, what: str, rel_tol: float = GRAD_REL_L2,
-               ulp_slack: bool = False):
+               term_sums: np.ndarray | None = None):
     assert np.isfinite(g_gpu).all(), f"{what}: non-finite values"
     err = np.abs(g_gpu - g_ref)
-    if ulp_slack:
-        big = np.abs(g_ref) >= ULP_SLACK_FROM
-        check_grad.slack_elements += int(big.sum())
-        small_err = err[~big].max() if (~big).any() else 0.0
-        assert small_err <= GRAD_MAX_ABS, f"{what}: max-abs {small_err:.3e} > {GRAD_MAX_ABS} where |ref| < 16"
-        excess = err[big] - (GRAD_MAX_ABS + BF16_ULP_REL * np.abs(g_ref[big]))
-        assert excess.size == 0 or excess.max() <= 0, f"{what}: error exceeds 5e-2 + 2^-8|ref| by {excess.max():.3e}"
+    if term_sums is not None:
+        bound = GRAD_MAX_ABS + BF16_U * term_sums + halfulp_bf16(np.abs(g_ref) + GRAD_MAX_ABS)
+        excess = err - bound
+        assert excess.max() <= 0, f"{what}: error exceeds 5e-2 + 2^-8 T + half a bf16 ulp by {excess.max():.3e}"
+        check_grad.over_budget += int((err > GRAD_MAX_ABS).sum())
     else:
         assert err.max() <= GRAD_MAX_ABS, f"{what}: max-abs {err.max():.3e} > {GRAD_MAX_ABS}"
     ref_norm = np.linalg.norm(g_ref)
@@ -69,5 +100,5 @@ def check_grad(g_gpu: np.ndarray, g_ref: np.ndarray, what: str, rel_tol: float =
     return err.max(), rel
 
 
-# number of elements checked under the ulp allowance (a test using it asserts that it is > 0)
-check_grad.slack_elements = 0
+# elements over the plain 5e-2 that the derived bound admitted (reported by the test using it)
+check_grad.over_budget = 0

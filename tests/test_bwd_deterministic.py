@@ -48,12 +48,12 @@ def _run(w, inputs=None, deterministic=True):
     return (q, k, v, do), grads
 
 
-def _check(w, heads=None, inputs=None, rel_tol=None, ulp_slack=False):
+def _check(w, heads=None, inputs=None, rel_tol=None):
     (q, k, v, do), grads = _run(w, inputs)
     dq, dk, dv = (f64(g) for g in grads)
     if heads is None:
         heads = [(b, h) for b in range(w.B) for h in range(w.H)]
-    kw = dict(ulp_slack=ulp_slack)
+    kw = {}
     if rel_tol is not None:
         kw["rel_tol"] = rel_tol
     for b, h in heads:
