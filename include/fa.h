@@ -57,7 +57,8 @@ typedef enum {
   FA_ERR_INVALID_ARG = 1,
   FA_ERR_UNSUPPORTED = 2,
   FA_ERR_CUDA = 3,
-  FA_ERR_TIMEOUT = 4
+  FA_ERR_TIMEOUT = 4,
+  FA_ERR_DEVICE_CHECK = 5
 } fa_status_t;
 
 /*
@@ -255,7 +256,9 @@ fa_status_t fa_bwd_dq_post(const void* workspace, size_t workspace_bytes, void* 
 /*
  * Synchronises `stream`, reads and clears the device status word of the current device.
  * Returns FA_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call,
- * FA_ERR_CUDA if the synchronisation itself failed, FA_OK otherwise.
+ * FA_ERR_DEVICE_CHECK if a device-side check failed (a full-TMEM allocation that did not start
+ * at column 0, or, in the debug build, an index outside its range), FA_ERR_CUDA if the
+ * synchronisation itself failed, FA_OK otherwise.
  */
 fa_status_t fa_get_device_status(void* stream);
 
@@ -270,6 +273,24 @@ fa_status_t fa_get_device_status(void* stream);
  * so read the status before launching anything else.
  */
 fa_status_t fa_selftest_wait_timeout(int limit_ms, void* stream);
+
+/*
+ * Debug build (libfa_debug.so: the same sources compiled with FA_DEBUG; no counterpart on the
+ * pages, it stands in for a memory checker).  Its kernels check their tile indices and global
+ * offsets on the device (a failed check skips the access and sets a status bit that
+ * fa_get_device_status reports as FA_ERR_DEVICE_CHECK; nothing traps) and count the tile pairs
+ * they visit, per kernel kind, in three blocks of 2^20 int counters kept by the library:
+ *   block 0, forward kernel:           [B*H][ceil(N/128) query tiles][ceil(N/128) key blocks]
+ *   block 1, backward key-tile kernel: [B*H][ceil(N/64) query tiles][ceil(N/128) key tiles]
+ *   block 2, deterministic dQ kernel:  [B*H][ceil(N/128) query tiles][ceil(N/64) key blocks]
+ * (row-major, one count per visit of the pair).
+ * fa_debug_build      : 1 in the debug build, 0 in the release build.
+ * fa_debug_visits     : synchronises `stream`, copies the first n counters (n <= 3 * 2^20,
+ *                       block b starting at b * 2^20) to the host array `counts`, then zeroes
+ *                       all of them when clear != 0.  FA_ERR_UNSUPPORTED in the release build.
+ */
+int fa_debug_build(void);
+fa_status_t fa_debug_visits(int* counts, size_t n, int clear, void* stream);
 
 /* Static, human-readable name of a status code. */
 const char* fa_status_string(fa_status_t s);

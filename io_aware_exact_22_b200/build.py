@@ -1,6 +1,8 @@
-"""Builds libfa.so in-tree (io_aware_exact_22_b200/libfa.so) with nvcc for sm_100a.
+"""Builds libfa.so in-tree (io_aware_exact_22_b200/libfa.so) with nvcc for sm_100a, and the
+debug build libfa_debug.so (the same sources with FA_DEBUG: device-side index checks and tile
+visit counters, see include/fa.h).
 
-    python -m io_aware_exact_22_b200.build [--force] [--verbose]
+    python -m io_aware_exact_22_b200.build [--force] [--verbose] [--debug | --all]
 
 Each .cu file under csrc/ is compiled to an object in _build/ (skipped when the object is
 newer than every source and header), then linked into one shared library against the static
@@ -23,6 +25,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libfa.so")
+BUILD_DEBUG = os.path.join(ROOT, "_build_debug")
+LIB_DEBUG = os.path.join(PKG, "libfa_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-O3",
@@ -51,17 +55,19 @@ def _stale(target: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_v: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, ptxas_v: bool = False, debug: bool = False) -> str:
+    bdir, lib = (BUILD_DEBUG, LIB_DEBUG) if debug else (BUILD, LIB)
+    flags = FLAGS + (["-DFA_DEBUG"] if debug else [])
+    os.makedirs(bdir, exist_ok=True)
     cc = nvcc()
     headers = _headers()
     objs = []
     jobs = []
     for src in _sources():
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(bdir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if force or _stale(obj, [src] + headers):
-            cmd = [cc, *ARCH, *FLAGS, "-c", src, "-o", obj]
+            cmd = [cc, *ARCH, *flags, "-c", src, "-o", obj]
             if ptxas_v:
                 cmd.insert(1, "-Xptxas=-v")
             jobs.append(cmd)
@@ -79,15 +85,15 @@ def build(force: bool = False, verbose: bool = False, ptxas_v: bool = False) -> 
                 sys.stderr.write(r.stderr)
             if r.returncode != 0:
                 raise RuntimeError(f"nvcc failed: {' '.join(cmd)}")
-    if force or jobs or _stale(LIB, objs):
-        cmd = [cc, *ARCH, "-shared", "-o", LIB, *objs, "-Xcompiler", "-fPIC"]
+    if force or jobs or _stale(lib, objs):
+        cmd = [cc, *ARCH, "-shared", "-o", lib, *objs, "-Xcompiler", "-fPIC"]
         if verbose:
             print(" ".join(cmd), flush=True)
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)
             raise RuntimeError("link failed")
-    return LIB
+    return lib
 
 
 def main():
@@ -95,8 +101,13 @@ def main():
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-v", action="store_true", help="print register/smem usage")
+    ap.add_argument("--debug", action="store_true", help="build libfa_debug.so only")
+    ap.add_argument("--all", action="store_true", help="build libfa.so and libfa_debug.so")
     args = ap.parse_args()
-    print(build(force=args.force, verbose=args.verbose, ptxas_v=args.ptxas_v))
+    if args.all or not args.debug:
+        print(build(force=args.force, verbose=args.verbose, ptxas_v=args.ptxas_v))
+    if args.all or args.debug:
+        print(build(force=args.force, verbose=args.verbose, ptxas_v=args.ptxas_v, debug=True))
 
 
 if __name__ == "__main__":

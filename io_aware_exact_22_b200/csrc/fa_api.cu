@@ -2,6 +2,7 @@
 // TMA tensor-map encoding and kernel launches.  No exception crosses this boundary and no
 // device memory is allocated here.
 #include "fa.h"
+#include "fa_debug.cuh"
 #include "fa_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -19,6 +20,27 @@
 namespace fa {
 
 __device__ uint32_t g_fa_status = 0;
+
+#ifdef FA_DEBUG
+// Visit counters of the debug build: three blocks of kDebugVisitInts ints (see debug_visits).
+__device__ int g_fa_visits[3 * kDebugVisitInts];
+#endif
+
+int* debug_visits(int kind) {
+#ifdef FA_DEBUG
+  static int* cached[64];
+  int dev = 0;
+  if (kind < 0 || kind > 2 || cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev] + kind * kDebugVisitInts;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_fa_visits) != cudaSuccess) return nullptr;
+  if (dev >= 0 && dev < 64) cached[dev] = static_cast<int*>(p);
+  return static_cast<int*>(p) + kind * kDebugVisitInts;
+#else
+  (void)kind;
+  return nullptr;
+#endif
+}
 
 uint32_t* device_status_word() {
   static uint32_t* cached[64];
@@ -231,6 +253,7 @@ const char* fa_status_string(fa_status_t s) {
     case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
     case FA_ERR_CUDA: return "FA_ERR_CUDA";
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    case FA_ERR_DEVICE_CHECK: return "FA_ERR_DEVICE_CHECK";
   }
   return "FA_ERR_UNKNOWN";
 }
@@ -673,7 +696,32 @@ fa_status_t fa_get_device_status(void* stream) {
   const uint32_t zero = 0;
   if (cudaMemcpyFromSymbol(&h, g_fa_status, sizeof(h)) != cudaSuccess) return FA_ERR_CUDA;
   if (h != 0 && cudaMemcpyToSymbol(g_fa_status, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
-  return h ? FA_ERR_TIMEOUT : FA_OK;
+  if (h & FA_DEV_TIMEOUT) return FA_ERR_TIMEOUT;
+  return h ? FA_ERR_DEVICE_CHECK : FA_OK;
+}
+
+int fa_debug_build(void) {
+#ifdef FA_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+fa_status_t fa_debug_visits(int* counts, size_t n, int clear, void* stream) {
+#ifdef FA_DEBUG
+  if (n > (size_t)(3 * kDebugVisitInts) || (n > 0 && counts == nullptr)) return FA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return FA_ERR_CUDA;
+  int* base = debug_visits(0);
+  if (base == nullptr) return FA_ERR_CUDA;
+  if (n > 0 && cudaMemcpy(counts, base, n * sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_CUDA;
+  if (clear && cudaMemset(base, 0, (size_t)(3 * kDebugVisitInts) * sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  if (clear && cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
+  return FA_OK;
+#else
+  (void)counts, (void)n, (void)clear, (void)stream;
+  return FA_ERR_UNSUPPORTED;
+#endif
 }
 
 }  // extern "C"

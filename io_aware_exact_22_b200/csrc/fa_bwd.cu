@@ -24,6 +24,7 @@
 //                   TMEM columns: S^T x2 [0,128), dP^T [128,192), dQ^T [192,256),
 //                   dV [256,384), dK [384,512).
 //   K4 fa_bwd_post  dQ = scale * accumulator, rounded to bf16.
+#include "fa_debug.cuh"
 #include "fa_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -228,6 +229,10 @@ __global__ void __launch_bounds__(448, 1)
     *abort_flag = 1;
   }
   const uint32_t tmem = 0u;
+  FA_DBG(if (!(bh < a.BH && j >= 0 && j < Tk && i0 >= 0)) {
+    if (threadIdx.x == 0) atomicOr(a.status, FA_DEV_BOUNDS);
+    *abort_flag = 1;
+  })
 
   if (warp == 13) {
     // ------------------------------------------------------------ TMA producer (whole warp)
@@ -248,6 +253,11 @@ __global__ void __launch_bounds__(448, 1)
         const int s = n % C::NSQ;
         const int i = i0 + n;
         if (!__all_sync(0xffffffffu, mbar_wait(qd_empty(s), ((n / C::NSQ) & 1) ^ 1, wc))) break;
+        FA_DBG(if (!dbg_check(i < Tq && C::BQ * i < a.N &&
+                                  ((size_t)bh * Tq + i + 1) * 128 <= (size_t)a.BH * Tq * 128, a.status)) {
+          *abort_flag = 1;
+          break;
+        })
         mbar_arrive_expect_tx_e(qd_full(s), 2 * C::QT + C::LDB);
         const uint32_t st = sb + C::ST_OFF + s * C::ST_BYTES;
         for (int b = 0; b < C::NBOX; ++b) {
@@ -374,6 +384,7 @@ __global__ void __launch_bounds__(448, 1)
                                        mbar_wait(s_full(b), (n >> 1) & 1, wc));
       if (!ok) break;
       tc_fence_after();
+      FA_DBG(if (g == 0 && wq == 0 && lane == 0) dbg_visit(a.visits, a.visits_cap, a.status, bh, Tq, i, Tk, j);)
       const uint32_t tS = tS0 + 64 * b;
       uint32_t sr[32];
       tmem_ld32(tS, sr);
@@ -462,6 +473,7 @@ __global__ void __launch_bounds__(448, 1)
       // one coalesced 128-byte request), the rest are staged as a [rows][32 d] fp32 slice in
       // shared memory and added by one TMA reduce-add.
       const int q0 = C::BQ * i;
+      FA_DBG(if (!dbg_check(q0 < a.N, a.status)) continue;)
       const int nred = min(kBwdDqRedRows, a.N - q0);
       float* dst = a.dq_acc + ((size_t)bh * a.N + q0) * C::D + wq * 32 + lane;
 #pragma unroll
@@ -609,8 +621,10 @@ static cudaError_t launch_bwd_main_t(const CUtensorMap& tq, const CUtensorMap& t
   const int Tk = (a.N + 127) / 128;
   const int Tq = (a.N + 63) / 64;
   const long long grid = (long long)a.BH * Tk;
+  BwdArgs b = a;
+  FA_DBG(b.visits = debug_visits(1); b.visits_cap = kDebugVisitInts;)
   fa_bwd_main_kernel<D, WITH_DQ><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, tdo, tdk, tdv,
-                                                                                    tdq, a, Tk, Tq);
+                                                                                    tdq, b, Tk, Tq);
   return cudaGetLastError();
 }
 

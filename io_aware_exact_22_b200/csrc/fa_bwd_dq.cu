@@ -12,6 +12,7 @@
 // registers), warp 4 issues MMAs, warp 5 issues TMA loads.
 // TMEM columns: S_b [64 b, 64 b + 64) and dP_b [128 + 64 b, + 64) for key blocks j with
 // b = j & 1 (dS_j, bf16, overwrites the first 32 columns of S_b), dQ [256, 256 + d).
+#include "fa_debug.cuh"
 #include "fa_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -106,6 +107,10 @@ __global__ void __launch_bounds__(192, 1)
     *abort_flag = 1;
   }
   const uint32_t tmem = 0u;
+  FA_DBG(if (!(bh < a.BH && it >= 0 && it < Tq128)) {
+    if (threadIdx.x == 0) atomicOr(a.status, FA_DEV_BOUNDS);
+    *abort_flag = 1;
+  })
 
   if (warp == 5) {
     // ------------------------------------------------------------ TMA producer (whole warp)
@@ -121,6 +126,10 @@ __global__ void __launch_bounds__(192, 1)
       for (; j < nblk; ++j) {
         const int s = j % C::NS;
         if (!__all_sync(0xffffffffu, mbar_wait(kv_empty(s), ((j / C::NS) & 1) ^ 1, wc))) break;
+        FA_DBG(if (!dbg_check(64 * j < a.N, a.status)) {
+          *abort_flag = 1;
+          break;
+        })
         mbar_arrive_expect_tx_e(kv_full(s), C::ST_BYTES);
         const uint32_t st = sb + C::KV_OFF + s * C::ST_BYTES;
         for (int b = 0; b < C::NBOX; ++b) {
@@ -205,6 +214,7 @@ __global__ void __launch_bounds__(192, 1)
       const int b = j & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(s_full(b), (j >> 1) & 1, wc));
       if (!ok) break;
+      FA_DBG(if (warp == 0 && lane == 0) dbg_visit(a.visits, a.visits_cap, a.status, bh, Tq128, it, Tk64, j);)
       tc_fence_after();
       uint32_t x[64], y[64];
       tmem_ld32(tmem + lane_off + C::T_S + 64 * b, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
@@ -300,7 +310,9 @@ static cudaError_t launch_dq_t(const CUtensorMap& tq, const CUtensorMap& tk, con
   const int Tq128 = (a.N + 127) / 128;
   const int Tq64 = (a.N + 63) / 64;
   const long long grid = (long long)a.BH * Tq128;
-  fa_bwd_dq_kernel<D><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, tdo, tdq, a, Tq128, Tq64);
+  BwdArgs b = a;
+  FA_DBG(b.visits = debug_visits(2); b.visits_cap = kDebugVisitInts;)
+  fa_bwd_dq_kernel<D><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, tdo, tdq, b, Tq128, Tq64);
   return cudaGetLastError();
 }
 

@@ -19,6 +19,7 @@
 // layout of an MMA A operand), so S_t is free as soon as its softmax warpgroup has loaded it
 // into registers: S_t for block j+1 is computed while the softmax of block j runs, and each
 // tile's chain per block is its softmax alone rather than S MMA + softmax + PV MMA.
+#include "fa_debug.cuh"
 #include "fa_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -150,6 +151,10 @@ __global__ void __launch_bounds__(320, 1)
     *abort_flag = 1;
   }
   const uint32_t tmem = 0u;
+  FA_DBG(if (!(bh < a.BH && qb >= 0 && qb < a.nqb && split < a.nsplit && kb1 <= Tk)) {
+    if (threadIdx.x == 0) atomicOr(a.status, FA_DEV_BOUNDS);
+    *abort_flag = 1;
+  })
 
   if (warp == 9) {
     // ------------------------------------------------------------ TMA producer (whole warp)
@@ -173,6 +178,11 @@ __global__ void __launch_bounds__(320, 1)
         const int s = it % C::NS;
         const uint32_t ph = (it / C::NS) & 1;
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(kv_empty(s), ph ^ 1, wc)))) return;
+        FA_DBG(if (!dbg_check(kb0 + j >= 0 && 128 * (kb0 + j) < a.N, a.status)) {
+          *abort_flag = 1;
+          ok = false;
+          return;
+        })
         mbar_arrive_expect_tx_e(kv_full(s), C::TILE);
         for (int b = 0; b < C::NBOX; ++b)
           tma_load_3d_e(sb + C::KV_OFF + s * C::TILE + b * 16384, m, kv_full(s), C::BOXW * b, 128 * (kb0 + j),
@@ -317,6 +327,8 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
       for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
       const int jg = kb0 + j;                 // key block index in the whole key range
+      FA_DBG(if (wq == 0 && lane == 0) dbg_visit(a.visits, a.visits_cap, a.status, bh, (a.N + 127) >> 7,
+                                                 2 * qb + t, Tk, jg);)
       const bool edge = (jg == ntile_g - 1);  // the only block that can hold the diagonal or the tail
       // P_t row r in shared memory: 16-byte chunks g of the 128-byte-swizzled K-major layout (64
       // bf16 or 128 E4M3 keys per 128-byte box row), each stored as soon as its four 32-bit
@@ -565,7 +577,9 @@ static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, co
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   const long long grid = (long long)a.BH * a.nqb * a.nsplit;
-  fa_fwd_kernel<D, PARTIAL, FP8><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, to, a);
+  FwdArgs b = a;
+  FA_DBG(b.visits = debug_visits(0); b.visits_cap = kDebugVisitInts;)
+  fa_fwd_kernel<D, PARTIAL, FP8><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, to, b);
   return cudaGetLastError();
 }
 

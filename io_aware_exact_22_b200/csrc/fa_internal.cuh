@@ -21,6 +21,9 @@ struct FwdArgs {
   const float* descale_q = nullptr;
   const float* descale_k = nullptr;
   const float* descale_v = nullptr;
+  // debug build: visit counters [BH][ceil(N/128)][ceil(N/128)] (null in the release build)
+  int* visits = nullptr;
+  long long visits_cap = 0;
 };
 
 struct BwdArgs {
@@ -39,7 +42,16 @@ struct BwdArgs {
   float* dk_acc = nullptr;
   float* dv_acc = nullptr;
   int block_major = 0;  // work order: 0 head-major, 1 key-tile-major (see fa_bwd_main_kernel)
+  // debug build: visit counters of the kernel launched with these arguments (null in release)
+  int* visits = nullptr;
+  long long visits_cap = 0;
 };
+
+// Debug build: device address of the visit-counter block of one kernel kind (0 forward,
+// 1 backward key-tile kernel, 2 deterministic dQ kernel), kDebugVisitInts counters each;
+// nullptr in the release build.
+constexpr long long kDebugVisitInts = 1LL << 20;
+int* debug_visits(int kind);
 
 // Backward dQ accumulation: of each 64-row query tile, the first kBwdDqRedRows rows are added
 // into the fp32 accumulator with per-thread reductions, the rest with one TMA reduce-add

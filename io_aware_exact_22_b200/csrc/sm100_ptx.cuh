@@ -15,6 +15,7 @@ namespace fa {
 enum : uint32_t {
   FA_DEV_TIMEOUT = 1u,    // a bounded wait ran out
   FA_DEV_TMEM_BASE = 2u,  // a full-TMEM allocation did not start at column 0
+  FA_DEV_BOUNDS = 8u,     // debug build: a device-side index check failed (the access was skipped)
 };
 
 // What a bounded wait needs: the CTA's abort flag (shared memory) and the device status word.

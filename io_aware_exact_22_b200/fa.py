@@ -21,12 +21,13 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.environ.get("FA_LIB_PATH", os.path.join(_HERE, "libfa.so"))
 
 STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_CUDA",
-          4: "FA_ERR_TIMEOUT"}
+          4: "FA_ERR_TIMEOUT", 5: "FA_ERR_DEVICE_CHECK"}
 EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_device_status",
            "fa_status_string", "fa_version", "fa_bwd_noalloc", "fa_selftest_wait_timeout",
            "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_default_splits",
            "fa_bwd_deterministic", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials",
-           "fa_bwd_prepare", "fa_bwd_accumulate", "fa_bwd_finish", "fa_bwd_main", "fa_bwd_dq_post")
+           "fa_bwd_prepare", "fa_bwd_accumulate", "fa_bwd_finish", "fa_bwd_main", "fa_bwd_dq_post",
+           "fa_debug_build", "fa_debug_visits")
 # Size of the library's built-in scratch used by fa_bwd_noalloc (include/fa.h).
 NOALLOC_MAX_SCRATCH_BYTES = 64 << 20
 
@@ -86,6 +87,10 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd_splitkv_workspace_bytes.restype = sz
         L.fa_fwd_splitkv_default_splits.argtypes = [i, i, i, i, i]
         L.fa_fwd_splitkv_default_splits.restype = i
+        L.fa_debug_build.argtypes = []
+        L.fa_debug_build.restype = i
+        L.fa_debug_visits.argtypes = [vp, sz, i, vp]
+        L.fa_debug_visits.restype = i
         L.fa_bwd_deterministic.argtypes = L.fa_bwd.argtypes
         L.fa_bwd_deterministic.restype = i
         _lib = L
@@ -217,6 +222,17 @@ def fa_status_string(code: int) -> str:
 
 def fa_version() -> int:
     return lib().fa_version()
+
+
+def fa_debug_build() -> int:
+    return lib().fa_debug_build()
+
+
+def fa_debug_visits(counts, n: int, clear: bool, stream=None) -> int:
+    """Copies the first n visit counters of the debug build into `counts` (a contiguous CPU
+    int32 tensor or numpy array), then zeroes them all when `clear`."""
+    ptr = counts.ctypes.data if hasattr(counts, "ctypes") else _ptr(counts)
+    return lib().fa_debug_visits(ptr, int(n), int(clear), _stream(stream))
 
 
 # ------------------------------------------------------------------ tensor conveniences
