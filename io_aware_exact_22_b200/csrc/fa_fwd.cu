@@ -9,11 +9,16 @@
 // special-jiahao.github.io, section 增量求解 softmax), and every exponent stays <= 2^8.
 //
 // One CTA owns 256 query rows of one (batch, head) as two 128-row tiles and streams the K/V
-// blocks through a shared-memory ring.  Roles (320 threads):
+// blocks through a shared-memory ring.  Roles (352 threads):
 //   warps 0-3  softmax warpgroup for query tile 0   (one thread per query row)
 //   warps 4-7  softmax warpgroup for query tile 1
-//   warp  8    MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j on the tensor core
+//   warp  8    score issuer (one thread): S_t = Q_t K_j^T on the tensor core
 //   warp  9    TMA producer (one thread): Q tiles once, then K_0, and K_{j+1} ahead of V_j
+//   warp  10   output issuer (one thread): O_t += P_t V_j on the tensor core
+// The two kinds of product touch disjoint TMEM columns (S against O) and shared memory (Q, K
+// against P, V), so they need no order between them, and with one issuer each a P V is issued
+// as soon as its P is written instead of after the other tile's score products: each tile's
+// chain per block (softmax, then P V) does not wait on the other tile.
 // TMEM (512 columns x 128 lanes, fp32): S_0 [0,128), S_1 [128,256), O_0 [256,256+d),
 // O_1 [256+d, 256+2d).  P_t goes to shared memory (bf16 or E4M3, the K-major 128-byte-swizzled
 // layout of an MMA A operand), so S_t is free as soon as its softmax warpgroup has loaded it
@@ -55,11 +60,12 @@ struct FwdCfg {
   static constexpr int KV_OFF = 2 * TILE;
   static constexpr int P_OFF = KV_OFF + NS * TILE;  // ring and P tiles together stage partial outputs
   static constexpr int BAR_OFF = P_OFF + 2 * PTILE;
-  // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], s_free[2], p_full[2], pv_done[2], o_full
-  static constexpr int NBAR = 1 + 2 * NS + 8 + 1;
+  // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], s_free[2], p_full[2], pv_done[2], o_full,
+  // s_done
+  static constexpr int NBAR = 1 + 2 * NS + 8 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM = MISC_OFF + 16 + 1024;  // + slack to align the base to 1024
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 352;
   static constexpr uint32_t TMEM_COLS = 512;
   // TMEM columns (a 512-column allocation always starts at column 0, lane 0)
   static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_O0 = 256, T_O1 = 256 + D;
@@ -75,7 +81,7 @@ struct FwdCfg {
 // PARTIAL: the CTA covers only its split's range of key blocks and writes the normalised
 // partial output O_s (fp32) and its LSE_s, to be combined by fa_fwd_merge_kernel.
 template <int D, bool PARTIAL, bool FP8 = false>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const FwdArgs a) {
@@ -118,6 +124,7 @@ __global__ void __launch_bounds__(320, 1)
   auto p_full = [&](int t) { return bar + 8u * (5 + 2 * C::NS + t); };   // P_t written
   auto pv_done = [&](int t) { return bar + 8u * (7 + 2 * C::NS + t); };  // P_t V_j added into O_t
   const uint32_t o_full = bar + 8u * (9 + 2 * C::NS);
+  const uint32_t s_done = bar + 8u * (10 + 2 * C::NS);  // every score product issued has completed
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gb + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + C::MISC_OFF + 4);
   const WaitCtx wc{abort_flag, a.status};
@@ -135,6 +142,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(pv_done(t), 1);
     }
     mbar_init(o_full, 1);
+    mbar_init(s_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -203,36 +211,15 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 8) {
-    // ------------------------------------------------------------ MMA issuer (whole warp)
+  } else if (warp == 8 || warp == 10) {
+    // ------------------------------------------------------------ MMA issuers (whole warps)
     if (!*abort_flag && nmax > 0) {
       const int nt[2] = {n0, n1};
       // Base descriptors; each MMA adds its byte offset (see sdesc_add).
       const uint64_t dQ_k = sdesc_sw128(sb + C::Q_OFF, 16, 1024);       // Q tiles, K-major
       const uint64_t dK_k = sdesc_sw128(sb + C::KV_OFF, 16, 1024);      // K stages, K-major
       const uint64_t dV_mn = sdesc_sw128(sb + C::KV_OFF, 16384, 1024);  // V stages, MN-major
-      auto issue_qk = [&](uint32_t dst, uint32_t qoff, uint32_t koff) {
-#pragma unroll
-        for (int k = 0; k < D / C::KSTEP; ++k) {  // 32 bytes of d per MMA
-          const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-          if constexpr (FP8)
-            mma_ss_e8(dst, sdesc_add(dQ_k, qoff + off), sdesc_add(dK_k, koff + off), C::IDESC_QK, k > 0);
-          else
-            mma_ss_e(dst, sdesc_add(dQ_k, qoff + off), sdesc_add(dK_k, koff + off), C::IDESC_QK, k > 0);
-        }
-      };
       const uint64_t dP_k = sdesc_sw128(sb + C::P_OFF, 16, 1024);       // P tiles, K-major
-      auto issue_pv = [&](uint32_t dst, uint32_t poff, uint32_t voff, bool acc) {
-#pragma unroll
-        for (int k = 0; k < 128 / C::KSTEP; ++k) {  // KSTEP keys (32 bytes of P) per MMA
-          const uint32_t po = poff + (k >> 2) * 16384 + (k & 3) * 32;
-          const uint32_t vo = voff + k * C::KSTEP * 128;
-          if constexpr (FP8)
-            mma_ss_e8(dst, sdesc_add(dP_k, po), sdesc_add(dV_mn, vo), C::IDESC_PV, (acc || k > 0) ? 1u : 0u);
-          else
-            mma_ss_e(dst, sdesc_add(dP_k, po), sdesc_add(dV_mn, vo), C::IDESC_PV, (acc || k > 0) ? 1u : 0u);
-        }
-      };
       // ring positions: K_0 first, then K_{j+1} (when there is one) before V_j
       auto pos_k = [&](int j) { return j == 0 ? 0 : 2 * j - 1; };
       auto pos_v = [&](int j) { return j + 1 < nmax ? 2 * j + 2 : 2 * j + 1; };
@@ -241,27 +228,28 @@ __global__ void __launch_bounds__(320, 1)
       auto wait_stage = [&](int it) {
         return __all_sync(0xffffffffu, mbar_wait(kv_full(it % C::NS), stage_par(it), wc));
       };
-      bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, wc));
-      if (ok) ok = wait_stage(0);
-      if (ok) {
-        tc_fence_after();
-        for (int t = 0; t < 2; ++t) {
-          if (nt[t] == 0) continue;
-          issue_qk(t ? C::T_S1 : C::T_S0, (uint32_t)(t * C::TILE), stage_addr(0));
-          mma_commit_e(s_full(t));
-        }
-        mma_commit_e(kv_empty(0));
-      }
-      for (int j = 0; j < nmax && ok; ++j) {
-        // S_t for block j+1, each as soon as tile t's softmax has loaded S_t for block j
-        if (j + 1 < nmax) {
-          const int itK = pos_k(j + 1);
+      bool ok = true;
+      if (warp == 8) {
+        // S_t for block j, each as soon as K_j has landed and tile t's softmax has loaded S_t of
+        // block j-1
+        auto issue_qk = [&](uint32_t dst, uint32_t qoff, uint32_t koff) {
+#pragma unroll
+          for (int k = 0; k < D / C::KSTEP; ++k) {  // 32 bytes of d per MMA
+            const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+            if constexpr (FP8)
+              mma_ss_e8(dst, sdesc_add(dQ_k, qoff + off), sdesc_add(dK_k, koff + off), C::IDESC_QK, k > 0);
+            else
+              mma_ss_e(dst, sdesc_add(dQ_k, qoff + off), sdesc_add(dK_k, koff + off), C::IDESC_QK, k > 0);
+          }
+        };
+        ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, wc));
+        for (int j = 0; j < nmax && ok; ++j) {
+          const int itK = pos_k(j);
           if (!(ok = wait_stage(itK))) break;
-          tc_fence_after();
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
-            if (j + 1 >= nt[t]) continue;
-            if (!(ok = __all_sync(0xffffffffu, mbar_wait(s_free(t), j & 1, wc)))) break;
+            if (j >= nt[t]) continue;
+            if (j > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(s_free(t), (j - 1) & 1, wc)))) break;
             tc_fence_after();
             issue_qk(t ? C::T_S1 : C::T_S0, (uint32_t)(t * C::TILE), stage_addr(itK));
             mma_commit_e(s_full(t));
@@ -269,23 +257,38 @@ __global__ void __launch_bounds__(320, 1)
           if (!ok) break;
           mma_commit_e(kv_empty(itK % C::NS));
         }
-        // O_t += P_t V_j, each as soon as tile t's softmax has written P_t
-        const int itV = pos_v(j);
-        if (!(ok = wait_stage(itV))) break;
-        tc_fence_after();
+        mma_commit_e(s_done);
+        if (!ok) mbar_wait_drain(s_done, 0);  // every issued MMA has completed before TMEM is freed
+      } else {
+        // O_t += P_t V_j, each as soon as V_j has landed and tile t's softmax has written P_t
+        auto issue_pv = [&](uint32_t dst, uint32_t poff, uint32_t voff, bool acc) {
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (j >= nt[t]) continue;
-          if (!(ok = __all_sync(0xffffffffu, mbar_wait(p_full(t), j & 1, wc)))) break;
-          tc_fence_after();
-          issue_pv(t ? C::T_O1 : C::T_O0, (uint32_t)(t * C::PTILE), stage_addr(itV), j > 0);
-          mma_commit_e(pv_done(t));
+          for (int k = 0; k < 128 / C::KSTEP; ++k) {  // KSTEP keys (32 bytes of P) per MMA
+            const uint32_t po = poff + (k >> 2) * 16384 + (k & 3) * 32;
+            const uint32_t vo = voff + k * C::KSTEP * 128;
+            if constexpr (FP8)
+              mma_ss_e8(dst, sdesc_add(dP_k, po), sdesc_add(dV_mn, vo), C::IDESC_PV, (acc || k > 0) ? 1u : 0u);
+            else
+              mma_ss_e(dst, sdesc_add(dP_k, po), sdesc_add(dV_mn, vo), C::IDESC_PV, (acc || k > 0) ? 1u : 0u);
+          }
+        };
+        for (int j = 0; j < nmax && ok; ++j) {
+          const int itV = pos_v(j);
+          if (!(ok = wait_stage(itV))) break;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (j >= nt[t]) continue;
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(p_full(t), j & 1, wc)))) break;
+            tc_fence_after();
+            issue_pv(t ? C::T_O1 : C::T_O0, (uint32_t)(t * C::PTILE), stage_addr(itV), j > 0);
+            mma_commit_e(pv_done(t));
+          }
+          if (!ok) break;
+          mma_commit_e(kv_empty(itV % C::NS));
         }
-        if (!ok) break;
-        mma_commit_e(kv_empty(itV % C::NS));
+        mma_commit_e(o_full);
+        if (!ok) mbar_wait_drain(o_full, 0);  // every issued MMA has completed before TMEM is freed
       }
-      mma_commit_e(o_full);
-      if (!ok) mbar_wait_drain(o_full, 0);  // every issued MMA has completed before TMEM is freed
     }
     __syncwarp();
   } else {
