@@ -124,12 +124,12 @@ struct BwdCfg {
   static constexpr int DQS_WARP = (BQ - kBwdDqRedRows) * 32 * 4;
   static constexpr int LD_OFF = DQS_OFF + 4 * DQS_WARP;
   static constexpr int BAR_OFF = LD_OFF + NSQ * LDB;
-  // kv_full, qd_full[3], qd_empty[3], s_full[2], dp_full, p_ready, ds_ready, dq_full,
-  // dq_free, ds_free[2], kv_done
-  static constexpr int NBAR = 1 + 2 * NSQ + 10;
+  // kv_full, qd_full[3], qd_empty[3], s_full[2], dp_full, p_ready[2], ds_ready[2], dq_full,
+  // dq_free, ds_free[2], kv_done, dv_done[2], sc_done
+  static constexpr int NBAR = 1 + 2 * NSQ + 15;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM = MISC_OFF + 16 + 1024;
-  static constexpr int THREADS = 448;
+  static constexpr int THREADS = 480;
   static constexpr uint32_t TMEM_COLS = 512;
   // TMEM columns (a 512-column allocation always starts at column 0, lane 0)
   // S^T is double-buffered: [0,64) for even query tiles, [64,128) for odd ones
@@ -139,12 +139,17 @@ struct BwdCfg {
   static constexpr uint32_t IDESC_Q = idesc_bf16(128, BQ, true, true);     // dQ^T
 };
 
-// Roles (448 threads):
+// Roles (480 threads):
 //   warps 0-3   compute warpgroup 0: P^T and dS^T for query columns [0, 32)  (one key row each)
 //   warps 4-7   compute warpgroup 1: the same for query columns [32, 64)
 //   warps 8-11  dQ^T drain: TMEM -> shared staging -> TMA reduce-add into the fp32 accumulator
-//   warp 12     MMA issuer (whole warp, one elected lane issues)
+//   warp 12     score issuer: S^T and dP^T (whole warp, one elected lane issues)
 //   warp 13     TMA producer (whole warp, one elected lane issues)
+//   warp 14     gradient issuer: dV, dK and dQ^T
+// Two issuers, so that neither kind of product waits behind the other's barriers and commits.
+// Their products share no accumulator; the one overwrite that crosses them (S^T of tile n+2
+// into the TMEM buffer whose P^T dV_n reads) waits for dv_done, which the gradient issuer
+// commits after dV_n, and a Q/dO stage is released when both have committed their last use.
 // Each compute warpgroup writes its packed P^T inside its own S^T columns, so neither
 // overwrites scores the other has not read yet: P^T of query columns [32g, 32g+32) sits at
 // TMEM columns [32g, 32g+16) of the tile's S^T buffer.  dS^T goes to shared memory only,
@@ -157,7 +162,7 @@ struct BwdCfg {
 // WITH_DQ = false: dK and dV only (dQ comes from fa_bwd_dq_kernel): no dQ^T MMA, no drain.  The dQ^T MMA puts d on the M dimension (128 TMEM lanes), so the
 // atomic dQ path exists for D = 128 only; D = 64 always runs with WITH_DQ = false.
 template <int D, bool WITH_DQ>
-__global__ void __launch_bounds__(448, 1)
+__global__ void __launch_bounds__(480, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                        const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
@@ -184,15 +189,24 @@ __global__ void __launch_bounds__(448, 1)
   const uint32_t kv_full = bar;
   auto qd_full = [&](int s) { return bar + 8u * (1 + s); };
   auto qd_empty = [&](int s) { return bar + 8u * (1 + C::NSQ + s); };
+  // barrier block after the ring's: s_full[2] 0, 8 | dp_full 16 | p_ready[2] 24, 32 | dq_full 40 |
+  // dq_free 48 | ds_free[2] 56, 64 | kv_done 72 | dv_done[2] 80, 88 | sc_done 96 | ds_ready[2]
+  // 104, 112: fifteen 8-byte barriers
+  static_assert(C::NBAR == 1 + 2 * C::NSQ + 15, "barrier block layout");
   const uint32_t bar2 = bar + 8u * (1 + 2 * C::NSQ);
   auto s_full = [&](int b) { return bar2 + 8u * b; };
   const uint32_t dp_full = bar2 + 16;
-  const uint32_t p_ready = bar2 + 24;
-  const uint32_t ds_ready = bar2 + 32;
+  // P_n and dS_n ready, one barrier per S^T / dS^T buffer (b = n & 1): a tile's arrival on a
+  // buffer needs the previous tile of that buffer consumed by both issuers, so no waiter ever
+  // falls two phases behind
+  auto p_ready = [&](int b) { return bar2 + 24 + 8u * b; };
+  auto ds_ready = [&](int b) { return bar2 + 104 + 8u * b; };
   const uint32_t dq_full = bar2 + 40;
   const uint32_t dq_free = bar2 + 48;
   auto ds_free = [&](int b) { return bar2 + 56 + 8u * b; };
   const uint32_t kv_done = bar2 + 72;
+  auto dv_done = [&](int b) { return bar2 + 80 + 8u * b; };  // dV_n (n & 1 == b) has completed
+  const uint32_t sc_done = bar2 + 96;                        // every score product has completed
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gb + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + C::MISC_OFF + 4);
   const WaitCtx wc{abort_flag, a.status};
@@ -201,18 +215,22 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(kv_full, 1);
     for (int s = 0; s < C::NSQ; ++s) {
       mbar_init(qd_full(s), 1);
-      mbar_init(qd_empty(s), 1);
+      mbar_init(qd_empty(s), 2);  // released by both issuers
     }
     mbar_init(dp_full, 1);
-    mbar_init(p_ready, 256);
-    mbar_init(ds_ready, 256);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(p_ready(b), 256);
+      mbar_init(ds_ready(b), 256);
+    }
     mbar_init(dq_full, 1);
     mbar_init(dq_free, 128);
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full(b), 1);
       mbar_init(ds_free(b), 1);
+      mbar_init(dv_done(b), 1);
     }
     mbar_init(kv_done, 1);
+    mbar_init(sc_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -273,14 +291,16 @@ __global__ void __launch_bounds__(448, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 12) {
-    // ------------------------------------------------------------ MMA issuer (whole warp)
-    // Issue order:  S_0, S_1, dP_0 | [P_n ready] dV_n, [dS_n ready] dP_{n+1}, dK_n, dQ_n, S_{n+2} | ...
-    // Every overwrite follows the last reader in issue order (tcgen05 MMAs issued by one
-    // thread execute in order): S_{n+2} follows dV_n, which reads P_n from the same buffer;
-    // dP_{n+1} follows the compute warps' read of dP_n (signalled by ds_ready).  S_{n+2} comes
-    // last because its Q tile is the most recently requested load; it is needed only after
-    // the compute warps have finished tile n+1.
+  } else if (warp == 12 || warp == 14) {
+    // ------------------------------------------------------------ MMA issuers (whole warps)
+    // Score issuer:    S_0, S_1, dP_0 | [dS_n ready] dP_(n+1), [dV_n done] S_(n+2) | ...
+    // Gradient issuer: [P_n ready] dV_n | [dS_n ready] dK_n, [drain done] dQ_n | ...
+    // Every overwrite follows its last reader: dP_(n+1) follows the compute warps' read of dP_n
+    // (ds_ready), S_(n+2) follows dV_n (dv_done), which reads P_n from the same TMEM buffer;
+    // dQ_n follows the drain's read of dQ_(n-1) (dq_free); the dS^T buffer is released after
+    // dK_n and dQ_n (ds_free), a Q/dO stage after S_n, dP_n (score issuer) and dV_n, dK_n
+    // (gradient issuer).  The gradient issuer's last commit (kv_done) also covers every score
+    // product: each one was consumed by the compute warps before the last dV or dK could start.
     if (!*abort_flag) {
       bool ok = __all_sync(0xffffffffu, mbar_wait(kv_full, 0, wc));
       // Base descriptors; each MMA adds its byte offset (see sdesc_add).
@@ -294,74 +314,88 @@ __global__ void __launch_bounds__(448, 1)
       const uint64_t dS_k = sdesc_sw128(sb + C::DS_OFF, 16, 1024);       // dS^T, K-major (dK)
       const uint64_t dS_mn = sdesc_sw128(sb + C::DS_OFF, 8192, 1024);    // dS^T, MN-major (dQ^T)
       auto st_off = [&](int n) { return (uint32_t)((n % C::NSQ) * C::ST_BYTES); };
-      auto issue_s = [&](int n) {  // S^T = K_j Q_i^T  (K over d), into buffer n & 1
-        const uint32_t so = st_off(n);
+      if (warp == 12) {
+        auto issue_s = [&](int n) {  // S^T = K_j Q_i^T  (K over d), into buffer n & 1
+          const uint32_t so = st_off(n);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32, qo = (k >> 2) * 8192 + (k & 3) * 32;
-          mma_ss_e(tmem + C::T_S + 64 * (n & 1), sdesc_add(dK_k, ko), sdesc_add(dQ_k, so + qo), C::IDESC_S, k > 0);
-        }
-        mma_commit_e(s_full(n & 1));
-      };
-      auto issue_dp = [&](int n) {  // dP^T = V_j dO_i^T
-        const uint32_t so = st_off(n);
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32, qo = (k >> 2) * 8192 + (k & 3) * 32;
-          mma_ss_e(tmem + C::T_DP, sdesc_add(dV_k, ko), sdesc_add(dO_k, so + qo), C::IDESC_S, k > 0);
-        }
-        mma_commit_e(dp_full);
-      };
-      auto wait_q = [&](int n) {
-        return __all_sync(0xffffffffu, mbar_wait(qd_full(n % C::NSQ), (n / C::NSQ) & 1, wc));
-      };
-      if (ok && count > 0) {
-        if ((ok = wait_q(0))) {
-          tc_fence_after();
-          issue_s(0);
-          if (count > 1 && (ok = wait_q(1))) {
-            tc_fence_after();
-            issue_s(1);
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32, qo = (k >> 2) * 8192 + (k & 3) * 32;
+            mma_ss_e(tmem + C::T_S + 64 * (n & 1), sdesc_add(dK_k, ko), sdesc_add(dQ_k, so + qo), C::IDESC_S, k > 0);
           }
-          if (ok) issue_dp(0);
+          mma_commit_e(s_full(n & 1));
+        };
+        auto issue_dp = [&](int n) {  // dP^T = V_j dO_i^T; the last score product of tile n
+          const uint32_t so = st_off(n);
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32, qo = (k >> 2) * 8192 + (k & 3) * 32;
+            mma_ss_e(tmem + C::T_DP, sdesc_add(dV_k, ko), sdesc_add(dO_k, so + qo), C::IDESC_S, k > 0);
+          }
+          mma_commit_e(dp_full);
+          mma_commit_e(qd_empty(n % C::NSQ));
+        };
+        auto wait_q = [&](int n) {
+          return __all_sync(0xffffffffu, mbar_wait(qd_full(n % C::NSQ), (n / C::NSQ) & 1, wc));
+        };
+        if (ok && count > 0) {
+          if ((ok = wait_q(0))) {
+            tc_fence_after();
+            issue_s(0);
+            if (count > 1 && (ok = wait_q(1))) {
+              tc_fence_after();
+              issue_s(1);
+            }
+            if (ok) issue_dp(0);
+          }
         }
-      }
-      for (int n = 0; n < count && ok; ++n) {
-        const int s = n % C::NSQ;
-        const int b = n & 1;
-        const uint32_t so = st_off(n);
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(p_ready, n & 1, wc)))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < 4; ++k)  // dV += P^T dO_i  (K over the 64 queries; A = P^T from TMEM)
-          mma_ts_e(tmem + C::T_DV, tmem + C::T_S + 64 * b + 32 * (k >> 1) + 8 * (k & 1),
-                   sdesc_add(dO_mn, so + k * 2048), C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(ds_ready, n & 1, wc)))) break;
-        tc_fence_after();
-        if (n + 1 < count) issue_dp(n + 1);  // Q/dO_{n+1} landed before S_{n+1} was issued
-#pragma unroll
-        for (int k = 0; k < 4; ++k)  // dK += dS^T Q_i  (K over the 64 queries; A = dS^T in smem)
-          mma_ss_e(tmem + C::T_DK, sdesc_add(dS_k, b * C::DS_BYTES + 32 * k), sdesc_add(dQ_mn, so + k * 2048),
-                   C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
-        if (WITH_DQ) {
-          if (!(ok = __all_sync(0xffffffffu, mbar_wait(dq_free, (n & 1) ^ 1, wc)))) break;
+        for (int n = 0; n < count && ok; ++n) {
+          if (n + 1 < count) {  // dO_(n+1) landed before S_(n+1) was issued
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(ds_ready(n & 1), (n >> 1) & 1, wc)))) break;
+            tc_fence_after();
+            issue_dp(n + 1);
+          }
+          if (n + 2 < count) {
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(dv_done(n & 1), (n >> 1) & 1, wc)))) break;
+            if (!(ok = wait_q(n + 2))) break;
+            tc_fence_after();
+            issue_s(n + 2);
+          }
+        }
+        mma_commit_e(sc_done);
+        if (!ok) mbar_wait_drain(sc_done, 0);
+      } else {
+        for (int n = 0; n < count && ok; ++n) {
+          const int s = n % C::NSQ;
+          const int b = n & 1;
+          const uint32_t so = st_off(n);
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(p_ready(b), (n >> 1) & 1, wc)))) break;
           tc_fence_after();
 #pragma unroll
-          for (int k = 0; k < 8; ++k)  // dQ_i^T = K_j^T dS^T  (K over the 128 keys)
-            mma_ss_e(tmem + C::T_DQ, sdesc_add(dK_mn, k * 2048), sdesc_add(dS_mn, b * C::DS_BYTES + k * 2048),
-                     C::IDESC_Q, k > 0);
-          mma_commit_e(dq_full);
-        }
-        mma_commit_e(ds_free(b));
-        mma_commit_e(qd_empty(s));
-        if (n + 2 < count) {
-          if (!(ok = wait_q(n + 2))) break;
+          for (int k = 0; k < 4; ++k)  // dV += P^T dO_i  (K over the 64 queries; A = P^T from TMEM)
+            mma_ts_e(tmem + C::T_DV, tmem + C::T_S + 64 * b + 32 * (k >> 1) + 8 * (k & 1),
+                     sdesc_add(dO_mn, so + k * 2048), C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
+          mma_commit_e(dv_done(b));
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(ds_ready(b), (n >> 1) & 1, wc)))) break;
           tc_fence_after();
-          issue_s(n + 2);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)  // dK += dS^T Q_i  (K over the 64 queries; A = dS^T in smem)
+            mma_ss_e(tmem + C::T_DK, sdesc_add(dS_k, b * C::DS_BYTES + 32 * k), sdesc_add(dQ_mn, so + k * 2048),
+                     C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
+          if (WITH_DQ) {
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(dq_free, (n & 1) ^ 1, wc)))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < 8; ++k)  // dQ_i^T = K_j^T dS^T  (K over the 128 keys)
+              mma_ss_e(tmem + C::T_DQ, sdesc_add(dK_mn, k * 2048), sdesc_add(dS_mn, b * C::DS_BYTES + k * 2048),
+                       C::IDESC_Q, k > 0);
+            mma_commit_e(dq_full);
+          }
+          mma_commit_e(ds_free(b));
+          mma_commit_e(qd_empty(s));
         }
+        mma_commit_e(kv_done);
+        if (!ok) mbar_wait_drain(kv_done, 0);
       }
-      mma_commit_e(kv_done);
-      if (!ok) mbar_wait_drain(kv_done, 0);
     }
     __syncwarp();
   } else if (warp < 8) {
@@ -416,7 +450,7 @@ __global__ void __launch_bounds__(448, 1)
       tmem_st16(tS, pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_ready);
+      mbar_arrive(p_ready(b));
 
       ok = __all_sync(0xffffffffu, mbar_wait(dp_full, n & 1, wc));
       if (!ok) break;
@@ -447,7 +481,7 @@ __global__ void __launch_bounds__(448, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();  // the tcgen05.ld of dP^T is complete before dP_{n+1} may overwrite it
-      mbar_arrive(ds_ready);
+      mbar_arrive(ds_ready(b));
     }
   } else {
     // ------------------------------------------------------------ dQ^T drain (one d index each)
