@@ -97,13 +97,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   if (mbar_try_wait(bar, parity)) return true;
   return mbar_wait_slow(bar, parity, w.abort_flag, w.status);
 }
-// The same wait with the slow path inlined, for kernels that rebalance registers with
-// setmaxnreg: code under a raised register budget cannot call out of line.
-__device__ __forceinline__ bool mbar_wait_inl(uint32_t bar, uint32_t parity, const WaitCtx& w) {
-  if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_loop(bar, parity, w.abort_flag, w.status);
-}
-
 // Wait used only on the abort path, to let copies already in flight land before exit.
 __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = globaltimer();
