@@ -107,15 +107,20 @@ fa_status_t check_shape(int B, int H, int N, int d, float scale, int causal, boo
 
 // Per-query-tile statistics of the backward: [BH][ceil(N/64)][128] fp32, rounded to 256 bytes.
 // Work order of the attention grids.  Under the causal mask a head's query blocks (forward) or
-// key tiles (backward) differ in length; launching every head's heaviest block first gives the
-// shortest tail, but spreads the blocks in flight over all heads, whose streamed operand pair
-// (K, V in the forward; Q, dO in the backward) must then stay in L2 together.  Measured on
-// B200 (126 MB L2): block-major gains up to 21 % (forward) and 8 % (backward) when that pair
-// spans at most ~67 MB for all heads, and loses 5-13 % at 134 MB and beyond.
-int block_major_order(long long BH, int N, int d, int elem_bytes, int causal) {
-  if (!causal) return 0;
-  const double pair_bytes = 2.0 * (double)BH * N * d * elem_bytes;
-  return pair_bytes <= 80.0 * 1024 * 1024 ? 1 : 0;
+// key tiles (backward) differ in length, so launching the heaviest first shortens the tail; but
+// the blocks in flight then spread over every head so ordered, whose streamed operand pair (K, V
+// in the forward; Q, dO in the backward) must stay in L2 together.  Heads therefore go in groups:
+// inside a group every head's heaviest block goes first, and the group is as many heads as have
+// their pairs within kWorkGroupBytes (L2 is 126 MB).  Measured on B200 (step time of forward +
+// backward): at B=1 H=32 N=16384 d=128, groups of 4 heads (32 MB) are 2.6 % faster than one head
+// (forward 4.8 %, backward key-tile kernel 1.7 %), groups of 8 and 16 lose part or all of it to
+// L2 misses; at B=2 H=16 N=4096, groups of 16 beat 4 and all 32 heads by 3.5 % and 1.3 %.
+constexpr double kWorkGroupBytes = 32.0 * 1024 * 1024;
+int work_group(long long BH, int N, int d, int elem_bytes, int causal) {
+  if (!causal) return 1;  // blocks of equal length: a head's blocks together
+  const double head_pair = 2.0 * (double)N * d * elem_bytes;
+  const long long g = (long long)(kWorkGroupBytes / head_pair);
+  return (int)std::max(1LL, std::min(BH, g));
 }
 
 size_t ld_bytes(long long bh, int N) {
@@ -283,7 +288,7 @@ fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* 
   a.causal = causal;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   a.nsplit = 1;
-  a.block_major = block_major_order(BH, N, d, 2, causal);
+  a.group = work_group(BH, N, d, 2, causal);
   if ((long long)a.BH * a.nqb > INT_MAX) return FA_ERR_INVALID_ARG;
   return launch_fwd(d, tq, tk, tv, to, a, (cudaStream_t)stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -314,7 +319,7 @@ fa_status_t fa_fwd_fp8(const void* q, const void* k, const void* v, const float*
   a.causal = causal;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   a.nsplit = 1;
-  a.block_major = block_major_order(BH, N, d, 1, causal);
+  a.group = work_group(BH, N, d, 1, causal);
   a.descale_q = descale_q;
   a.descale_k = descale_k;
   a.descale_v = descale_v;
@@ -420,7 +425,7 @@ fa_status_t fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o,
   a.causal = causal;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   a.nsplit = sp;
-  a.block_major = block_major_order(BH, N, d, 2, causal);
+  a.group = work_group(BH, N, d, 2, causal);
   cudaStream_t s = (cudaStream_t)stream;
   if (launch_fwd(d, tq, tk, tv, to, a, s) != cudaSuccess) return FA_ERR_CUDA;
   if (launch_fwd_merge(o_part, lse_part, o, lse, sp, rows, d, s) != cudaSuccess) return FA_ERR_CUDA;
@@ -451,7 +456,7 @@ fa_status_t fa_fwd_partial(const void* q, const void* k, const void* v, float* o
   a.causal = causal;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   a.nsplit = 1;
-  a.block_major = block_major_order(BH, N, d, 2, causal);
+  a.group = work_group(BH, N, d, 2, causal);
   return launch_fwd_partial(d, tq, tk, tv, to, a, (cudaStream_t)stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -511,7 +516,7 @@ static fa_status_t bwd_main_d128(const void* q, const void* k, const void* v, co
   a.causal = causal;
   a.scale = scale;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
-  a.block_major = block_major_order(BH, N, d, 2, causal);
+  a.group = work_group(BH, N, d, 2, causal);
   cudaError_t e = launch_bwd_main(d, tq, tk, tv, tdo, tdk, tdv, tdq, a, s);
   if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -674,7 +679,7 @@ fa_status_t fa_bwd_deterministic(const void* q, const void* k, const void* v, co
   a.causal = causal;
   a.scale = scale;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
-  a.block_major = block_major_order(BH, N, d, 2, causal);
+  a.group = work_group(BH, N, d, 2, causal);
   if (launch_bwd_pre(o, dO, lse, ld, nullptr, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
   if (launch_bwd_main(d, tq64, tk128, tv128, tdo64, tdk, tdv, tdk, a, s, false) != cudaSuccess) return FA_ERR_CUDA;
   if (launch_bwd_dq(d, tq128, tk64, tv64, tdo128, tdq, a, s) != cudaSuccess) return FA_ERR_CUDA;

@@ -178,10 +178,15 @@ __global__ void __launch_bounds__(480, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // head-major (a head's key tiles together, heaviest first) or tile-major (every head's
-  // heaviest key tile first); see fa_fwd_kernel for the trade-off
-  const int bh = a.block_major ? (int)(blockIdx.x % a.BH) : (int)(blockIdx.x / Tk);
-  const int j = a.block_major ? (int)(blockIdx.x / a.BH) : (int)(blockIdx.x % Tk);  // keys [128 j, +128)
+  // heads in groups of a.group, every head's heaviest key tile first within a group (see
+  // fa_fwd_kernel for the trade-off)
+  const int item = (int)blockIdx.x;
+  const int per_group = a.group * Tk;
+  const int g0 = item / per_group * a.group;
+  const int gn = min(a.group, a.BH - g0);
+  const int r = item - item / per_group * per_group;
+  const int bh = g0 + r % gn;
+  const int j = r / gn;  // keys [128 j, +128)
   const int i0 = a.causal ? 2 * j : 0;         // first query tile with a visible pair
   const int count = max(0, Tq - i0);
 

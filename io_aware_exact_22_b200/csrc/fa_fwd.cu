@@ -94,13 +94,17 @@ __global__ void __launch_bounds__(352, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: (head bh, block of 256 query rows, key split); heavier causal blocks first
+  // ---- work item: (head bh, block of 256 query rows, key split).  Heads go in groups of
+  // a.group, and within a group every head's heaviest query block goes first: group 1 keeps a
+  // head's blocks together (its K/V stays in L2), group BH gives the shortest causal tail.
   const int split = blockIdx.x % a.nsplit;
   const int item = blockIdx.x / a.nsplit;
-  // head-major (a head's query blocks together, heaviest first: its K/V stays in L2) or
-  // block-major (every head's heaviest block first: the shortest tail under the causal mask)
-  const int bh = a.block_major ? item % a.BH : item / a.nqb;
-  const int qb = a.nqb - 1 - (a.block_major ? item / a.BH : item % a.nqb);
+  const int per_group = a.group * a.nqb;
+  const int g0 = item / per_group * a.group;  // first head of the group
+  const int gn = min(a.group, a.BH - g0);     // heads in the group (the last may be short)
+  const int r = item - item / per_group * per_group;
+  const int bh = g0 + r % gn;
+  const int qb = a.nqb - 1 - r / gn;
   const int q0 = qb * 256;
   const int Tk = (a.N + 127) >> 7;
   const bool has1 = (q0 + 128) < a.N;

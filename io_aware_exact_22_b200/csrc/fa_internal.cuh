@@ -16,7 +16,7 @@ struct FwdArgs {
   int causal;        // 0 / 1
   float scale_log2;  // scale * log2(e)
   int nsplit;        // key-range splits per (head, query block); 1 = whole key range
-  int block_major = 0;  // work order: 0 head-major, 1 query-block-major (see fa_fwd_kernel)
+  int group = 1;      // work order: heads per group, heaviest query block first within a group
   // FP8 forward only: per-(b,h) dequantisation factors [BH], or null for 1
   const float* descale_q = nullptr;
   const float* descale_k = nullptr;
@@ -41,7 +41,7 @@ struct BwdArgs {
   // fp32 [BH, N, d] accumulators instead of being stored as bf16 (the sequence-sharded backward)
   float* dk_acc = nullptr;
   float* dv_acc = nullptr;
-  int block_major = 0;  // work order: 0 head-major, 1 key-tile-major (see fa_bwd_main_kernel)
+  int group = 1;  // work order: heads per group, heaviest key tile first within a group
   // debug build: visit counters of the kernel launched with these arguments (null in release)
   int* visits = nullptr;
   long long visits_cap = 0;

@@ -61,12 +61,16 @@ def main():
     total = 0
     for d in (64, 128):
         for causal in (False, True):
-            for N in (1, 129, 1000, 4096):
-                B, H = 1, 2
+            # ragged lengths on two heads; and (d = 128, causal) ten heads long enough that the
+            # work order puts them in groups of fewer heads, the last group short
+            shapes = [(1, 2, N) for N in (1, 129, 1000, 4096)]
+            if d == 128 and causal:
+                shapes.append((1, 10, 16384))
+            for B, H, N in shapes:
                 BH = B * H
                 w = custom(B, H, N, d, causal, seed=N + d, backward=True)
                 q, k, v, do = (t.cuda() for t in make_inputs(w))
-                tag = f"d={d} causal={int(causal)} N={N}"
+                tag = f"d={d} causal={int(causal)} BH={BH} N={N}"
                 o, lse = fa.forward(q, k, v, causal, w.scale)
                 status_ok("fwd " + tag)
                 total += check("fwd " + tag, 0, BH, N, 128, 128, causal)
