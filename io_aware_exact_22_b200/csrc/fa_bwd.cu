@@ -124,16 +124,18 @@ struct BwdCfg {
   static constexpr int DQS_WARP = (BQ - kBwdDqRedRows) * 32 * 4;
   static constexpr int LD_OFF = DQS_OFF + 4 * DQS_WARP;
   static constexpr int BAR_OFF = LD_OFF + NSQ * LDB;
-  // kv_full, qd_full[3], qd_empty[3], s_full[2], dp_full, p_ready[2], ds_ready[2], dq_full,
-  // dq_free, ds_free[2], kv_done, dv_done[2], sc_done
-  static constexpr int NBAR = 1 + 2 * NSQ + 15;
+  // kv_full, qd_full[3], qd_empty[3], s_full[2], dp_full[2], p_ready[2], ds_ready[2],
+  // dq_full[2], dq_free[2], ds_free[2], kv_done, dv_done[2], sc_done
+  static constexpr int NBAR = 1 + 2 * NSQ + 18;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM = MISC_OFF + 16 + 1024;
   static constexpr int THREADS = 480;
   static constexpr uint32_t TMEM_COLS = 512;
   // TMEM columns (a 512-column allocation always starts at column 0, lane 0)
-  // S^T is double-buffered: [0,64) for even query tiles, [64,128) for odd ones
-  static constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 192, T_DV = 256, T_DK = 384;
+  // S^T is double-buffered: [0,64) for even query tiles, [64,128) for odd ones.  So is the
+  // gradient pair at T_G: tile n's dP^T goes to [T_G + 64 (n & 1), +64), and once dS_n has
+  // been computed from it, tile n's dQ^T goes to the same columns.
+  static constexpr uint32_t T_S = 0, T_G = 128, T_DV = 256, T_DK = 384;
   static constexpr uint32_t IDESC_S = idesc_bf16(128, BQ, false, false);   // S^T, dP^T
   static constexpr uint32_t IDESC_KV = idesc_bf16(128, D, false, true);    // dV, dK (B MN-major)
   static constexpr uint32_t IDESC_Q = idesc_bf16(128, BQ, true, true);     // dQ^T
@@ -157,8 +159,10 @@ struct BwdCfg {
 //
 // The schedule keeps the slow chains (scores -> P on the compute warps, P -> dV on the tensor
 // core) off each other's critical path: S^T is double-buffered, so S_{n+2} is issued right
-// after dV_n; and since dK reads dS^T from shared memory, the dP^T columns are free as soon
-// as dS_n is computed, so dP_{n+1} is issued before dK_n and dQ_n.
+// after dV_n.  dP^T and dQ^T share two alternating TMEM buffers: dP_n is dead once dS_n is
+// computed, so dQ_n takes its columns, and dP_{n+1} goes to the other buffer as soon as the
+// drain has read dQ_{n-1} from it (without dQ: as soon as dS_{n-1} is computed), so it is
+// done before the compute warps need it instead of being issued after dS_n.
 // WITH_DQ = false: dK and dV only (dQ comes from fa_bwd_dq_kernel): no dQ^T MMA, no drain.  The dQ^T MMA puts d on the M dimension (128 TMEM lanes), so the
 // atomic dQ path exists for D = 128 only; D = 64 always runs with WITH_DQ = false.
 template <int D, bool WITH_DQ>
@@ -194,24 +198,26 @@ __global__ void __launch_bounds__(480, 1)
   const uint32_t kv_full = bar;
   auto qd_full = [&](int s) { return bar + 8u * (1 + s); };
   auto qd_empty = [&](int s) { return bar + 8u * (1 + C::NSQ + s); };
-  // barrier block after the ring's: s_full[2] 0, 8 | dp_full 16 | p_ready[2] 24, 32 | dq_full 40 |
-  // dq_free 48 | ds_free[2] 56, 64 | kv_done 72 | dv_done[2] 80, 88 | sc_done 96 | ds_ready[2]
-  // 104, 112: fifteen 8-byte barriers
-  static_assert(C::NBAR == 1 + 2 * C::NSQ + 15, "barrier block layout");
+  // barrier block after the ring's: s_full[2] 0, 8 | dp_full[2] 16, 24 | p_ready[2] 32, 40 |
+  // dq_full[2] 48, 56 | dq_free[2] 64, 72 | ds_free[2] 80, 88 | kv_done 96 | dv_done[2] 104, 112 |
+  // sc_done 120 | ds_ready[2] 128, 136: eighteen 8-byte barriers
+  static_assert(C::NBAR == 1 + 2 * C::NSQ + 18, "barrier block layout");
   const uint32_t bar2 = bar + 8u * (1 + 2 * C::NSQ);
   auto s_full = [&](int b) { return bar2 + 8u * b; };
-  const uint32_t dp_full = bar2 + 16;
+  // The gradient-pair buffers (b = n & 1), one barrier each way: dP_n complete (dp_full),
+  // dQ_n complete (dq_full), dQ_n read by the drain (dq_free)
+  auto dp_full = [&](int b) { return bar2 + 16 + 8u * b; };
   // P_n and dS_n ready, one barrier per S^T / dS^T buffer (b = n & 1): a tile's arrival on a
   // buffer needs the previous tile of that buffer consumed by both issuers, so no waiter ever
   // falls two phases behind
-  auto p_ready = [&](int b) { return bar2 + 24 + 8u * b; };
-  auto ds_ready = [&](int b) { return bar2 + 104 + 8u * b; };
-  const uint32_t dq_full = bar2 + 40;
-  const uint32_t dq_free = bar2 + 48;
-  auto ds_free = [&](int b) { return bar2 + 56 + 8u * b; };
-  const uint32_t kv_done = bar2 + 72;
-  auto dv_done = [&](int b) { return bar2 + 80 + 8u * b; };  // dV_n (n & 1 == b) has completed
-  const uint32_t sc_done = bar2 + 96;                        // every score product has completed
+  auto p_ready = [&](int b) { return bar2 + 32 + 8u * b; };
+  auto ds_ready = [&](int b) { return bar2 + 128 + 8u * b; };
+  auto dq_full = [&](int b) { return bar2 + 48 + 8u * b; };
+  auto dq_free = [&](int b) { return bar2 + 64 + 8u * b; };
+  auto ds_free = [&](int b) { return bar2 + 80 + 8u * b; };
+  const uint32_t kv_done = bar2 + 96;
+  auto dv_done = [&](int b) { return bar2 + 104 + 8u * b; };  // dV_n (n & 1 == b) has completed
+  const uint32_t sc_done = bar2 + 120;                        // every score product has completed
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gb + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + C::MISC_OFF + 4);
   const WaitCtx wc{abort_flag, a.status};
@@ -222,13 +228,13 @@ __global__ void __launch_bounds__(480, 1)
       mbar_init(qd_full(s), 1);
       mbar_init(qd_empty(s), 2);  // released by both issuers
     }
-    mbar_init(dp_full, 1);
     for (int b = 0; b < 2; ++b) {
+      mbar_init(dp_full(b), 1);
       mbar_init(p_ready(b), 256);
       mbar_init(ds_ready(b), 256);
+      mbar_init(dq_full(b), 1);
+      mbar_init(dq_free(b), 128);
     }
-    mbar_init(dq_full, 1);
-    mbar_init(dq_free, 128);
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full(b), 1);
       mbar_init(ds_free(b), 1);
@@ -298,13 +304,14 @@ __global__ void __launch_bounds__(480, 1)
     __syncwarp();
   } else if (warp == 12 || warp == 14) {
     // ------------------------------------------------------------ MMA issuers (whole warps)
-    // Score issuer:    S_0, S_1, dP_0 | [dS_n ready] dP_(n+1), [dV_n done] S_(n+2) | ...
-    // Gradient issuer: [P_n ready] dV_n | [dS_n ready] dK_n, [drain done] dQ_n | ...
-    // Every overwrite follows its last reader: dP_(n+1) follows the compute warps' read of dP_n
-    // (ds_ready), S_(n+2) follows dV_n (dv_done), which reads P_n from the same TMEM buffer;
-    // dQ_n follows the drain's read of dQ_(n-1) (dq_free); the dS^T buffer is released after
-    // dK_n and dQ_n (ds_free), a Q/dO stage after S_n, dP_n (score issuer) and dV_n, dK_n
-    // (gradient issuer).  The gradient issuer's last commit (kv_done) also covers every score
+    // Score issuer:    S_0, S_1, dP_0 | [dQ_(n-1) drained] dP_(n+1), [dV_n done] S_(n+2) | ...
+    // Gradient issuer: [P_n ready] dV_n | [dS_n ready] dK_n, dQ_n | ...
+    // Every overwrite follows its last reader: dP_(n+1) follows the drain's read of dQ_(n-1)
+    // from the same gradient-pair buffer (dq_free; without dQ, the compute warps' read of
+    // dP_(n-1), ds_ready), dQ_n follows the compute warps' read of dP_n (ds_ready), S_(n+2)
+    // follows dV_n (dv_done), which reads P_n from the same TMEM buffer; the dS^T buffer is
+    // released after dK_n and dQ_n (ds_free), a Q/dO stage after S_n, dP_n (score issuer) and
+    // dV_n, dK_n (gradient issuer).  The gradient issuer's last commit (kv_done) also covers every score
     // product: each one was consumed by the compute warps before the last dV or dK could start.
     if (!*abort_flag) {
       bool ok = __all_sync(0xffffffffu, mbar_wait(kv_full, 0, wc));
@@ -334,9 +341,10 @@ __global__ void __launch_bounds__(480, 1)
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
             const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32, qo = (k >> 2) * 8192 + (k & 3) * 32;
-            mma_ss_e(tmem + C::T_DP, sdesc_add(dV_k, ko), sdesc_add(dO_k, so + qo), C::IDESC_S, k > 0);
+            mma_ss_e(tmem + C::T_G + 64 * (n & 1), sdesc_add(dV_k, ko), sdesc_add(dO_k, so + qo), C::IDESC_S,
+                     k > 0);
           }
-          mma_commit_e(dp_full);
+          mma_commit_e(dp_full(n & 1));
           mma_commit_e(qd_empty(n % C::NSQ));
         };
         auto wait_q = [&](int n) {
@@ -355,7 +363,11 @@ __global__ void __launch_bounds__(480, 1)
         }
         for (int n = 0; n < count && ok; ++n) {
           if (n + 1 < count) {  // dO_(n+1) landed before S_(n+1) was issued
-            if (!(ok = __all_sync(0xffffffffu, mbar_wait(ds_ready(n & 1), (n >> 1) & 1, wc)))) break;
+            if (n >= 1) {  // buffer (n+1) & 1 last held tile n-1's dQ^T (or, without dQ, its dP^T)
+              const int b1 = (n - 1) & 1;
+              const uint32_t ph = ((n - 1) >> 1) & 1;
+              if (!(ok = __all_sync(0xffffffffu, mbar_wait(WITH_DQ ? dq_free(b1) : ds_ready(b1), ph, wc)))) break;
+            }
             tc_fence_after();
             issue_dp(n + 1);
           }
@@ -387,13 +399,11 @@ __global__ void __launch_bounds__(480, 1)
             mma_ss_e(tmem + C::T_DK, sdesc_add(dS_k, b * C::DS_BYTES + 32 * k), sdesc_add(dQ_mn, so + k * 2048),
                      C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
           if (WITH_DQ) {
-            if (!(ok = __all_sync(0xffffffffu, mbar_wait(dq_free, (n & 1) ^ 1, wc)))) break;
-            tc_fence_after();
 #pragma unroll
-            for (int k = 0; k < 8; ++k)  // dQ_i^T = K_j^T dS^T  (K over the 128 keys)
-              mma_ss_e(tmem + C::T_DQ, sdesc_add(dK_mn, k * 2048), sdesc_add(dS_mn, b * C::DS_BYTES + k * 2048),
-                       C::IDESC_Q, k > 0);
-            mma_commit_e(dq_full);
+            for (int k = 0; k < 8; ++k)  // dQ_i^T = K_j^T dS^T (K over the 128 keys), over dP_n's columns
+              mma_ss_e(tmem + C::T_G + 64 * b, sdesc_add(dK_mn, k * 2048),
+                       sdesc_add(dS_mn, b * C::DS_BYTES + k * 2048), C::IDESC_Q, k > 0);
+            mma_commit_e(dq_full(b));
           }
           mma_commit_e(ds_free(b));
           mma_commit_e(qd_empty(s));
@@ -412,7 +422,7 @@ __global__ void __launch_bounds__(480, 1)
     const bool key_ok = key < a.N;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS0 = tmem + lane_off + C::T_S + 32 * g;  // + 64 for odd query tiles
-    const uint32_t tDP = tmem + lane_off + C::T_DP + 32 * g;
+    const uint32_t tDP = tmem + lane_off + C::T_G + 32 * g;  // + 64 for odd query tiles
     const float cs = a.scale_log2;
     bool ok = !*abort_flag;
     for (int n = 0; n < count && ok; ++n) {
@@ -457,10 +467,10 @@ __global__ void __launch_bounds__(480, 1)
       tc_fence_before();
       mbar_arrive(p_ready(b));
 
-      ok = __all_sync(0xffffffffu, mbar_wait(dp_full, n & 1, wc));
+      ok = __all_sync(0xffffffffu, mbar_wait(dp_full(b), (n >> 1) & 1, wc));
       if (!ok) break;
       tc_fence_after();
-      tmem_ld32(tDP, sr);
+      tmem_ld32(tDP + 64 * b, sr);
       tmem_wait_ld();
       reg_fence(sr);
 #pragma unroll
@@ -485,7 +495,7 @@ __global__ void __launch_bounds__(480, 1)
             make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
       }
       fence_proxy_async_smem();
-      tc_fence_before();  // the tcgen05.ld of dP^T is complete before dP_{n+1} may overwrite it
+      tc_fence_before();  // the tcgen05.ld of dP^T is complete before dQ_n may overwrite it
       mbar_arrive(ds_ready(b));
     }
   } else {
@@ -497,16 +507,18 @@ __global__ void __launch_bounds__(480, 1)
     bool ok = !*abort_flag;
     for (int n = 0; n < (WITH_DQ ? count : 0) && ok; ++n) {
       const int i = i0 + n;
-      ok = __all_sync(0xffffffffu, mbar_wait(dq_full, n & 1, wc));
+      const int b = n & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(dq_full(b), (n >> 1) & 1, wc));
       if (!ok) break;
       tc_fence_after();
       uint32_t v[64];
-      tmem_ld32(tmem + lane_off + C::T_DQ, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_ld32(tmem + lane_off + C::T_DQ + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      const uint32_t tq = tmem + lane_off + C::T_G + 64 * b;
+      tmem_ld32(tq, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_ld32(tq + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
       tmem_wait_ld();
       reg_fence(v);
       tc_fence_before();
-      mbar_arrive(dq_free);  // one dQ^T buffer: the next dQ MMA may overwrite it now
+      mbar_arrive(dq_free(b));  // dP_(n+2) may overwrite these columns now
       // Split between two paths that use different resources: the first kBwdDqRedRows query
       // rows are added with fp32 reductions straight from registers (lane = d, so each row is
       // one coalesced 128-byte request), the rest are staged as a [rows][32 d] fp32 slice in
