@@ -124,7 +124,7 @@ struct BwdCfg {
   static constexpr int DQS_WARP = (BQ - kBwdDqRedRows) * 32 * 4;
   static constexpr int LD_OFF = DQS_OFF + 4 * DQS_WARP;
   static constexpr int BAR_OFF = LD_OFF + NSQ * LDB;
-  // kv_full, qd_full[3], qd_empty[3], s_full[2], dp_full[2], p_ready[2], ds_ready[2],
+  // kv_full, qd_full[3], qd_empty[3], s_full, s_free, dp_full[2], p_ready[2], ds_ready[2],
   // dq_full[2], dq_free[2], ds_free[2], kv_done, dv_done[2], sc_done
   static constexpr int NBAR = 1 + 2 * NSQ + 18;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
@@ -132,10 +132,11 @@ struct BwdCfg {
   static constexpr int THREADS = 480;
   static constexpr uint32_t TMEM_COLS = 512;
   // TMEM columns (a 512-column allocation always starts at column 0, lane 0)
-  // S^T is double-buffered: [0,64) for even query tiles, [64,128) for odd ones.  So is the
+  // S^T has one buffer [0, 64), released as soon as the compute warps have loaded it.  P^T
+  // (bf16, two per column) is double-buffered: tile n's at [T_P + 32 (n & 1), +32).  So is the
   // gradient pair at T_G: tile n's dP^T goes to [T_G + 64 (n & 1), +64), and once dS_n has
   // been computed from it, tile n's dQ^T goes to the same columns.
-  static constexpr uint32_t T_S = 0, T_G = 128, T_DV = 256, T_DK = 384;
+  static constexpr uint32_t T_S = 0, T_P = 64, T_G = 128, T_DV = 256, T_DK = 384;
   static constexpr uint32_t IDESC_S = idesc_bf16(128, BQ, false, false);   // S^T, dP^T
   static constexpr uint32_t IDESC_KV = idesc_bf16(128, D, false, true);    // dV, dK (B MN-major)
   static constexpr uint32_t IDESC_Q = idesc_bf16(128, BQ, true, true);     // dQ^T
@@ -149,17 +150,18 @@ struct BwdCfg {
 //   warp 13     TMA producer (whole warp, one elected lane issues)
 //   warp 14     gradient issuer: dV, dK and dQ^T
 // Two issuers, so that neither kind of product waits behind the other's barriers and commits.
-// Their products share no accumulator; the one overwrite that crosses them (S^T of tile n+2
-// into the TMEM buffer whose P^T dV_n reads) waits for dv_done, which the gradient issuer
-// commits after dV_n, and a Q/dO stage is released when both have committed their last use.
-// Each compute warpgroup writes its packed P^T inside its own S^T columns, so neither
-// overwrites scores the other has not read yet: P^T of query columns [32g, 32g+32) sits at
-// TMEM columns [32g, 32g+16) of the tile's S^T buffer.  dS^T goes to shared memory only,
-// where it is the A operand of dK += dS^T Q_i and the B operand of dQ^T = K_j^T dS^T.
+// Their products share no accumulator; the one overwrite that crosses them (dP^T of tile n+1
+// into the columns whose dQ^T of tile n-1 the drain reads) waits for dq_free, and a Q/dO
+// stage is released when both have committed their last use.  P^T of query columns
+// [32g, 32g+32) sits at TMEM columns [16g, 16g+16) of the tile's P^T buffer.  dS^T goes to
+// shared memory only, where it is the A operand of dK += dS^T Q_i and the B operand of
+// dQ^T = K_j^T dS^T.
 //
 // The schedule keeps the slow chains (scores -> P on the compute warps, P -> dV on the tensor
-// core) off each other's critical path: S^T is double-buffered, so S_{n+2} is issued right
-// after dV_n.  dP^T and dQ^T share two alternating TMEM buffers: dP_n is dead once dS_n is
+// core) off each other's critical path: with P^T in its own buffers, S_{n+1} is issued as soon
+// as the compute warps have loaded S_n into registers, long before they need it, and a P^T
+// buffer is rewritten two tiles after its dV.  dP^T and dQ^T share two alternating TMEM
+// buffers: dP_n is dead once dS_n is
 // computed, so dQ_n takes its columns, and dP_{n+1} goes to the other buffer as soon as the
 // drain has read dQ_{n-1} from it (without dQ: as soon as dS_{n-1} is computed), so it is
 // done before the compute warps need it instead of being issued after dS_n.
@@ -198,16 +200,17 @@ __global__ void __launch_bounds__(480, 1)
   const uint32_t kv_full = bar;
   auto qd_full = [&](int s) { return bar + 8u * (1 + s); };
   auto qd_empty = [&](int s) { return bar + 8u * (1 + C::NSQ + s); };
-  // barrier block after the ring's: s_full[2] 0, 8 | dp_full[2] 16, 24 | p_ready[2] 32, 40 |
+  // barrier block after the ring's: s_full 0 | s_free 8 | dp_full[2] 16, 24 | p_ready[2] 32, 40 |
   // dq_full[2] 48, 56 | dq_free[2] 64, 72 | ds_free[2] 80, 88 | kv_done 96 | dv_done[2] 104, 112 |
   // sc_done 120 | ds_ready[2] 128, 136: eighteen 8-byte barriers
   static_assert(C::NBAR == 1 + 2 * C::NSQ + 18, "barrier block layout");
   const uint32_t bar2 = bar + 8u * (1 + 2 * C::NSQ);
-  auto s_full = [&](int b) { return bar2 + 8u * b; };
+  const uint32_t s_full = bar2;      // S_n complete
+  const uint32_t s_free = bar2 + 8;  // S_n loaded by both compute warpgroups
   // The gradient-pair buffers (b = n & 1), one barrier each way: dP_n complete (dp_full),
   // dQ_n complete (dq_full), dQ_n read by the drain (dq_free)
   auto dp_full = [&](int b) { return bar2 + 16 + 8u * b; };
-  // P_n and dS_n ready, one barrier per S^T / dS^T buffer (b = n & 1): a tile's arrival on a
+  // P_n and dS_n ready, one barrier per P^T / dS^T buffer (b = n & 1): a tile's arrival on a
   // buffer needs the previous tile of that buffer consumed by both issuers, so no waiter ever
   // falls two phases behind
   auto p_ready = [&](int b) { return bar2 + 32 + 8u * b; };
@@ -235,8 +238,9 @@ __global__ void __launch_bounds__(480, 1)
       mbar_init(dq_full(b), 1);
       mbar_init(dq_free(b), 128);
     }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 256);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(s_full(b), 1);
       mbar_init(ds_free(b), 1);
       mbar_init(dv_done(b), 1);
     }
@@ -304,14 +308,14 @@ __global__ void __launch_bounds__(480, 1)
     __syncwarp();
   } else if (warp == 12 || warp == 14) {
     // ------------------------------------------------------------ MMA issuers (whole warps)
-    // Score issuer:    S_0, S_1, dP_0 | [dQ_(n-1) drained] dP_(n+1), [dV_n done] S_(n+2) | ...
+    // Score issuer:    S_0, dP_0 | [S_n loaded] S_(n+1), [dQ_(n-1) drained] dP_(n+1) | ...
     // Gradient issuer: [P_n ready] dV_n | [dS_n ready] dK_n, dQ_n | ...
-    // Every overwrite follows its last reader: dP_(n+1) follows the drain's read of dQ_(n-1)
-    // from the same gradient-pair buffer (dq_free; without dQ, the compute warps' read of
-    // dP_(n-1), ds_ready), dQ_n follows the compute warps' read of dP_n (ds_ready), S_(n+2)
-    // follows dV_n (dv_done), which reads P_n from the same TMEM buffer; the dS^T buffer is
-    // released after dK_n and dQ_n (ds_free), a Q/dO stage after S_n, dP_n (score issuer) and
-    // dV_n, dK_n (gradient issuer).  The gradient issuer's last commit (kv_done) also covers every score
+    // Every overwrite follows its last reader: S_(n+1) follows the compute warps' load of S_n
+    // (s_free), dP_(n+1) follows the drain's read of dQ_(n-1) from the same gradient-pair buffer
+    // (dq_free; without dQ, the compute warps' read of dP_(n-1), ds_ready), dQ_n follows the
+    // compute warps' read of dP_n (ds_ready), P_(n+2) follows dV_n (dv_done, waited by the
+    // compute warps); the dS^T buffer is released after dK_n and dQ_n (ds_free), a Q/dO stage
+    // after S_n, dP_n (score issuer) and dV_n, dK_n (gradient issuer).  The gradient issuer's last commit (kv_done) also covers every score
     // product: each one was consumed by the compute warps before the last dV or dK could start.
     if (!*abort_flag) {
       bool ok = __all_sync(0xffffffffu, mbar_wait(kv_full, 0, wc));
@@ -327,14 +331,14 @@ __global__ void __launch_bounds__(480, 1)
       const uint64_t dS_mn = sdesc_sw128(sb + C::DS_OFF, 8192, 1024);    // dS^T, MN-major (dQ^T)
       auto st_off = [&](int n) { return (uint32_t)((n % C::NSQ) * C::ST_BYTES); };
       if (warp == 12) {
-        auto issue_s = [&](int n) {  // S^T = K_j Q_i^T  (K over d), into buffer n & 1
+        auto issue_s = [&](int n) {  // S^T = K_j Q_i^T  (K over d)
           const uint32_t so = st_off(n);
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
             const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32, qo = (k >> 2) * 8192 + (k & 3) * 32;
-            mma_ss_e(tmem + C::T_S + 64 * (n & 1), sdesc_add(dK_k, ko), sdesc_add(dQ_k, so + qo), C::IDESC_S, k > 0);
+            mma_ss_e(tmem + C::T_S, sdesc_add(dK_k, ko), sdesc_add(dQ_k, so + qo), C::IDESC_S, k > 0);
           }
-          mma_commit_e(s_full(n & 1));
+          mma_commit_e(s_full);
         };
         auto issue_dp = [&](int n) {  // dP^T = V_j dO_i^T; the last score product of tile n
           const uint32_t so = st_off(n);
@@ -354,29 +358,21 @@ __global__ void __launch_bounds__(480, 1)
           if ((ok = wait_q(0))) {
             tc_fence_after();
             issue_s(0);
-            if (count > 1 && (ok = wait_q(1))) {
-              tc_fence_after();
-              issue_s(1);
-            }
-            if (ok) issue_dp(0);
+            issue_dp(0);
           }
         }
-        for (int n = 0; n < count && ok; ++n) {
-          if (n + 1 < count) {  // dO_(n+1) landed before S_(n+1) was issued
-            if (n >= 1) {  // buffer (n+1) & 1 last held tile n-1's dQ^T (or, without dQ, its dP^T)
-              const int b1 = (n - 1) & 1;
-              const uint32_t ph = ((n - 1) >> 1) & 1;
-              if (!(ok = __all_sync(0xffffffffu, mbar_wait(WITH_DQ ? dq_free(b1) : ds_ready(b1), ph, wc)))) break;
-            }
+        for (int n = 0; n + 1 < count && ok; ++n) {
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(s_free, n & 1, wc)))) break;
+          if (!(ok = wait_q(n + 1))) break;
+          tc_fence_after();
+          issue_s(n + 1);
+          if (n >= 1) {  // buffer (n+1) & 1 last held tile n-1's dQ^T (or, without dQ, its dP^T)
+            const int b1 = (n - 1) & 1;
+            const uint32_t ph = ((n - 1) >> 1) & 1;
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(WITH_DQ ? dq_free(b1) : ds_ready(b1), ph, wc)))) break;
             tc_fence_after();
-            issue_dp(n + 1);
           }
-          if (n + 2 < count) {
-            if (!(ok = __all_sync(0xffffffffu, mbar_wait(dv_done(n & 1), (n >> 1) & 1, wc)))) break;
-            if (!(ok = wait_q(n + 2))) break;
-            tc_fence_after();
-            issue_s(n + 2);
-          }
+          issue_dp(n + 1);
         }
         mma_commit_e(sc_done);
         if (!ok) mbar_wait_drain(sc_done, 0);
@@ -389,7 +385,7 @@ __global__ void __launch_bounds__(480, 1)
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 4; ++k)  // dV += P^T dO_i  (K over the 64 queries; A = P^T from TMEM)
-            mma_ts_e(tmem + C::T_DV, tmem + C::T_S + 64 * b + 32 * (k >> 1) + 8 * (k & 1),
+            mma_ts_e(tmem + C::T_DV, tmem + C::T_P + 32 * b + 8 * k,
                      sdesc_add(dO_mn, so + k * 2048), C::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
           mma_commit_e(dv_done(b));
           if (!(ok = __all_sync(0xffffffffu, mbar_wait(ds_ready(b), (n >> 1) & 1, wc)))) break;
@@ -421,7 +417,8 @@ __global__ void __launch_bounds__(480, 1)
     const int key = 128 * j + r;
     const bool key_ok = key < a.N;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS0 = tmem + lane_off + C::T_S + 32 * g;  // + 64 for odd query tiles
+    const uint32_t tS = tmem + lane_off + C::T_S + 32 * g;
+    const uint32_t tP0 = tmem + lane_off + C::T_P + 16 * g;  // + 32 for odd query tiles
     const uint32_t tDP = tmem + lane_off + C::T_G + 32 * g;  // + 64 for odd query tiles
     const float cs = a.scale_log2;
     bool ok = !*abort_flag;
@@ -430,16 +427,17 @@ __global__ void __launch_bounds__(480, 1)
       const int i = i0 + n;
       const int b = n & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(qd_full(s), (n / C::NSQ) & 1, wc) &&
-                                       mbar_wait(s_full(b), (n >> 1) & 1, wc));
+                                       mbar_wait(s_full, n & 1, wc));
       if (!ok) break;
       tc_fence_after();
       FA_DBG(if (g == 0 && wq == 0 && lane == 0) dbg_visit(a.visits, a.visits_cap, a.status, bh, Tq, i, Tk, j);)
-      const uint32_t tS = tS0 + 64 * b;
       uint32_t sr[32];
       tmem_ld32(tS, sr);
       const float* ldp = reinterpret_cast<const float*>(gb + C::LD_OFF + s * C::LDB) + 32 * g;
       tmem_wait_ld();
       reg_fence(sr);
+      tc_fence_before();
+      mbar_arrive(s_free);  // S_n is in registers: S_(n+1) may overwrite it
       // causal: query 64 i + 32 g + c sees this key iff it is >= key
       const int first_vis = a.causal ? (key - C::BQ * i - 32 * g) : -1;  // first visible column
       float p[32];
@@ -462,7 +460,11 @@ __global__ void __launch_bounds__(480, 1)
       uint32_t pk[16];
 #pragma unroll
       for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(p[2 * c], p[2 * c + 1]);
-      tmem_st16(tS, pk);
+      // P^T buffer b last held P_(n-2): wait until dV_(n-2) has read it
+      ok = __all_sync(0xffffffffu, mbar_wait(dv_done(b), ((n >> 1) & 1) ^ 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      tmem_st16(tP0 + 32 * b, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_ready(b));
