@@ -465,7 +465,8 @@ def measure_variants(w, dev, stream, qd, kd, vd, o, lse, dod, dq, dk, dv, ws, ws
                           "unsplit_ms": round(ms_u, 4),
                           "unsplit_tflops": round(ws2.fwd_flops() / (ms_u * 1e-3) / 1e12, 1)}
     del q2, k2, v2, o2, l2, wsk
-    # d = 64 backward (two-pass path), B=4 H=16 N=1024 d=64 non-causal
+    # d = 64 backward (one pass, dQ by fp32 reductions; the deterministic two-pass path beside
+    # it), B=4 H=16 N=1024 d=64 non-causal
     w64 = custom(4, 16, 1024, 64, False, seed=0, backward=True)
     q6, k6, v6, d6 = (t.to(dev) for t in make_inputs(w64, with_grad=True))
     o6, l6 = torch.empty_like(q6), torch.empty((4, 16, 1024), device=dev, dtype=torch.float32)
@@ -476,9 +477,13 @@ def measure_variants(w, dev, stream, qd, kd, vd, o, lse, dod, dq, dk, dv, ws, ws
     ms = _time_ms(lambda: chk(fa.fa_bwd(q6, k6, v6, o6, d6, l6, *g6, w6, wb6, 4, 16, 1024, 64, w64.scale, 0, sp),
                               "fa_bwd d=64"), stream)
     tf = w64.bwd_flops() / (ms * 1e-3) / 1e12
-    out["bwd_d64"] = {"kernels": "fa_bwd_main_kernel<64, no dQ> + fa_bwd_dq_kernel<64>",
+    ms2 = _time_ms(lambda: chk(fa.fa_bwd_deterministic(q6, k6, v6, o6, d6, l6, *g6, w6, wb6, 4, 16, 1024, 64,
+                                                       w64.scale, 0, sp), "fa_bwd_deterministic d=64"), stream)
+    out["bwd_d64"] = {"kernels": "fa_bwd_pre_kernel<64> + fa_bwd_main_kernel<64> + fa_bwd_post_kernel",
                       "shape": "B=4 H=16 N=1024 d=64", "ms": round(ms, 4), "tflops": round(tf, 1),
-                      "peak": peak, "frac": round(tf / peak, 4)}
+                      "peak": peak, "frac": round(tf / peak, 4),
+                      "deterministic_ms": round(ms2, 4),
+                      "deterministic_tflops": round(w64.bwd_flops() / (ms2 * 1e-3) / 1e12, 1)}
     # sequence sharded into 4 pieces (ring schedule), every rank's pieces on this GPU in turn:
     # the partial-result and merge overhead of sharding, without the exchange
     from io_aware_exact_22_b200 import ring

@@ -163,8 +163,8 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
  *   workspace      : device scratch of at least fa_bwd_workspace_bytes(B,H,N,d) bytes,
  *                    256-byte aligned; its contents on entry do not matter and on exit
  *                    are unspecified.  Concurrent calls need distinct workspaces.
- * At d == 128, dQ is summed over key tiles with fp32 atomics (dK, dV in a fixed order); at
- * d == 64 the call runs fa_bwd_deterministic's two passes.
+ * dQ is summed over key tiles with fp32 reductions (dK, dV in a fixed order), at both head
+ * dimensions; fa_bwd_deterministic gives a dQ summed in a fixed order instead.
  */
 fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o,
                    const void* dO, const float* lse, void* dq, void* dk, void* dv,
@@ -213,7 +213,7 @@ fa_status_t fa_bwd_deterministic(const void* q, const void* k, const void* v, co
 
 /*
  * The backward in three steps, for callers that hold the keys in pieces (the sequence-sharded
- * backward: every key set's contribution is added in turn).  d == 128.  The workspace has
+ * backward: every key set's contribution is added in turn).  d in {64, 128}.  The workspace has
  * fa_bwd's layout and size; dk_acc, dv_acc are caller-owned fp32 [B,H,N,d] accumulators
  * (16-byte aligned) for the keys of one piece, zeroed by the caller before the first addition.
  *   fa_bwd_prepare    : from this rank's o, dO (bf16) and lse (fp32), the per-row statistics
@@ -237,7 +237,7 @@ fa_status_t fa_bwd_finish(const void* workspace, size_t workspace_bytes, const f
                           int B, int H, int N, int d, float scale, void* stream);
 
 /*
- * fa_bwd (d == 128) taken apart into its three kernels, so that each can be launched, and
+ * fa_bwd taken apart into its three kernels, so that each can be launched, and
  * timed, on its own.  fa_bwd_prepare (above), then fa_bwd_main, then fa_bwd_dq_post, on one
  * stream and one workspace, give exactly what fa_bwd gives.
  *   fa_bwd_main    : the key-tile pass on prepared statistics: recomputes S and P tile by tile,
@@ -245,7 +245,7 @@ fa_status_t fa_bwd_finish(const void* workspace, size_t workspace_bytes, const f
  *                    aligned) and adds dS K into the workspace's fp32 dQ accumulator.
  *                    q, k, v, dO as for fa_bwd.
  *   fa_bwd_dq_post : dq = scale * accumulator, rounded to bf16 ([B,H,N,d], 16-byte aligned).
- * Same error rules as fa_bwd; d != 128 returns FA_ERR_UNSUPPORTED.
+ * Same error rules as fa_bwd (d in {64, 128}).
  */
 fa_status_t fa_bwd_main(const void* q, const void* k, const void* v, const void* dO,
                         void* workspace, size_t workspace_bytes, void* dk, void* dv,

@@ -482,15 +482,12 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   return ld_bytes((long long)B * H, N) + (size_t)rows * d * 4;
 }
 
-// The key-tile kernel of fa_bwd on prepared statistics: bf16 dK, dV stored, dQ added into the
+// The key-tile kernel of fa_bwd on prepared statistics (d = 64 or 128): bf16 dK, dV stored (or,
+// with dk_acc set, scale * dK and dV added into fp32 accumulators), dQ added into the
 // workspace's fp32 accumulator.  Arguments are checked by the callers.
-// The key-tile kernel of fa_bwd on prepared statistics: bf16 dK, dV stored (or, with dk_acc set,
-// scale * dK and dV added into fp32 accumulators), dQ added into the workspace's fp32
-// accumulator.  Arguments are checked by the callers.
-static fa_status_t bwd_main_d128(const void* q, const void* k, const void* v, const void* dO, void* workspace,
-                                 void* dk, void* dv, int BH, int N, float scale, int causal, cudaStream_t s,
-                                 float* dk_acc = nullptr, float* dv_acc = nullptr) {
-  const int d = 128;
+static fa_status_t bwd_main_dq(const void* q, const void* k, const void* v, const void* dO, void* workspace,
+                               void* dk, void* dv, int BH, int N, int d, float scale, int causal, cudaStream_t s,
+                               float* dk_acc = nullptr, float* dv_acc = nullptr) {
   float* ld = reinterpret_cast<float*>(workspace);
   float* dq_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + ld_bytes(BH, N));
   CUtensorMap tq, tk, tv, tdo, tdk, tdv, tdq;
@@ -540,11 +537,6 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
   bool empty = false;
   fa_status_t st = check_shape(B, H, N, d, scale, causal, &empty);
   if (st != FA_OK || empty) return st;
-  // d = 64: the key pass has no atomic dQ path there, so dQ comes from the query pass
-  if (d == 64)
-    return fa_bwd_deterministic(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes, B, H, N, d, scale,
-                                causal, stream);
-  if (d != 128) return FA_ERR_UNSUPPORTED;
   if ((st = check_bwd_io(q, k, v, dO, dk, dv, workspace, workspace_bytes, B, H, N, d)) != FA_OK) return st;
   if (!o || !lse || !dq || !aligned(o, 16) || !aligned(dq, 16) || !aligned(lse, 4)) return FA_ERR_INVALID_ARG;
   if ((st = check_device()) != FA_OK) return st;
@@ -554,7 +546,7 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
   float* dq_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + ld_bytes(BH, N));
   cudaStream_t s = (cudaStream_t)stream;
   if (launch_bwd_pre(o, dO, lse, ld, dq_acc, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
-  if ((st = bwd_main_d128(q, k, v, dO, workspace, dk, dv, BH, N, scale, causal, s)) != FA_OK) return st;
+  if ((st = bwd_main_dq(q, k, v, dO, workspace, dk, dv, BH, N, d, scale, causal, s)) != FA_OK) return st;
   if (launch_bwd_post(dq_acc, dq, rows * d, scale, s) != cudaSuccess) return FA_ERR_CUDA;
   return FA_OK;
 }
@@ -565,10 +557,9 @@ fa_status_t fa_bwd_main(const void* q, const void* k, const void* v, const void*
   bool empty = false;
   fa_status_t st = check_shape(B, H, N, d, scale, causal, &empty);
   if (st != FA_OK || empty) return st;
-  if (d != 128) return FA_ERR_UNSUPPORTED;
   if ((st = check_bwd_io(q, k, v, dO, dk, dv, workspace, workspace_bytes, B, H, N, d)) != FA_OK) return st;
   if ((st = check_device()) != FA_OK) return st;
-  return bwd_main_d128(q, k, v, dO, workspace, dk, dv, B * H, N, scale, causal, (cudaStream_t)stream);
+  return bwd_main_dq(q, k, v, dO, workspace, dk, dv, B * H, N, d, scale, causal, (cudaStream_t)stream);
 }
 
 fa_status_t fa_bwd_dq_post(const void* workspace, size_t workspace_bytes, void* dq, int B, int H, int N, int d,
@@ -576,7 +567,6 @@ fa_status_t fa_bwd_dq_post(const void* workspace, size_t workspace_bytes, void* 
   bool empty = false;
   fa_status_t st = check_shape(B, H, N, d, scale, 0, &empty);
   if (st != FA_OK || empty) return st;
-  if (d != 128) return FA_ERR_UNSUPPORTED;
   if (!workspace || !dq || !aligned(workspace, 256) || !aligned(dq, 16)) return FA_ERR_INVALID_ARG;
   if (workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
   if ((st = check_device()) != FA_OK) return st;
@@ -591,7 +581,6 @@ fa_status_t fa_bwd_prepare(const void* o, const void* dO, const float* lse, void
   bool empty = false;
   fa_status_t st = check_shape(B, H, N, d, 1.0f, 0, &empty);
   if (st != FA_OK || empty) return st;
-  if (d != 128) return FA_ERR_UNSUPPORTED;
   if (!o || !dO || !lse || !workspace) return FA_ERR_INVALID_ARG;
   if (!aligned(o, 16) || !aligned(dO, 16) || !aligned(lse, 4) || !aligned(workspace, 256)) return FA_ERR_INVALID_ARG;
   if (workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
@@ -609,14 +598,13 @@ fa_status_t fa_bwd_accumulate(const void* q, const void* k, const void* v, const
   bool empty = false;
   fa_status_t st = check_shape(B, H, N, d, scale, causal, &empty);
   if (st != FA_OK || empty) return st;
-  if (d != 128) return FA_ERR_UNSUPPORTED;
   if (!q || !k || !v || !dO || !workspace || !dk_acc || !dv_acc) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dO, 16) || !aligned(workspace, 256) ||
       !aligned(dk_acc, 16) || !aligned(dv_acc, 16))
     return FA_ERR_INVALID_ARG;
   if (workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
   if ((st = check_device()) != FA_OK) return st;
-  return bwd_main_d128(q, k, v, dO, workspace, nullptr, nullptr, B * H, N, scale, causal, (cudaStream_t)stream,
+  return bwd_main_dq(q, k, v, dO, workspace, nullptr, nullptr, B * H, N, d, scale, causal, (cudaStream_t)stream,
                        dk_acc, dv_acc);
 }
 
@@ -625,7 +613,6 @@ fa_status_t fa_bwd_finish(const void* workspace, size_t workspace_bytes, const f
   bool empty = false;
   fa_status_t st = check_shape(B, H, N, d, scale, 0, &empty);
   if (st != FA_OK || empty) return st;
-  if (d != 128) return FA_ERR_UNSUPPORTED;
   if (!workspace || !dk_acc || !dv_acc || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   if (!aligned(workspace, 256) || !aligned(dk_acc, 16) || !aligned(dv_acc, 16) || !aligned(dq, 16) ||
       !aligned(dk, 16) || !aligned(dv, 16))

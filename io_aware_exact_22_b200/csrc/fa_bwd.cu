@@ -120,7 +120,11 @@ struct BwdCfg {
   static constexpr int ST_BYTES = 2 * QT;
   static constexpr int DS_OFF = ST_OFF + NSQ * ST_BYTES;  // dS^T, two buffers of 128 x 64 bf16
   static constexpr int DS_BYTES = 128 * BQ * 2;
-  static constexpr int DQS_OFF = DS_OFF + 2 * DS_BYTES;   // dQ staging: 4 warps x [rows][32 d] fp32
+  // d = 64: 16 KB of zeros after the dS^T buffers, the rows d = 64..127 of the dQ^T MMA's A
+  // operand, so that dQ^T keeps M = 128 (its TMEM lanes 64..127 come out exactly 0)
+  static constexpr int Z_OFF = DS_OFF + 2 * DS_BYTES;
+  static constexpr int Z_BYTES = D == 64 ? 128 * 64 * 2 : 0;
+  static constexpr int DQS_OFF = Z_OFF + Z_BYTES;   // dQ staging: 4 warps x [rows][32 d] fp32
   static constexpr int DQS_WARP = (BQ - kBwdDqRedRows) * 32 * 4;
   static constexpr int LD_OFF = DQS_OFF + 4 * DQS_WARP;
   static constexpr int BAR_OFF = LD_OFF + NSQ * LDB;
@@ -165,8 +169,10 @@ struct BwdCfg {
 // computed, so dQ_n takes its columns, and dP_{n+1} goes to the other buffer as soon as the
 // drain has read dQ_{n-1} from it (without dQ: as soon as dS_{n-1} is computed), so it is
 // done before the compute warps need it instead of being issued after dS_n.
-// WITH_DQ = false: dK and dV only (dQ comes from fa_bwd_dq_kernel): no dQ^T MMA, no drain.  The dQ^T MMA puts d on the M dimension (128 TMEM lanes), so the
-// atomic dQ path exists for D = 128 only; D = 64 always runs with WITH_DQ = false.
+// WITH_DQ = false: dK and dV only (dQ comes from fa_bwd_dq_kernel): no dQ^T MMA, no drain.
+// The dQ^T MMA puts d on the M dimension, which is 128 TMEM lanes; at D = 64 its A operand
+// (K_j^T) is extended by 64 rows of zeros in shared memory, so rows 64..127 of dQ^T are 0 and
+// only the first two drain warps have anything to add.
 template <int D, bool WITH_DQ>
 __global__ void __launch_bounds__(480, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -175,7 +181,6 @@ __global__ void __launch_bounds__(480, 1)
                        const __grid_constant__ CUtensorMap tmdQ, const BwdArgs a, const int Tk,
                        const int Tq) {
   static_assert(D == 64 || D == 128, "head dimension");
-  static_assert(!WITH_DQ || D == 128, "the dQ^T MMA needs M = d = 128");
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -236,7 +241,7 @@ __global__ void __launch_bounds__(480, 1)
       mbar_init(p_ready(b), 256);
       mbar_init(ds_ready(b), 256);
       mbar_init(dq_full(b), 1);
-      mbar_init(dq_free(b), 128);
+      mbar_init(dq_free(b), D);  // the drain warps that hold dQ^T rows: one per 32 of d
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, 256);
@@ -252,6 +257,11 @@ __global__ void __launch_bounds__(480, 1)
   if (warp == 12) {
     tmem_alloc(sb + C::MISC_OFF, C::TMEM_COLS);
     tmem_relinquish();
+  }
+  if (C::Z_BYTES > 0) {
+    for (int i = threadIdx.x; i < C::Z_BYTES / 16; i += C::THREADS)
+      reinterpret_cast<uint4*>(gb + C::Z_OFF)[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();  // visible to the tensor core's reads
   }
   tc_fence_before();
   __syncthreads();
@@ -322,7 +332,8 @@ __global__ void __launch_bounds__(480, 1)
       // Base descriptors; each MMA adds its byte offset (see sdesc_add).
       const uint64_t dK_k = sdesc_sw128(sb + C::K_OFF, 16, 1024);        // K_j, K-major (S^T)
       const uint64_t dV_k = sdesc_sw128(sb + C::V_OFF, 16, 1024);        // V_j, K-major (dP^T)
-      const uint64_t dK_mn = sdesc_sw128(sb + C::K_OFF, 16384, 1024);    // K_j, MN-major (dQ^T)
+      // K_j, MN-major (dQ^T): rows d = 64..127 one leading-byte offset away (D = 64: the zeros)
+      const uint64_t dK_mn = sdesc_sw128(sb + C::K_OFF, D == 128 ? 16384 : C::Z_OFF - C::K_OFF, 1024);
       const uint64_t dQ_k = sdesc_sw128(sb + C::ST_OFF, 16, 1024);       // Q_i, K-major (S^T)
       const uint64_t dO_k = sdesc_sw128(sb + C::ST_OFF + C::QT, 16, 1024);  // dO_i, K-major (dP^T)
       const uint64_t dQ_mn = sdesc_sw128(sb + C::ST_OFF, 8192, 1024);    // Q_i, MN-major (dK)
@@ -507,7 +518,8 @@ __global__ void __launch_bounds__(480, 1)
     float* stage = reinterpret_cast<float*>(gb + C::DQS_OFF + wq * C::DQS_WARP);
     const uint32_t stage_s = sb + C::DQS_OFF + wq * C::DQS_WARP;
     bool ok = !*abort_flag;
-    for (int n = 0; n < (WITH_DQ ? count : 0) && ok; ++n) {
+    // rows d >= D of dQ^T are zero (D = 64): their warps have nothing to drain
+    for (int n = 0; n < (WITH_DQ && wq * 32 < D ? count : 0) && ok; ++n) {
       const int i = i0 + n;
       const int b = n & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(dq_full(b), (n >> 1) & 1, wc));
@@ -684,10 +696,9 @@ static cudaError_t launch_bwd_main_t(const CUtensorMap& tq, const CUtensorMap& t
 cudaError_t launch_bwd_main(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
                             const CUtensorMap& tdq, const BwdArgs& a, cudaStream_t stream, bool with_dq) {
-  if (d == 64) {
-    if (with_dq) return cudaErrorNotSupported;
-    return launch_bwd_main_t<64, false>(tq, tk, tv, tdo, tdk, tdv, tdq, a, stream);
-  }
+  if (d == 64)
+    return with_dq ? launch_bwd_main_t<64, true>(tq, tk, tv, tdo, tdk, tdv, tdq, a, stream)
+                   : launch_bwd_main_t<64, false>(tq, tk, tv, tdo, tdk, tdv, tdq, a, stream);
   if (d != 128) return cudaErrorNotSupported;
   return with_dq ? launch_bwd_main_t<128, true>(tq, tk, tv, tdo, tdk, tdv, tdq, a, stream)
                  : launch_bwd_main_t<128, false>(tq, tk, tv, tdo, tdk, tdv, tdq, a, stream);

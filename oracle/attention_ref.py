@@ -170,7 +170,7 @@ def attention_forward_fp8(q8, k8, v8, descale_q, descale_k, descale_v, scale: fl
 
 
 def attention_backward_head(q, k, v, do, scale: float, causal: bool, row_chunk: int = 4096,
-                            rows: np.ndarray | None = None):
+                            rows: np.ndarray | None = None, o=None):
     """Gradients of O = softmax(scale * Q K^T) V for one head, by plain calculus of the
     materialised forward (the pages only say the backward recomputes the scores from the
     saved inputs and a few statistics, [xinc] section 7):
@@ -184,12 +184,17 @@ def attention_backward_head(q, k, v, do, scale: float, causal: bool, row_chunk: 
     and dK are split into chunks of ``row_chunk`` rows only to bound memory.  ``rows``
     restricts the computation to the given query rows: dQ and D are then filled for those
     rows only and dK, dV hold those rows' contributions (used to time bounded samples).
+    ``o``, when given, is a stored forward output [N, d] (for instance the bf16 O a kernel
+    wrote): D_i is then rowsum(dO o O) of that O, which equals sum_j P_ij dP_ij when O = P V
+    exactly, so that the gradients are those of a backward that reads the saved output (the
+    pages' backward works from the saved inputs and statistics, [xinc] section 7).
     Returns (dQ, dK, dV, D).
     """
     q = _f64(q)
     k = _f64(k)
     v = _f64(v)
     do = _f64(do)
+    o = None if o is None else _f64(o)
     N = q.shape[0]
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
@@ -202,7 +207,7 @@ def attention_backward_head(q, k, v, do, scale: float, causal: bool, row_chunk: 
         p, _, _ = softmax_rows(s)
         dv += p.T @ do[r]
         dp = do[r] @ v.T
-        dvec[r] = (p * dp).sum(axis=-1)
+        dvec[r] = (p * dp).sum(axis=-1) if o is None else (do[r] * o[r]).sum(axis=-1)
         ds = p * (dp - dvec[r][:, None])
         dq[r] = scale * (ds @ k)
         dk += scale * (ds.T @ q[r])

@@ -81,11 +81,10 @@ def main():
                         total += check(f"splitkv{sp} " + tag, 0, BH, N, 128, 128, causal)
                 fa.backward(q, k, v, o, do, lse, causal, w.scale)
                 status_ok("bwd " + tag)
-                if d == 128:
-                    total += check("bwd key tiles " + tag, 1, BH, N, 64, 128, causal)
-                    fa.backward(q, k, v, o, do, lse, causal, w.scale, deterministic=True)
-                    status_ok("bwd deterministic " + tag)
-                # d = 64 always, d = 128 deterministic: key-tile pass then query-tile dQ pass
+                total += check("bwd key tiles " + tag, 1, BH, N, 64, 128, causal)
+                fa.backward(q, k, v, o, do, lse, causal, w.scale, deterministic=True)
+                status_ok("bwd deterministic " + tag)
+                # deterministic: key-tile pass, then query-tile dQ pass
                 buf = np.zeros(3 * BLOCK, dtype=np.int32)
                 assert fa.fa_debug_visits(buf, buf.size, False) == 0
                 for block, rq, rk in ((1, 64, 128), (2, 128, 64)):

@@ -138,7 +138,7 @@ def _bwd_main(**kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(q=0), INVALID), (dict(dO=0), INVALID), (dict(ws=0), INVALID), (dict(dv=0), INVALID),
     (dict(ws=A16 + 16), INVALID), (dict(dk=A16 + 8), INVALID), (dict(wsb=10), INVALID),
-    (dict(d=64), UNSUPPORTED), (dict(d=96), UNSUPPORTED), (dict(N=-1), INVALID),
+    (dict(d=32), UNSUPPORTED), (dict(d=96), UNSUPPORTED), (dict(N=-1), INVALID),
     (dict(scale=0.0), INVALID), (dict(causal=2), INVALID),
 ])
 def test_backward_main_rejects_bad_arguments(kw, code):
@@ -151,7 +151,7 @@ def test_backward_main_rejects_bad_arguments(kw, code):
     ((A16 + 16, 1 << 40, A16, 1, 1, 128, 128, 0.1), INVALID),
     ((A16, 1 << 40, A16 + 4, 1, 1, 128, 128, 0.1), INVALID),
     ((A16, 100, A16, 1, 1, 128, 128, 0.1), INVALID),
-    ((A16, 1 << 40, A16, 1, 1, 128, 64, 0.1), UNSUPPORTED),
+    ((A16, 1 << 40, A16, 1, 1, 128, 96, 0.1), UNSUPPORTED),
     ((A16, 1 << 40, A16, 1, 1, 128, 128, -1.0), INVALID),
     ((A16, 1 << 40, A16, 1, 1, 0, 128, 0.1), OK),
 ])

@@ -45,10 +45,11 @@ def _run(w, inputs=None, deterministic=True):
     grads = fa.backward(qd, kd, vd, o, dod, lse, w.causal, w.scale, deterministic=deterministic)
     torch.cuda.synchronize()
     assert fa.fa_get_device_status() == 0
+    _run.o = f64(o)
     return (q, k, v, do), grads
 
 
-def _check(w, heads=None, inputs=None, rel_tol=None):
+def _check(w, heads=None, inputs=None, rel_tol=None, given_o=False):
     (q, k, v, do), grads = _run(w, inputs)
     dq, dk, dv = (f64(g) for g in grads)
     if heads is None:
@@ -59,7 +60,8 @@ def _check(w, heads=None, inputs=None, rel_tol=None):
     for b, h in heads:
         gq, gk, gv, _ = oracle.attention_backward_head(to_f64(q[b, h]), to_f64(k[b, h]),
                                                        to_f64(v[b, h]), to_f64(do[b, h]),
-                                                       w.scale, w.causal)
+                                                       w.scale, w.causal,
+                                                       o=_run.o[b, h] if given_o else None)
         check_grad(dq[b, h], gq, f"dQ[{b},{h}]", **kw)
         check_grad(dk[b, h], gk, f"dK[{b},{h}]", **kw)
         check_grad(dv[b, h], gv, f"dV[{b},{h}]", **kw)
@@ -70,9 +72,11 @@ def _check(w, heads=None, inputs=None, rel_tol=None):
 @pytest.mark.gpu
 @pytest.mark.parametrize("N", [1, 2, 63, 64, 65, 127, 128, 129, 191, 255, 256, 257, 300, 513])
 @pytest.mark.parametrize("causal", [True, False])
-def test_ragged_lengths(cuda_ok, N, causal):
-    # N <= 4: see the matching case of the atomic backward for why 3e-2 bounds rel-L2 there
-    _check(custom(1, 2, N, 128, causal, seed=N, backward=True), rel_tol=3e-2 if N <= 4 else None)
+@pytest.mark.parametrize("d", [64, 128])
+def test_ragged_lengths(cuda_ok, N, causal, d):
+    # N <= 4: the reference takes D_i from the stored bf16 O (see the matching case of the
+    # atomic backward for why)
+    _check(custom(1, 2, N, d, causal, seed=N + d, backward=True), given_o=N <= 4)
 
 
 @pytest.mark.gpu
@@ -116,14 +120,12 @@ def test_zero_upstream_gradient(cuda_ok):
 
 
 # ---------------------------------------------------------------- head dimension 64
-# fa_bwd at d = 64 runs the same two passes (the key pass has no atomic dQ path there).
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("N", [1, 3, 64, 65, 127, 128, 129, 200, 257, 513])
 @pytest.mark.parametrize("causal", [True, False])
 def test_d64_ragged_lengths(cuda_ok, N, causal):
-    _check(custom(1, 2, N, 64, causal, seed=100 + N, backward=True),
-           rel_tol=3e-2 if N <= 4 else None)
+    _check(custom(1, 2, N, 64, causal, seed=100 + N, backward=True), given_o=N <= 4)
 
 
 @pytest.mark.gpu
@@ -145,10 +147,17 @@ def test_d64_multi_head_workload_sampled(cuda_ok):
 
 
 @pytest.mark.gpu
-def test_d64_fa_bwd_is_the_two_pass_path(cuda_ok):
-    w = custom(1, 3, 700, 64, True, seed=9, backward=True)
+@pytest.mark.parametrize("d", [64, 128])
+def test_one_pass_and_two_pass_agree(cuda_ok, d):
+    # Both paths accumulate dK and dV with the same MMAs in the same order, so those match bit
+    # for bit; dQ is the same fp32 sum taken in another order, so after rounding to bf16 the
+    # two differ by at most one unit in the last place of the larger, plus the reordering
+    # error of the fp32 sums (a few 2^-24 of the terms, below 2^-12 of the largest entry).
+    w = custom(1, 3, 700, d, True, seed=9, backward=True)
     inputs = make_inputs(w)
     _, gd = _run(w, inputs, deterministic=True)
     _, ga = _run(w, inputs, deterministic=False)
-    for a, b in zip(gd, ga):
-        assert torch.equal(a, b)
+    assert torch.equal(gd[1], ga[1]) and torch.equal(gd[2], ga[2])
+    a, b = ga[0].float(), gd[0].float()
+    ulp = torch.maximum(a.abs(), b.abs()) * 2.0 ** -7
+    assert bool(((a - b).abs() <= ulp + 2.0 ** -12 * b.abs().max()).all())

@@ -24,16 +24,20 @@ def _gpu(w, inputs=None):
     dq, dk, dv = fa.backward(qd, kd, vd, o, dod, lse, w.causal, w.scale)
     torch.cuda.synchronize()
     assert fa.fa_get_device_status() == 0
+    _gpu.o = f64(o)
     return (q, k, v, do), (f64(dq), f64(dk), f64(dv))
 
 
-def _check_heads(w, heads=None, inputs=None, rel_tol=None, term_bound=False):
+def _check_heads(w, heads=None, inputs=None, rel_tol=None, term_bound=False, given_o=False):
+    """given_o: the oracle's D_i = rowsum(dO o O) is taken from the bf16 O the forward stored
+    (the backward's own input) instead of the exact one."""
     (q, k, v, do), (dq, dk, dv) = _gpu(w, inputs)
     if heads is None:
         heads = [(b, h) for b in range(w.B) for h in range(w.H)]
     for b, h in heads:
         args = [to_f64(t[b, h]) for t in (q, k, v, do)]
-        gq, gk, gv, _ = oracle.attention_backward_head(*args, w.scale, w.causal)
+        gq, gk, gv, _ = oracle.attention_backward_head(*args, w.scale, w.causal,
+                                                       o=_gpu.o[b, h] if given_o else None)
         sums = abs_term_sums(*args, w.scale, w.causal) if term_bound else (None, None, None)
         kw = {}
         if rel_tol is not None:
@@ -47,22 +51,32 @@ def _check_heads(w, heads=None, inputs=None, rel_tol=None, term_bound=False):
 
 @pytest.mark.parametrize("N", [1, 2, 63, 64, 65, 127, 128, 129, 191, 192, 255, 256, 257, 300, 513])
 @pytest.mark.parametrize("causal", [True, False])
-def test_ragged_lengths(cuda_ok, N, causal):
+@pytest.mark.parametrize("d", [64, 128])
+def test_ragged_lengths(cuda_ok, N, causal, d):
     # With N <= 4 every row of dQ (and of dK) is a combination of at most four scalars
-    # dS_ij, so rel-L2 is the relative error of those few scalars; it is set by the bf16
-    # rounding of O inside D_i = rowsum(dO o O) (about 2^-9 ||dO|| ||O|| against |dP_ij - D_i|)
-    # and the bf16 rounding of dS, and is bounded by 3e-2 instead of 1e-2 there.
-    _check_heads(custom(1, 2, N, 128, causal, seed=N, backward=True),
-                 rel_tol=3e-2 if N <= 4 else None)
+    # dS_ij = P_ij (dP_ij - D_i) that nearly cancel (sum_j dS_ij = 0), so an error of 2^-9
+    # ||dO|| ||O|| in D_i from the bf16 rounding of the stored O can be most of a row's value
+    # (12.7 % of dQ at d = 64, N = 2, causal, this seed).  There the reference takes D_i from
+    # that same stored O, the backward's input, and the plain 1e-2 applies.
+    _check_heads(custom(1, 2, N, d, causal, seed=N + d, backward=True), given_o=N <= 4)
 
 
-@pytest.mark.parametrize("B,H,N,causal", [(2, 3, 700, True), (1, 4, 1100, False), (2, 2, 1536, True)])
-def test_multi_head_several_tiles(cuda_ok, B, H, N, causal):
-    _check_heads(custom(B, H, N, 128, causal, seed=13, backward=True))
+@pytest.mark.parametrize("B,H,N,causal,d", [(2, 3, 700, True, 128), (1, 4, 1100, False, 128),
+                                             (2, 2, 1536, True, 128), (2, 3, 1000, True, 64),
+                                             (4, 2, 1024, False, 64), (1, 2, 2049, True, 64)])
+def test_multi_head_several_tiles(cuda_ok, B, H, N, causal, d):
+    _check_heads(custom(B, H, N, d, causal, seed=13, backward=True))
 
 
-def test_large_scores(cuda_ok):
-    _check_heads(custom(1, 2, 1024, 128, True, seed=21, qk_std=math.sqrt(3.0), backward=True))
+@pytest.mark.parametrize("d", [64, 128])
+def test_large_scores(cuda_ok, d):
+    _check_heads(custom(1, 2, 1024, d, True, seed=21, qk_std=math.sqrt(3.0), backward=True))
+
+
+def test_d64_multi_head_workload_shape_sampled(cuda_ok):
+    # B=4, H=16, N=1024, d=64 non-causal (the multi-head forward workload's shape), four heads
+    w = custom(4, 16, 1024, 64, False, seed=0, backward=True)
+    _check_heads(w, heads=[(0, 0), (1, 7), (2, 9), (3, 15)])
 
 
 def test_backward_workload_full_size(cuda_ok):
@@ -103,9 +117,10 @@ def test_repeatable_up_to_atomic_order(cuda_ok):
     assert np.abs(dq1 - dq2).max() <= 2e-2
 
 
-def test_three_step_backward_equals_fa_bwd(cuda_ok):
+@pytest.mark.parametrize("d", [64, 128])
+def test_three_step_backward_equals_fa_bwd(cuda_ok, d):
     # fa_bwd_prepare, fa_bwd_main, fa_bwd_dq_post launch exactly fa_bwd's kernels
-    w = custom(2, 2, 777, 128, True, seed=17, backward=True)
+    w = custom(2, 2, 777, d, True, seed=17, backward=True)
     q, k, v, do = (t.cuda() for t in make_inputs(w))
     o, lse = fa.forward(q, k, v, True, w.scale)
     ref = fa.backward(q, k, v, o, do, lse, True, w.scale)

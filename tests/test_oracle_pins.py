@@ -255,6 +255,35 @@ def test_row_term_identity(causal):
     np.testing.assert_allclose(dvec, (do * o).sum(-1), atol=1e-12)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_given_output(causal):
+    # With the exact forward output, D_i from rowsum(dO * O) is the same number as
+    # rowsum(P * dP), so every gradient is unchanged.
+    n, d, scale = 40, 10, 0.35
+    q, k, v, do = _rand(n, d), _rand(n, d), _rand(n, d), _rand(n, d)
+    o, _ = ref.attention_forward_head(q, k, v, scale, causal)
+    a = ref.attention_backward_head(q, k, v, do, scale, causal)
+    b = ref.attention_backward_head(q, k, v, do, scale, causal, o=o)
+    for x, y in zip(a, b):
+        np.testing.assert_allclose(x, y, atol=1e-12)
+    # A change delta of one output row i moves D_i by rowsum(dO_i * delta) and nothing else:
+    # dS_i by -P_i times that, so dQ_i by -scale * that * (P_i K) and dK by -scale * that *
+    # P_i^T Q_i, while dV and every other row of dQ stay as they were.
+    i = 17
+    delta = np.zeros_like(o)
+    delta[i] = _rand(d) * 1e-3
+    c = ref.attention_backward_head(q, k, v, do, scale, causal, o=o + delta)
+    p, _, _ = ref.softmax_rows(ref.scaled_scores(q, k, scale, causal))
+    dd = float((do[i] * delta[i]).sum())
+    want_dq = a[0].copy()
+    want_dq[i] -= scale * dd * (p[i] @ k)
+    want_dk = a[1] - scale * dd * np.outer(p[i], q[i])
+    np.testing.assert_allclose(c[0], want_dq, atol=1e-12)
+    np.testing.assert_allclose(c[1], want_dk, atol=1e-12)
+    np.testing.assert_allclose(c[2], a[2], atol=1e-12)
+    np.testing.assert_allclose(c[3][i] - a[3][i], dd, atol=1e-12)
+
+
 def test_backward_row_chunking_is_the_same_computation():
     n, d = 90, 8
     q, k, v, do = _rand(n, d), _rand(n, d), _rand(n, d), _rand(n, d)

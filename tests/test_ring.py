@@ -167,18 +167,18 @@ def test_ring_round_trip_on_gloo_ranks(world):
 
 
 @pytest.mark.parametrize("fn", ["prepare", "accumulate", "finish"])
-def test_backward_pieces_reject_d64_and_null(fn):
+def test_backward_pieces_reject_other_d_and_null(fn):
     a = A16
     if fn == "prepare":
-        assert fa.fa_bwd_prepare(a, a, a, a, 1 << 30, 1, 2, 256, 64, 0) == UNSUPPORTED
+        assert fa.fa_bwd_prepare(a, a, a, a, 1 << 30, 1, 2, 256, 96, 0) == UNSUPPORTED
         assert fa.fa_bwd_prepare(0, a, a, a, 1 << 30, 1, 2, 256, 128, 0) == INVALID
         assert fa.fa_bwd_prepare(a, a, a, a, 10, 1, 2, 256, 128, 0) == INVALID
     elif fn == "accumulate":
-        assert fa.fa_bwd_accumulate(a, a, a, a, a, 1 << 30, a, a, 1, 2, 256, 64, 0.1, 0, 0) == UNSUPPORTED
+        assert fa.fa_bwd_accumulate(a, a, a, a, a, 1 << 30, a, a, 1, 2, 256, 96, 0.1, 0, 0) == UNSUPPORTED
         assert fa.fa_bwd_accumulate(a, a, a, a, a, 1 << 30, 0, a, 1, 2, 256, 128, 0.1, 0, 0) == INVALID
         assert fa.fa_bwd_accumulate(a, a, a, a, a, 1 << 30, a + 4, a, 1, 2, 256, 128, 0.1, 0, 0) == INVALID
     else:
-        assert fa.fa_bwd_finish(a, 1 << 30, a, a, a, a, a, 1, 2, 256, 64, 0.1, 0) == UNSUPPORTED
+        assert fa.fa_bwd_finish(a, 1 << 30, a, a, a, a, a, 1, 2, 256, 96, 0.1, 0) == UNSUPPORTED
         assert fa.fa_bwd_finish(a, 1 << 30, a, a, 0, a, a, 1, 2, 256, 128, 0.1, 0) == INVALID
 
 
