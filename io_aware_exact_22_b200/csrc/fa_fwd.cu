@@ -26,6 +26,8 @@
 // tile's chain per block is its softmax alone rather than S MMA + softmax + PV MMA.
 #include "fa_debug.cuh"
 #include "fa_internal.cuh"
+
+#include <algorithm>
 #include "sm100_ptx.cuh"
 
 #include <cmath>
@@ -54,15 +56,17 @@ struct FwdCfg {
   static constexpr int KSTEP = 32 / EB;            // elements of K per MMA (32 bytes)
   static constexpr int PTILE = 128 * 128 * EB;     // bytes of one P tile (128 rows x 128 keys)
   static constexpr int OTILE = 128 * D * 2;        // bytes of one 128-row bf16 output tile
-  // O staging: the dead Q tiles (bf16) or the idle K/V ring (FP8: Q tiles are half as large)
-  static constexpr int OST_OFF = FP8 ? 2 * TILE : 0;
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = 2 * TILE;
   static constexpr int P_OFF = KV_OFF + NS * TILE;  // ring and P tiles together stage partial outputs
   static constexpr int BAR_OFF = P_OFF + 2 * PTILE;
-  // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], s_free[2], p_full[2], pv_done[2], o_full,
-  // s_done
-  static constexpr int NBAR = 1 + 2 * NS + 8 + 2;
+  // O staging, tile t at OST_OFF + t * OST_STRIDE: the dead P tile (bf16; the Q tiles may
+  // already hold the next item's queries) or the idle K/V ring (FP8, one item per CTA)
+  static constexpr int OST_OFF = FP8 ? KV_OFF : P_OFF;
+  static constexpr int OST_STRIDE = FP8 ? OTILE : PTILE;
+  // barriers: q_full, q_empty, kv_full[NS], kv_empty[NS], s_full[2], s_free[2], p_full[2],
+  // pv_done[2], o_full[2], o_free[2], s_done, pv_end
+  static constexpr int NBAR = 2 + 2 * NS + 12 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM = MISC_OFF + 16 + 1024;  // + slack to align the base to 1024
   static constexpr int THREADS = 352;
@@ -80,6 +84,17 @@ struct FwdCfg {
 
 // PARTIAL: the CTA covers only its split's range of key blocks and writes the normalised
 // partial output O_s (fp32) and its LSE_s, to be combined by fa_fwd_merge_kernel.
+//
+// Work list.  An item is (head bh, block of 256 query rows, key split).  With a.persistent = 0
+// every CTA takes one item, in the grouped heaviest-first order (heads in groups of a.group;
+// within a group every head's heaviest query block first: group 1 keeps a head's blocks
+// together, so its K/V stays in L2, group BH gives the shortest causal tail), and the
+// hardware hands the next CTA to the first SM that frees up.  With a.persistent = 1 (whole key
+// range, bf16) a grid of at most one CTA per SM walks the list itself: each head's query
+// blocks in the order heaviest, lightest, second heaviest, second lightest, ..., so that under
+// the causal mask consecutive pairs cost the same, and CTA c takes pairs c, c + grid, ...;
+// the next item's Q load and first score products then overlap the current item's last
+// blocks and output, and the CTA's setup is paid once.
 template <int D, bool PARTIAL, bool FP8 = false>
 __global__ void __launch_bounds__(352, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -87,54 +102,79 @@ __global__ void __launch_bounds__(352, 1)
                   const FwdArgs a) {
   static_assert(!FP8 || (D == 128 && !PARTIAL), "FP8: d = 128, whole key range");
   using C = FwdCfg<D, FP8>;
+  constexpr bool kOutInP = !PARTIAL && !FP8;  // the output is staged in the tile's own P tile
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
   uint8_t* gb = smem_raw + (sb - raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // ---- work item: (head bh, block of 256 query rows, key split).  Heads go in groups of
-  // a.group, and within a group every head's heaviest query block goes first: group 1 keeps a
-  // head's blocks together (its K/V stays in L2), group BH gives the shortest causal tail.
-  const int split = blockIdx.x % a.nsplit;
-  const int item = blockIdx.x / a.nsplit;
-  const int per_group = a.group * a.nqb;
-  const int g0 = item / per_group * a.group;  // first head of the group
-  const int gn = min(a.group, a.BH - g0);     // heads in the group (the last may be short)
-  const int r = item - item / per_group * per_group;
-  const int bh = g0 + r % gn;
-  const int qb = a.nqb - 1 - r / gn;
-  const int q0 = qb * 256;
   const int Tk = (a.N + 127) >> 7;
-  const bool has1 = (q0 + 128) < a.N;
-  // visible key blocks of each query tile, over the whole key range
-  const int n0g = a.causal ? min(Tk, 2 * qb + 1) : Tk;
-  const int n1g = has1 ? (a.causal ? min(Tk, 2 * qb + 2) : Tk) : 0;
-  // this split's contiguous share [kb0, kb1) of the key blocks, and each tile's count in it
-  const int nmaxg = max(n0g, n1g);
-  const int kb0 = (int)((long long)split * nmaxg / a.nsplit);
-  const int kb1 = (int)((long long)(split + 1) * nmaxg / a.nsplit);
-  const int n0 = max(0, min(kb1, n0g) - kb0);
-  const int n1 = max(0, min(kb1, n1g) - kb0);
-  const int nmax = max(n0, n1);
+  const int total = a.BH * a.nqb * a.nsplit;  // items (the host checks that this fits an int)
+  // list index of this CTA's k-th item, or -1 past its last
+  auto item_at = [&](int k) -> int {
+    if (!a.persistent) return k == 0 ? (int)blockIdx.x : -1;
+    const long long idx = 2 * ((long long)blockIdx.x + (long long)(k >> 1) * gridDim.x) + (k & 1);
+    return idx < total ? (int)idx : -1;
+  };
+  struct Item {
+    int bh, qb, split, q0, kb0, n0, n1, nmax, n0g, n1g;
+    bool has1;
+  };
+  auto decode = [&](int idx) -> Item {
+    Item w;
+    if (a.persistent) {
+      w.split = 0;
+      w.bh = idx / a.nqb;
+      const int p = idx - w.bh * a.nqb;
+      w.qb = (p & 1) ? (p >> 1) : a.nqb - 1 - (p >> 1);
+    } else {
+      w.split = idx % a.nsplit;
+      const int item = idx / a.nsplit;
+      const int per_group = a.group * a.nqb;
+      const int g0 = item / per_group * a.group;  // first head of the group
+      const int gn = min(a.group, a.BH - g0);     // heads in the group (the last may be short)
+      const int r = item - item / per_group * per_group;
+      w.bh = g0 + r % gn;
+      w.qb = a.nqb - 1 - r / gn;
+    }
+    w.q0 = w.qb * 256;
+    w.has1 = (w.q0 + 128) < a.N;
+    // visible key blocks of each query tile, over the whole key range
+    w.n0g = a.causal ? min(Tk, 2 * w.qb + 1) : Tk;
+    w.n1g = w.has1 ? (a.causal ? min(Tk, 2 * w.qb + 2) : Tk) : 0;
+    // this split's contiguous share [kb0, kb1) of the key blocks, and each tile's count in it
+    const int nmaxg = max(w.n0g, w.n1g);
+    w.kb0 = (int)((long long)w.split * nmaxg / a.nsplit);
+    const int kb1 = (int)((long long)(w.split + 1) * nmaxg / a.nsplit);
+    w.n0 = max(0, min(kb1, w.n0g) - w.kb0);
+    w.n1 = max(0, min(kb1, w.n1g) - w.kb0);
+    w.nmax = max(w.n0, w.n1);
+    FA_DBG(if (!dbg_check(w.bh < a.BH && w.qb >= 0 && w.qb < a.nqb && w.split < a.nsplit && kb1 <= Tk, a.status))
+               *reinterpret_cast<volatile int*>(gb + C::MISC_OFF + 4) = 1;)
+    return w;
+  };
 
   const uint32_t bar = sb + C::BAR_OFF;
-  const uint32_t q_full = bar;
-  auto kv_full = [&](int s) { return bar + 8u * (1 + s); };
-  auto kv_empty = [&](int s) { return bar + 8u * (1 + C::NS + s); };
-  auto s_full = [&](int t) { return bar + 8u * (1 + 2 * C::NS + t); };   // S_t computed
-  auto s_free = [&](int t) { return bar + 8u * (3 + 2 * C::NS + t); };   // S_t loaded by its softmax
-  auto p_full = [&](int t) { return bar + 8u * (5 + 2 * C::NS + t); };   // P_t written
-  auto pv_done = [&](int t) { return bar + 8u * (7 + 2 * C::NS + t); };  // P_t V_j added into O_t
-  const uint32_t o_full = bar + 8u * (9 + 2 * C::NS);
-  const uint32_t s_done = bar + 8u * (10 + 2 * C::NS);  // every score product issued has completed
+  const uint32_t q_full = bar;                                               // Q tiles landed
+  const uint32_t q_empty = bar + 8u;                                         // Q tiles read by every S
+  auto kv_full = [&](int s) { return bar + 8u * (2 + s); };
+  auto kv_empty = [&](int s) { return bar + 8u * (2 + C::NS + s); };
+  auto s_full = [&](int t) { return bar + 8u * (2 + 2 * C::NS + t); };    // S_t computed
+  auto s_free = [&](int t) { return bar + 8u * (4 + 2 * C::NS + t); };    // S_t loaded by its softmax
+  auto p_full = [&](int t) { return bar + 8u * (6 + 2 * C::NS + t); };    // P_t written
+  auto pv_done = [&](int t) { return bar + 8u * (8 + 2 * C::NS + t); };   // P_t V_j added into O_t
+  auto o_full = [&](int t) { return bar + 8u * (10 + 2 * C::NS + t); };   // O_t of the item complete
+  auto o_free = [&](int t) { return bar + 8u * (12 + 2 * C::NS + t); };   // O_t read by the epilogue
+  const uint32_t s_done = bar + 8u * (14 + 2 * C::NS);  // every score product issued has completed
+  const uint32_t pv_end = bar + 8u * (15 + 2 * C::NS);  // every P V product issued has completed
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gb + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + C::MISC_OFF + 4);
   const WaitCtx wc{abort_flag, a.status};
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(kv_full(s), 1);
       mbar_init(kv_empty(s), 1);
@@ -144,9 +184,11 @@ __global__ void __launch_bounds__(352, 1)
       mbar_init(s_free(t), 128);
       mbar_init(p_full(t), 128);
       mbar_init(pv_done(t), 1);
+      mbar_init(o_full(t), 1);
+      mbar_init(o_free(t), 128);
     }
-    mbar_init(o_full, 1);
     mbar_init(s_done, 1);
+    mbar_init(pv_end, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -163,51 +205,60 @@ __global__ void __launch_bounds__(352, 1)
     *abort_flag = 1;
   }
   const uint32_t tmem = 0u;
-  FA_DBG(if (!(bh < a.BH && qb >= 0 && qb < a.nqb && split < a.nsplit && kb1 <= Tk)) {
-    if (threadIdx.x == 0) atomicOr(a.status, FA_DEV_BOUNDS);
-    *abort_flag = 1;
-  })
+  // ring positions within an item of nmax blocks: K_0 first, then K_{j+1} (when there is
+  // one) before V_j; every item takes 2 nmax consecutive positions
+  auto pos_k = [](int j) { return j == 0 ? 0 : 2 * j - 1; };
+  auto pos_v = [](int j, int nmax) { return j + 1 < nmax ? 2 * j + 2 : 2 * j + 1; };
 
   if (warp == 9) {
     // ------------------------------------------------------------ TMA producer (whole warp)
-    if (!*abort_flag && nmax > 0) {
+    if (!*abort_flag) {
       if (elect_one()) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
       }
       const uint64_t keep = policy_evict_last();
-      const int nq = has1 ? 2 : 1;
-      mbar_arrive_expect_tx_e(q_full, nq * C::TILE);
-      for (int t = 0; t < nq; ++t)
-        for (int b = 0; b < C::NBOX; ++b)
-          tma_load_3d_e(sb + C::Q_OFF + t * C::TILE + b * 16384, &tmQ, q_full, C::BOXW * b, q0 + 128 * t,
-                        bh, keep);
-      // ring order: K_0, then K_{j+1} (when there is one) before V_j
-      int it = 0;
+      int it = 0;  // ring position over all items
+      int ni = 0;  // items whose Q tiles were loaded
       bool ok = true;
-      auto load = [&](const CUtensorMap* m, int j) {
-        const int s = it % C::NS;
-        const uint32_t ph = (it / C::NS) & 1;
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(kv_empty(s), ph ^ 1, wc)))) return;
-        FA_DBG(if (!dbg_check(kb0 + j >= 0 && 128 * (kb0 + j) < a.N, a.status)) {
-          *abort_flag = 1;
-          ok = false;
-          return;
-        })
-        mbar_arrive_expect_tx_e(kv_full(s), C::TILE);
-        for (int b = 0; b < C::NBOX; ++b)
-          tma_load_3d_e(sb + C::KV_OFF + s * C::TILE + b * 16384, m, kv_full(s), C::BOXW * b, 128 * (kb0 + j),
-                        bh, keep);
-        ++it;
-      };
-      load(&tmK, 0);
-      for (int j = 0; j < nmax && ok; ++j) {
-        if (j + 1 < nmax) load(&tmK, j + 1);
-        if (ok) load(&tmV, j);
+      for (int k = 0; ok; ++k) {
+        const int idx = item_at(k);
+        if (idx < 0) break;
+        const Item w = decode(idx);
+        if (w.nmax == 0) continue;
+        // the Q tiles are reused once every score product of the previous item has completed
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(q_empty, (ni & 1) ^ 1, wc)))) break;
+        const int nq = w.has1 ? 2 : 1;
+        mbar_arrive_expect_tx_e(q_full, nq * C::TILE);
+        for (int t = 0; t < nq; ++t)
+          for (int b = 0; b < C::NBOX; ++b)
+            tma_load_3d_e(sb + C::Q_OFF + t * C::TILE + b * 16384, &tmQ, q_full, C::BOXW * b, w.q0 + 128 * t,
+                          w.bh, keep);
+        ++ni;
+        auto load = [&](const CUtensorMap* m, int j) {
+          const int s = it % C::NS;
+          const uint32_t ph = (it / C::NS) & 1;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(kv_empty(s), ph ^ 1, wc)))) return;
+          FA_DBG(if (!dbg_check(w.kb0 + j >= 0 && 128 * (w.kb0 + j) < a.N, a.status)) {
+            *abort_flag = 1;
+            ok = false;
+            return;
+          })
+          mbar_arrive_expect_tx_e(kv_full(s), C::TILE);
+          for (int b = 0; b < C::NBOX; ++b)
+            tma_load_3d_e(sb + C::KV_OFF + s * C::TILE + b * 16384, m, kv_full(s), C::BOXW * b,
+                          128 * (w.kb0 + j), w.bh, keep);
+          ++it;
+        };
+        load(&tmK, 0);
+        for (int j = 0; j < w.nmax && ok; ++j) {
+          if (j + 1 < w.nmax) load(&tmK, j + 1);
+          if (ok) load(&tmV, j);
+        }
       }
       if (!ok) {  // let copies already issued land before the CTA exits
-        mbar_wait_drain(q_full, 0);
+        if (ni > 0) mbar_wait_drain(q_full, (ni - 1) & 1);
         for (int back = 1; back <= C::NS && it - back >= 0; ++back) {
           const int i2 = it - back;
           mbar_wait_drain(kv_full(i2 % C::NS), (i2 / C::NS) & 1);
@@ -217,25 +268,22 @@ __global__ void __launch_bounds__(352, 1)
     __syncwarp();
   } else if (warp == 8 || warp == 10) {
     // ------------------------------------------------------------ MMA issuers (whole warps)
-    if (!*abort_flag && nmax > 0) {
-      const int nt[2] = {n0, n1};
+    if (!*abort_flag) {
       // Base descriptors; each MMA adds its byte offset (see sdesc_add).
       const uint64_t dQ_k = sdesc_sw128(sb + C::Q_OFF, 16, 1024);       // Q tiles, K-major
       const uint64_t dK_k = sdesc_sw128(sb + C::KV_OFF, 16, 1024);      // K stages, K-major
       const uint64_t dV_mn = sdesc_sw128(sb + C::KV_OFF, 16384, 1024);  // V stages, MN-major
       const uint64_t dP_k = sdesc_sw128(sb + C::P_OFF, 16, 1024);       // P tiles, K-major
-      // ring positions: K_0 first, then K_{j+1} (when there is one) before V_j
-      auto pos_k = [&](int j) { return j == 0 ? 0 : 2 * j - 1; };
-      auto pos_v = [&](int j) { return j + 1 < nmax ? 2 * j + 2 : 2 * j + 1; };
       auto stage_addr = [&](int it) { return (uint32_t)((it % C::NS) * C::TILE); };
       auto stage_par = [&](int it) { return (uint32_t)((it / C::NS) & 1); };
       auto wait_stage = [&](int it) {
         return __all_sync(0xffffffffu, mbar_wait(kv_full(it % C::NS), stage_par(it), wc));
       };
       bool ok = true;
+      int ibase = 0;  // ring position of the item's first load
       if (warp == 8) {
-        // S_t for block j, each as soon as K_j has landed and tile t's softmax has loaded S_t of
-        // block j-1
+        // S_t for block j, each as soon as K_j has landed and tile t's softmax has loaded the
+        // previous S_t (of this item or the one before)
         auto issue_qk = [&](uint32_t dst, uint32_t qoff, uint32_t koff) {
 #pragma unroll
           for (int k = 0; k < D / C::KSTEP; ++k) {  // 32 bytes of d per MMA
@@ -246,25 +294,40 @@ __global__ void __launch_bounds__(352, 1)
               mma_ss_e(dst, sdesc_add(dQ_k, qoff + off), sdesc_add(dK_k, koff + off), C::IDESC_QK, k > 0);
           }
         };
-        ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, wc));
-        for (int j = 0; j < nmax && ok; ++j) {
-          const int itK = pos_k(j);
-          if (!(ok = wait_stage(itK))) break;
+        int ni = 0;               // items issued
+        int cs[2] = {0, 0};       // S_t products issued, over all items
+        for (int kk = 0; ok; ++kk) {
+          const int idx = item_at(kk);
+          if (idx < 0) break;
+          const Item w = decode(idx);
+          if (w.nmax == 0) continue;
+          const int nt[2] = {w.n0, w.n1};
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(q_full, ni & 1, wc)))) break;
+          for (int j = 0; j < w.nmax && ok; ++j) {
+            const int itK = ibase + pos_k(j);
+            if (!(ok = wait_stage(itK))) break;
 #pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            if (j >= nt[t]) continue;
-            if (j > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(s_free(t), (j - 1) & 1, wc)))) break;
-            tc_fence_after();
-            issue_qk(t ? C::T_S1 : C::T_S0, (uint32_t)(t * C::TILE), stage_addr(itK));
-            mma_commit_e(s_full(t));
+            for (int t = 0; t < 2; ++t) {
+              if (j >= nt[t]) continue;
+              if (cs[t] > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(s_free(t), (cs[t] - 1) & 1, wc)))) break;
+              tc_fence_after();
+              issue_qk(t ? C::T_S1 : C::T_S0, (uint32_t)(t * C::TILE), stage_addr(itK));
+              mma_commit_e(s_full(t));
+              ++cs[t];
+            }
+            if (!ok) break;
+            mma_commit_e(kv_empty(itK % C::NS));
           }
           if (!ok) break;
-          mma_commit_e(kv_empty(itK % C::NS));
+          mma_commit_e(q_empty);  // the Q tiles are free once these products have completed
+          ibase += 2 * w.nmax;
+          ++ni;
         }
         mma_commit_e(s_done);
         if (!ok) mbar_wait_drain(s_done, 0);  // every issued MMA has completed before TMEM is freed
       } else {
-        // O_t += P_t V_j, each as soon as V_j has landed and tile t's softmax has written P_t
+        // O_t += P_t V_j, each as soon as V_j has landed and tile t's softmax has written P_t; the
+        // first of an item also after the epilogue has read the previous item's O_t
         auto issue_pv = [&](uint32_t dst, uint32_t poff, uint32_t voff, bool acc) {
 #pragma unroll
           for (int k = 0; k < 128 / C::KSTEP; ++k) {  // KSTEP keys (32 bytes of P) per MMA
@@ -276,22 +339,52 @@ __global__ void __launch_bounds__(352, 1)
               mma_ss_e(dst, sdesc_add(dP_k, po), sdesc_add(dV_mn, vo), C::IDESC_PV, (acc || k > 0) ? 1u : 0u);
           }
         };
-        for (int j = 0; j < nmax && ok; ++j) {
-          const int itV = pos_v(j);
-          if (!(ok = wait_stage(itV))) break;
+        int cp[2] = {0, 0};  // P_t consumed, over all items
+        int co[2] = {0, 0};  // items whose O_t was completed
+        for (int kk = 0; ok; ++kk) {
+          const int idx = item_at(kk);
+          if (idx < 0) break;
+          const Item w = decode(idx);
+          if (w.nmax == 0) continue;
+          const int nt[2] = {w.n0, w.n1};
+          for (int j = 0; j < w.nmax && ok; ++j) {
+            const int itV = ibase + pos_v(j, w.nmax);
+            if (!(ok = wait_stage(itV))) break;
 #pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            if (j >= nt[t]) continue;
-            if (!(ok = __all_sync(0xffffffffu, mbar_wait(p_full(t), j & 1, wc)))) break;
-            tc_fence_after();
-            issue_pv(t ? C::T_O1 : C::T_O0, (uint32_t)(t * C::PTILE), stage_addr(itV), j > 0);
-            mma_commit_e(pv_done(t));
+            for (int t = 0; t < 2; ++t) {
+              if (j >= nt[t]) continue;
+              if (j == 0 && co[t] > 0 &&
+                  !(ok = __all_sync(0xffffffffu, mbar_wait(o_free(t), (co[t] - 1) & 1, wc))))
+                break;
+              if (!(ok = __all_sync(0xffffffffu, mbar_wait(p_full(t), cp[t] & 1, wc)))) break;
+              tc_fence_after();
+              issue_pv(t ? C::T_O1 : C::T_O0, (uint32_t)(t * C::PTILE), stage_addr(itV), j > 0);
+              mma_commit_e(pv_done(t));
+              ++cp[t];
+              // bf16, whole key range: O_t of this item is complete once this product is (its
+              // output is staged in P_t, which no other product reads).  Split and FP8 outputs
+              // are staged in the K/V ring, idle only once every product of the item is done.
+              if (kOutInP && j == nt[t] - 1) {
+                mma_commit_e(o_full(t));
+                ++co[t];
+              }
+            }
+            if (!ok) break;
+            mma_commit_e(kv_empty(itV % C::NS));
           }
           if (!ok) break;
-          mma_commit_e(kv_empty(itV % C::NS));
+          if (!kOutInP) {
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+              if (nt[t] > 0) {
+                mma_commit_e(o_full(t));
+                ++co[t];
+              }
+          }
+          ibase += 2 * w.nmax;
         }
-        mma_commit_e(o_full);
-        if (!ok) mbar_wait_drain(o_full, 0);  // every issued MMA has completed before TMEM is freed
+        mma_commit_e(pv_end);
+        if (!ok) mbar_wait_drain(pv_end, 0);  // every issued MMA has completed before TMEM is freed
       }
     }
     __syncwarp();
@@ -300,12 +393,29 @@ __global__ void __launch_bounds__(352, 1)
     const int t = warp >> 2;
     const int wq = warp & 3;
     const int r = wq * 32 + lane;  // row within the query tile == TMEM lane
-    const int ntile = t ? n1 : n0;      // blocks of this split
-    const int ntile_g = t ? n1g : n0g;  // blocks of the whole key range
-    const int qrow = q0 + 128 * t + r;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tSrow = tmem + lane_off + 128u * t;
     const uint32_t tOrow = tmem + lane_off + 256u + (uint32_t)(D * t);
+    bool ok = !*abort_flag;
+    bool store_pending = false;  // this warp's O store may still be reading the P_t rows
+    int ns = 0;  // S_t blocks consumed, over all items (s_full phases)
+    int np = 0;  // P_t blocks written, over all items (pv_done phases)
+    int no = 0;  // items whose O_t this warpgroup wrote out (o_full phases)
+    for (int kk = 0; ok; ++kk) {
+    const int idx = item_at(kk);
+    if (idx < 0) break;
+    const Item wk = decode(idx);
+    const int bh = wk.bh, qb = wk.qb, split = wk.split, kb0 = wk.kb0;
+    (void)qb;
+    (void)split;
+    const int ntile = t ? wk.n1 : wk.n0;      // blocks of this split
+    const int ntile_g = t ? wk.n1g : wk.n0g;  // blocks of the whole key range
+    const int qrow = wk.q0 + 128 * t + r;
+    if (wk.nmax == 0 || ntile == 0) {
+      // this split holds no key block of this tile: an empty partial (weight 0 in the merge)
+      if (PARTIAL && qrow < a.N) a.lse[((size_t)split * a.BH + bh) * a.N + qrow] = -INFINITY;
+      continue;
+    }
     float cs = a.scale_log2;
     float vmul = 1.f;  // FP8: V's dequantisation factor, applied to O at the end
     if constexpr (FP8) {
@@ -315,10 +425,10 @@ __global__ void __launch_bounds__(352, 1)
     }
     float m_ref = -INFINITY;  // reference max, base-2 scaled units
     float l = 0.f;
-    bool ok = !*abort_flag;
 
     for (int j = 0; j < ntile && ok; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full(t), j & 1, wc));
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full(t), ns & 1, wc));
+      ++ns;
       if (!ok) break;
       tc_fence_after();
       uint32_t sr[128];
@@ -420,11 +530,16 @@ __global__ void __launch_bounds__(352, 1)
       l *= alpha;
       // P_t V_{j-1} must have been added into O_t before P_t is rewritten or O_t rescaled
       if (j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(pv_done(t), (j - 1) & 1, wc));
+        ok = __all_sync(0xffffffffu, mbar_wait(pv_done(t), (np - 1) & 1, wc));
         if (!ok) break;
       }
       float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
       if constexpr (FP8) mneg += C::P_SHIFT;
+      if (store_pending) {  // the previous item's O store has read this warp's rows of P_t
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+        store_pending = false;
+      }
       float rsum;
       if (!edge) {
         rsum = exp_full(mneg);
@@ -475,21 +590,21 @@ __global__ void __launch_bounds__(352, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(p_full(t));
+      ++np;
     }
 
-    if (PARTIAL && ntile == 0 && ok) {
-      // this split holds no key block of this tile: an empty partial (weight 0 in the merge)
-      if (qrow < a.N) a.lse[((size_t)split * a.BH + bh) * a.N + qrow] = -INFINITY;
-    } else if (ntile > 0 && ok) {
+    if (ok) {
       // ---------------------------------------------------------- epilogue
-      ok = __all_sync(0xffffffffu, mbar_wait(o_full, 0, wc));
+      ok = __all_sync(0xffffffffu, mbar_wait(o_full(t), no & 1, wc));
+      ++no;
       if (ok) {
         tc_fence_after();
         const float inv = (l > 0.f) ? vmul / l : 0.f;
-        const int row0 = q0 + 128 * t + 32 * wq;
+        const int row0 = wk.q0 + 128 * t + 32 * wq;
         if (!PARTIAL) {
-          // Q_t (bf16) or the K/V ring (FP8) is dead once o_full has fired
-          uint8_t* stage = gb + C::OST_OFF + t * C::OTILE;
+          // P_t (bf16) or the K/V ring (FP8) is dead once o_full has fired; each warp stages
+          // and stores its own 32 rows, the rows whose P it writes
+          uint8_t* stage = gb + C::OST_OFF + t * C::OST_STRIDE;
 #pragma unroll
           for (int b = 0; b < D / 64; ++b) {
 #pragma unroll
@@ -510,15 +625,17 @@ __global__ void __launch_bounds__(352, 1)
               }
             }
           }
+          tc_fence_before();
+          mbar_arrive(o_free(t));  // O_t is read: the next item's first P V may overwrite it
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0 && row0 < a.N) {
             for (int b = 0; b < D / 64; ++b)
-              tma_store_3d(&tmO, sb + C::OST_OFF + t * C::OTILE + b * 16384 + wq * 4096, 64 * b, row0, bh);
+              tma_store_3d(&tmO, sb + C::OST_OFF + t * C::OST_STRIDE + b * 16384 + wq * 4096, 64 * b, row0, bh);
             bulk_commit();
-            bulk_wait_read0();
           }
           __syncwarp();
+          store_pending = true;  // waited for before this warp next writes P_t, or at exit
           if (qrow < a.N)
             a.lse[(size_t)bh * a.N + qrow] =
                 (l > 0.f) ? (m_ref - C::P_SHIFT + log2f(l)) * 0.69314718055994530942f : -INFINITY;
@@ -541,6 +658,8 @@ __global__ void __launch_bounds__(352, 1)
               *reinterpret_cast<float4*>(stage + b * 16384 + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
             }
           }
+          tc_fence_before();
+          mbar_arrive(o_free(t));
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0 && row0 < a.N) {
@@ -556,6 +675,9 @@ __global__ void __launch_bounds__(352, 1)
         }
       }
     }
+    }  // items
+    if (lane == 0) bulk_wait0();  // every O store has completed before the CTA exits
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -573,7 +695,8 @@ static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, co
   static_assert(C::SMEM <= 232448, "shared memory budget");
   static_assert(C::SMEM > 116 * 1024, "one CTA per SM: each allocates all 512 TMEM columns");
   static_assert(2 * 128 * D * 4 <= C::NS * C::TILE + 2 * C::PTILE, "partial-output staging must fit the ring and P");
-  static_assert(C::OST_OFF + 2 * C::OTILE <= C::BAR_OFF, "output staging must fit");
+  static_assert(C::OTILE <= C::OST_STRIDE && C::OST_OFF + C::OST_STRIDE + C::OTILE <= C::BAR_OFF,
+                "output staging must fit");
   static bool attr_set[64];  // per device: the attribute outlives the call
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -583,8 +706,29 @@ static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, co
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  const long long grid = (long long)a.BH * a.nqb * a.nsplit;
+  const long long items = (long long)a.BH * a.nqb * a.nsplit;
+  if (items > INT_MAX) return cudaErrorInvalidValue;
   FwdArgs b = a;
+  long long grid = items;
+  b.persistent = 0;
+  if (!PARTIAL && !FP8) {
+    // The whole key range in bf16: at most one CTA per SM, each walking its pairs of items,
+    // when the items are of equal length (no mask) or many per SM.  Under the causal mask with
+    // few items per SM the hardware's dispatch of one CTA per item (to whichever SM frees up
+    // first) balances the uneven items better.  Measured on B200: persistent is 1-3 % faster
+    // at B=1 H=32 N=16384 causal (13.8 items per SM) and 6 % at B=4 H=16 N=1024 without mask,
+    // 17 % slower at B=2 H=16 N=4096 causal (3.5 items per SM).
+    static int sms[64];
+    if (dev >= 0 && dev < 64 && sms[dev] == 0) {
+      e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return e;
+    }
+    const long long nsm = (dev >= 0 && dev < 64 && sms[dev] > 0) ? sms[dev] : 148;
+    if (!a.causal || items >= 8 * nsm) {
+      b.persistent = 1;
+      grid = std::min((items + 1) / 2, nsm);
+    }
+  }
   FA_DBG(b.visits = debug_visits(0); b.visits_cap = kDebugVisitInts;)
   fa_fwd_kernel<D, PARTIAL, FP8><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, to, b);
   return cudaGetLastError();

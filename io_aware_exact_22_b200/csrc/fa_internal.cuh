@@ -17,6 +17,7 @@ struct FwdArgs {
   float scale_log2;  // scale * log2(e)
   int nsplit;        // key-range splits per (head, query block); 1 = whole key range
   int group = 1;      // work order: heads per group, heaviest query block first within a group
+  int persistent = 0;  // set by the launcher: CTAs walk the work list in pairs (see fa_fwd_kernel)
   // FP8 forward only: per-(b,h) dequantisation factors [BH], or null for 1
   const float* descale_q = nullptr;
   const float* descale_k = nullptr;
