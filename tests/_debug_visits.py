@@ -64,10 +64,11 @@ def main():
             # ragged lengths on two heads; and (d = 128, causal) ten heads long enough that the
             # work order puts them in groups of fewer heads, the last group short, and forty
             # heads of 8000 rows: enough query blocks for the forward's persistent CTAs, whose
-            # last block of each head has a single query tile
+            # last block of each head has a single query tile; and 240 heads of 1100 rows, five
+            # query blocks per head (pairs of items across two heads)
             shapes = [(1, 2, N) for N in (1, 129, 1000, 4096)]
             if d == 128 and causal:
-                shapes += [(1, 10, 16384), (1, 40, 8000)]
+                shapes += [(1, 10, 16384), (1, 40, 8000), (1, 240, 1100)]
             for B, H, N in shapes:
                 BH = B * H
                 w = custom(B, H, N, d, causal, seed=N + d, backward=True)

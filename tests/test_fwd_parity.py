@@ -79,6 +79,26 @@ def test_long_sequence_workload_sampled(cuda_ok):
     _sampled_rows_check(w, (q, k, v), f64(o), f64(lse), [(0, h) for h in range(32)], 52)
 
 
+@pytest.mark.parametrize("H,causal", [(240, True), (3, False)])
+def test_persistent_odd_block_count(cuda_ok, H, causal):
+    # N = 1100: five 256-row query blocks per head, the last with a single 128-row tile.  With
+    # the causal mask 240 heads give 1 200 items (enough for the persistent CTAs), 3 heads
+    # without it 15: an odd count per head puts pairs across two heads and leaves the list's
+    # last pair with one item.  Every row of 4 heads against the oracle, sampled rows of
+    # several more.
+    w = custom(1, H, 1100, 128, causal, seed=H)
+    (q, k, v), o, lse = _run(w)
+    o, lse = f64(o), f64(lse)
+    full = [(0, 0), (0, 1), (0, H // 2), (0, H - 1)] if H > 3 else [(0, h) for h in range(H)]
+    for b, h in full:
+        o_ref, l_ref = oracle.attention_forward_head(to_f64(q[b, h]), to_f64(k[b, h]), to_f64(v[b, h]),
+                                                     w.scale, w.causal)
+        check_o(o[b, h], o_ref, f"O[{b},{h}]")
+        check_lse(lse[b, h], l_ref)
+    if H > 3:
+        _sampled_rows_check(w, (q, k, v), o, lse, [(0, h) for h in range(0, H, 17)], 16)
+
+
 def _sampled_rows_check(w, inputs, o, lse, heads, rows_per_head):
     q, k, v = inputs
     rng = np.random.default_rng(0)
