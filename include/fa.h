@@ -149,6 +149,33 @@ fa_status_t fa_merge_partials(const float* o_parts, const float* lse_parts, int 
                               float* lse, int B, int H, int N, int d, void* stream);
 
 /*
+ * The same pieces combined as they come, without one partial result per piece: attention of q
+ * over one more set of keys k, v (all [B,H,N,d] bf16, the same N; causal as fa_fwd_partial),
+ * folded into a running partial result of these queries over the key sets seen before.  The
+ * running result (o_part fp32 [B,H,N,d], lse_part fp32 [B,H,N], fa_fwd_partial's format) is
+ * the state the kernel starts from: each row's LSE is its softmax reference, its sum relative to
+ * that reference is 1 and its output starts as o_part's row, and the key blocks of this set then
+ * update them exactly as blocks of one longer key range would ("Flash Attention",
+ * special-jiahao.github.io, section 增量求解 softmax: block results rescaled to a common
+ * reference and added).
+ *   flags & FA_CARRY_IN    : (o_part, lse_part) hold the running result, read first (rows with
+ *                            LSE = -inf have seen no key); without it the running result is
+ *                            empty and their contents do not matter
+ *   flags & FA_CARRY_FINAL : the result goes to o (bf16 [B,H,N,d], 16-byte aligned) and lse
+ *                            (fp32 [B,H,N], natural log), as fa_fwd writes them; without it it
+ *                            is written back into (o_part, lse_part), in place
+ * Calls for one set of queries run in order on one stream.  fa_fwd_carry over key sets 1..P,
+ * the first without FA_CARRY_IN and the last with FA_CARRY_FINAL, gives what fa_fwd over the
+ * concatenated keys gives (up to rounding order); memory is one running result whatever P is.
+ * d in {64, 128}; alignment as fa_fwd_partial; other flag bits return FA_ERR_INVALID_ARG.
+ */
+#define FA_CARRY_IN 1
+#define FA_CARRY_FINAL 2
+fa_status_t fa_fwd_carry(const void* q, const void* k, const void* v, float* o_part, float* lse_part,
+                         void* o, float* lse, int B, int H, int N, int d, float scale, int causal,
+                         int flags, void* stream);
+
+/*
  * Bytes of device workspace that fa_bwd needs: per 64-row query tile, the fp32 base-2 LSE and
  * row term D_i of its 64 rows (B*H*ceil(N/64)*128 floats, rounded up to 256 bytes), followed
  * by the fp32 dQ accumulator [B*H*N*d].  Returns 0 for an empty or invalid shape.

@@ -460,6 +460,45 @@ fa_status_t fa_fwd_partial(const void* q, const void* k, const void* v, float* o
   return launch_fwd_partial(d, tq, tk, tv, to, a, (cudaStream_t)stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+fa_status_t fa_fwd_carry(const void* q, const void* k, const void* v, float* o_part, float* lse_part, void* o,
+                         float* lse, int B, int H, int N, int d, float scale, int causal, int flags,
+                         void* stream) {
+  bool empty = false;
+  fa_status_t st = check_shape(B, H, N, d, scale, causal, &empty);
+  if (st != FA_OK || empty) return st;
+  if (flags & ~(FA_CARRY_IN | FA_CARRY_FINAL)) return FA_ERR_INVALID_ARG;
+  const bool in = (flags & FA_CARRY_IN) != 0, fin = (flags & FA_CARRY_FINAL) != 0;
+  if (!q || !k || !v || !o_part || !lse_part || (fin && (!o || !lse))) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o_part, 16) || !aligned(lse_part, 4) ||
+      (fin && (!aligned(o, 16) || !aligned(lse, 4))))
+    return FA_ERR_INVALID_ARG;
+  if ((st = check_device()) != FA_OK) return st;
+  const int BH = B * H;
+  if ((long long)BH * ((N + 255) / 256) > INT_MAX) return FA_ERR_INVALID_ARG;
+  CUtensorMap tq, tk, tv, to;
+  if (!make_tmap_bf16(&tq, q, BH, N, d, 128) || !make_tmap_bf16(&tk, k, BH, N, d, 128) ||
+      !make_tmap_bf16(&tv, v, BH, N, d, 128) ||
+      !(fin ? make_tmap_bf16(&to, o, BH, N, d, 32) : make_tmap_f32(&to, o_part, BH, N, d, 32, 32, true)))
+    return FA_ERR_CUDA;
+  FwdArgs a;
+  if (!(a.status = device_status_word())) return FA_ERR_CUDA;
+  a.lse = fin ? lse : lse_part;
+  a.N = N;
+  a.BH = BH;
+  a.nqb = (N + 255) / 256;
+  a.causal = causal;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  a.nsplit = 1;
+  a.group = work_group(BH, N, d, 2, causal);
+  if (in) {  // each CTA reads its rows' carried result before it writes them
+    a.carry_o = o_part;
+    a.carry_lse = lse_part;
+  }
+  const cudaError_t e = fin ? launch_fwd(d, tq, tk, tv, to, a, (cudaStream_t)stream)
+                            : launch_fwd_partial(d, tq, tk, tv, to, a, (cudaStream_t)stream);
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 fa_status_t fa_merge_partials(const float* o_parts, const float* lse_parts, int nparts, void* o, float* lse,
                               int B, int H, int N, int d, void* stream) {
   bool empty = false;

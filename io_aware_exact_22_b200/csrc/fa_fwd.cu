@@ -208,6 +208,7 @@ __global__ void __launch_bounds__(352, 1)
   // ring positions within an item of nmax blocks: K_0 first, then K_{j+1} (when there is
   // one) before V_j; every item takes 2 nmax consecutive positions
   auto pos_k = [](int j) { return j == 0 ? 0 : 2 * j - 1; };
+  const bool carry = !FP8 && a.carry_o != nullptr;  // rows continue from a carried partial result
   auto pos_v = [](int j, int nmax) { return j + 1 < nmax ? 2 * j + 2 : 2 * j + 1; };
 
   if (warp == 9) {
@@ -358,7 +359,8 @@ __global__ void __launch_bounds__(352, 1)
                 break;
               if (!(ok = __all_sync(0xffffffffu, mbar_wait(p_full(t), cp[t] & 1, wc)))) break;
               tc_fence_after();
-              issue_pv(t ? C::T_O1 : C::T_O0, (uint32_t)(t * C::PTILE), stage_addr(itV), j > 0);
+              // the first product of an item accumulates onto a carried O (written by the softmax)
+              issue_pv(t ? C::T_O1 : C::T_O0, (uint32_t)(t * C::PTILE), stage_addr(itV), j > 0 || carry);
               mma_commit_e(pv_done(t));
               ++cp[t];
               // bf16, whole key range: O_t of this item is complete once this product is (its
@@ -413,7 +415,7 @@ __global__ void __launch_bounds__(352, 1)
     const int qrow = wk.q0 + 128 * t + r;
     if (wk.nmax == 0 || ntile == 0) {
       // this split holds no key block of this tile: an empty partial (weight 0 in the merge)
-      if (PARTIAL && qrow < a.N) a.lse[((size_t)split * a.BH + bh) * a.N + qrow] = -INFINITY;
+      if (PARTIAL && !carry && qrow < a.N) a.lse[((size_t)split * a.BH + bh) * a.N + qrow] = -INFINITY;
       continue;
     }
     float cs = a.scale_log2;
@@ -425,6 +427,33 @@ __global__ void __launch_bounds__(352, 1)
     }
     float m_ref = -INFINITY;  // reference max, base-2 scaled units
     float l = 0.f;
+    if (carry) {
+      // Continue from a partial result over other keys ([jiahao] 增量求解 softmax: the blocks'
+      // sums and outputs rescaled to a common reference): its LSE is the reference, the sum
+      // relative to it is 1 and O_t starts as its normalised output, so the block loop below
+      // carries on as if those keys had come first.  A row that has seen no key starts empty.
+      const float L = qrow < a.N ? a.carry_lse[(size_t)bh * a.N + qrow] : -INFINITY;
+      const bool has = L > -INFINITY;
+      if (has) {
+        m_ref = L * 1.4426950408889634074f;
+        l = 1.f;
+      }
+      const float* src = a.carry_o + ((size_t)bh * a.N + (has ? qrow : 0)) * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D; cc += 32) {
+        uint32_t ov[32];
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 f = has ? *reinterpret_cast<const float4*>(src + cc + 4 * e4) : make_float4(0.f, 0.f, 0.f, 0.f);
+          ov[4 * e4 + 0] = __float_as_uint(f.x);
+          ov[4 * e4 + 1] = __float_as_uint(f.y);
+          ov[4 * e4 + 2] = __float_as_uint(f.z);
+          ov[4 * e4 + 3] = __float_as_uint(f.w);
+        }
+        tmem_st32(tOrow + cc, ov);
+      }
+      tmem_wait_st();
+    }
 
     for (int j = 0; j < ntile && ok; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(s_full(t), ns & 1, wc));
@@ -572,8 +601,9 @@ __global__ void __launch_bounds__(352, 1)
         rsum = rs0 + rs1;
       }
       l += rsum;
-      if (j > 0 && __any_sync(0xffffffffu, move)) {
-        // O_t holds sum_{j' < j} of P V relative to the old reference: rescale by alpha.
+      if ((j > 0 || carry) && __any_sync(0xffffffffu, move)) {
+        // O_t holds sum_{j' < j} of P V (and a carried output) relative to the old reference:
+        // rescale by alpha.
         tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < D; cc += 32) {

@@ -22,6 +22,11 @@ struct FwdArgs {
   const float* descale_q = nullptr;
   const float* descale_k = nullptr;
   const float* descale_v = nullptr;
+  // Carried partial result (bf16 kernels, whole key range): when set, the rows continue from
+  // a normalised output carry_o [BH, N, d] fp32 and its natural-log LSE carry_lse [BH, N] over
+  // other keys (rows with LSE = -inf have seen none)
+  const float* carry_o = nullptr;
+  const float* carry_lse = nullptr;
   // debug build: visit counters [BH][ceil(N/128)][ceil(N/128)] (null in the release build)
   int* visits = nullptr;
   long long visits_cap = 0;

@@ -25,7 +25,7 @@ STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_E
 EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_device_status",
            "fa_status_string", "fa_version", "fa_bwd_noalloc", "fa_selftest_wait_timeout",
            "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_default_splits",
-           "fa_bwd_deterministic", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials",
+           "fa_bwd_deterministic", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials", "fa_fwd_carry",
            "fa_bwd_prepare", "fa_bwd_accumulate", "fa_bwd_finish", "fa_bwd_main", "fa_bwd_dq_post",
            "fa_debug_build", "fa_debug_visits")
 # Size of the library's built-in scratch used by fa_bwd_noalloc (include/fa.h).
@@ -57,6 +57,8 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd_partial.restype = i
         L.fa_merge_partials.argtypes = [vp, vp, i, vp, vp, i, i, i, i, vp]
         L.fa_merge_partials.restype = i
+        L.fa_fwd_carry.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
+        L.fa_fwd_carry.restype = i
         L.fa_bwd_prepare.argtypes = [vp, vp, vp, vp, sz, i, i, i, i, vp]
         L.fa_bwd_prepare.restype = i
         L.fa_bwd_accumulate.argtypes = [vp, vp, vp, vp, vp, sz, vp, vp, i, i, i, i, f, i, vp]
@@ -129,6 +131,14 @@ def fa_fwd_fp8(q, k, v, descale_q, descale_k, descale_v, o, lse, B, H, N, d, sca
 def fa_fwd_partial(q, k, v, o_part, lse_part, B, H, N, d, scale, causal, stream=None) -> int:
     return lib().fa_fwd_partial(_ptr(q), _ptr(k), _ptr(v), _ptr(o_part), _ptr(lse_part), B, H, N, d,
                                 float(scale), int(causal), _stream(stream))
+
+
+FA_CARRY_IN, FA_CARRY_FINAL = 1, 2
+
+
+def fa_fwd_carry(q, k, v, o_part, lse_part, o, lse, B, H, N, d, scale, causal, flags, stream=None) -> int:
+    return lib().fa_fwd_carry(_ptr(q), _ptr(k), _ptr(v), _ptr(o_part), _ptr(lse_part), _ptr(o), _ptr(lse), B, H,
+                              N, d, float(scale), int(causal), int(flags), _stream(stream))
 
 
 def fa_merge_partials(o_parts, lse_parts, nparts, o, lse, B, H, N, d, stream=None) -> int:

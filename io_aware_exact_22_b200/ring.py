@@ -4,11 +4,12 @@ Rank r of W holds the r-th contiguous shard of the sequence of q, k and v (each 
 global positions [r n, r n + n)).  The K/V shards travel around the ring (rank r sends to
 r + 1 and receives from r - 1, one shard per step, through torch.distributed point-to-point
 calls, NCCL on GPUs); while a shard is in flight the rank computes its queries' partial result
-over the shard it holds, with fa_fwd_partial: unmasked for a shard that lies entirely before
-its queries, with the causal mask for its own shard, skipped for shards after it (causal).
-fa_merge_partials then combines the partial results by the softmax merge of "Flash Attention"
-(special-jiahao.github.io, section 增量求解 softmax), which is what makes the pieces add up to
-exact attention over the whole sequence.
+over the shard it holds and folds it into one running partial result (fa_fwd_carry): unmasked
+for a shard that lies entirely before its queries, with the causal mask for its own shard,
+skipped for shards after it (causal).  The fold is the two-block softmax merge of "Flash
+Attention" (special-jiahao.github.io, section 增量求解 softmax), done inside the kernel: the
+running result is the starting state of the next shard's block loop, which is what makes the
+pieces add up to exact attention over the whole sequence with one running result per rank.
 
 The backward passes each K/V shard round the ring together with fp32 accumulators for its
 dK and dV: every rank adds its queries' contribution (fa_bwd_accumulate, which also adds into
@@ -72,21 +73,21 @@ def visible_shards(r: int, W: int, causal: bool):
 
 
 def _accumulate(q, shard_iter, r: int, W: int, causal: bool, scale: float, out, lse, stream=None):
+    """Folds each visible shard, as it arrives, into one running partial result of this rank's
+    queries (fa_fwd_carry); the last visible shard writes the bf16 output and LSE."""
     B, H, n, d = q.shape
     vis = visible_shards(r, W, causal)
-    parts_o = torch.empty((len(vis), B, H, n, d), device=q.device, dtype=torch.float32)
-    parts_l = torch.empty((len(vis), B, H, n), device=q.device, dtype=torch.float32)
+    run_o = torch.empty((B, H, n, d), device=q.device, dtype=torch.float32)
+    run_l = torch.empty((B, H, n), device=q.device, dtype=torch.float32)
     i = 0
     for src, ks, vs in shard_iter:
         if src not in vis:
             continue
-        rc = fa.fa_fwd_partial(q, ks, vs, parts_o[i], parts_l[i], B, H, n, d, scale, vis[src], stream)
+        flags = (fa.FA_CARRY_IN if i > 0 else 0) | (fa.FA_CARRY_FINAL if i == len(vis) - 1 else 0)
+        rc = fa.fa_fwd_carry(q, ks, vs, run_o, run_l, out, lse, B, H, n, d, scale, vis[src], flags, stream)
         if rc:
-            raise fa.FAError(rc, "fa_fwd_partial")
+            raise fa.FAError(rc, "fa_fwd_carry")
         i += 1
-    rc = fa.fa_merge_partials(parts_o, parts_l, i, out, lse, B, H, n, d, stream)
-    if rc:
-        raise fa.FAError(rc, "fa_merge_partials")
     return out, lse
 
 

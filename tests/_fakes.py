@@ -11,7 +11,9 @@ from io_aware_exact_22_b200 import fa, ring
 class FakeFA:
     """fp64 stand-ins for the piece calls, each following its contract in include/fa.h:
     fa_fwd_partial writes O_s = softmax-normalised partial output and its natural-log LSE;
-    fa_merge_partials combines parts by their LSEs; fa_bwd_prepare keeps D = rowsum(dO o O) and
+    fa_merge_partials combines parts by their LSEs; fa_fwd_carry merges this key set's partial
+    result into the running one the same way (or starts it), and writes it back or, with
+    FA_CARRY_FINAL, to the output; fa_bwd_prepare keeps D = rowsum(dO o O) and
     LSE with a zeroed dQ accumulator in the workspace; fa_bwd_accumulate adds dS K into that
     accumulator and scale dS^T Q, P^T dO into the dK, dV accumulators; fa_bwd_finish writes
     scale * dQ and the two accumulators."""
@@ -33,6 +35,28 @@ class FakeFA:
         lse = torch.logsumexp(s, -1)
         o_part.copy_(torch.exp(s - lse[..., None]) @ v.double())
         lse_part.copy_(lse)
+        return 0
+
+    FA_CARRY_IN, FA_CARRY_FINAL = fa.FA_CARRY_IN, fa.FA_CARRY_FINAL
+
+    def fa_fwd_carry(self, q, k, v, o_part, lse_part, o, lse, B, H, n, d, scale, causal, flags, stream=None):
+        s = self._scores(q, k, scale, causal)
+        L = torch.logsumexp(s, -1)
+        O = torch.exp(s - L[..., None]) @ v.double()
+        if flags & fa.FA_CARRY_IN:
+            L0, O0 = lse_part.double(), o_part.double()
+            m = torch.maximum(L0, L)
+            m = torch.where(torch.isfinite(m), m, torch.zeros_like(m))  # rows with no key yet
+            w0, w1 = torch.exp(L0 - m), torch.exp(L - m)
+            tot = w0 + w1
+            O = (w0[..., None] * O0 + w1[..., None] * O) / tot[..., None]
+            L = m + torch.log(tot)
+        if flags & fa.FA_CARRY_FINAL:
+            o.copy_(O)
+            lse.copy_(L)
+        else:
+            o_part.copy_(O)
+            lse_part.copy_(L)
         return 0
 
     def fa_merge_partials(self, o_parts, lse_parts, nparts, o, lse, B, H, n, d, stream=None):

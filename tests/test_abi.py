@@ -157,3 +157,18 @@ def test_backward_main_rejects_bad_arguments(kw, code):
 ])
 def test_backward_dq_post_rejects_bad_arguments(args, code):
     assert fa.fa_bwd_dq_post(*args, 0) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(flags=4), INVALID), (dict(flags=-1), INVALID), (dict(q=0), INVALID), (dict(o_part=0), INVALID),
+    (dict(o=0), INVALID), (dict(lse=0), INVALID), (dict(o_part=A16 + 8), INVALID), (dict(o=A16 + 2), INVALID),
+    (dict(d=96), UNSUPPORTED), (dict(N=-1), INVALID), (dict(scale=0.0), INVALID), (dict(N=0), OK),
+])
+def test_carry_rejects_bad_arguments(kw, code):
+    args = dict(q=A16, k=A16, v=A16, o_part=A16, lse_part=A16, o=A16, lse=A16, B=1, H=1, N=128, d=128,
+                scale=0.125, causal=0, flags=fa.FA_CARRY_IN | fa.FA_CARRY_FINAL)
+    args.update(kw)
+    assert fa.fa_fwd_carry(args["q"], args["k"], args["v"], args["o_part"], args["lse_part"], args["o"],
+                           args["lse"], args["B"], args["H"], args["N"], args["d"], args["scale"], args["causal"],
+                           args["flags"], 0) == code
+

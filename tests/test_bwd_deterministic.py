@@ -38,19 +38,24 @@ def test_empty_problem_is_a_no_op():
                                    1, 0, 100, 128, 0.1, 0, 0) == OK
 
 
-def _run(w, inputs=None, deterministic=True):
+def _run_with_o(w, inputs=None, deterministic=True):
+    """Inputs (CPU), gradients (GPU) and the forward's stored output O (fp64 numpy)."""
     q, k, v, do = inputs if inputs is not None else make_inputs(w, with_grad=True)
     qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
     o, lse = fa.forward(qd, kd, vd, w.causal, w.scale)
     grads = fa.backward(qd, kd, vd, o, dod, lse, w.causal, w.scale, deterministic=deterministic)
     torch.cuda.synchronize()
     assert fa.fa_get_device_status() == 0
-    _run.o = f64(o)
-    return (q, k, v, do), grads
+    return (q, k, v, do), grads, f64(o)
+
+
+def _run(w, inputs=None, deterministic=True):
+    ins, grads, _ = _run_with_o(w, inputs, deterministic)
+    return ins, grads
 
 
 def _check(w, heads=None, inputs=None, rel_tol=None, given_o=False):
-    (q, k, v, do), grads = _run(w, inputs)
+    (q, k, v, do), grads, o_st = _run_with_o(w, inputs)
     dq, dk, dv = (f64(g) for g in grads)
     if heads is None:
         heads = [(b, h) for b in range(w.B) for h in range(w.H)]
@@ -61,7 +66,7 @@ def _check(w, heads=None, inputs=None, rel_tol=None, given_o=False):
         gq, gk, gv, _ = oracle.attention_backward_head(to_f64(q[b, h]), to_f64(k[b, h]),
                                                        to_f64(v[b, h]), to_f64(do[b, h]),
                                                        w.scale, w.causal,
-                                                       o=_run.o[b, h] if given_o else None)
+                                                       o=o_st[b, h] if given_o else None)
         check_grad(dq[b, h], gq, f"dQ[{b},{h}]", **kw)
         check_grad(dk[b, h], gk, f"dK[{b},{h}]", **kw)
         check_grad(dv[b, h], gv, f"dV[{b},{h}]", **kw)

@@ -17,27 +17,32 @@ from tests._helpers import abs_term_sums, check_grad, f64
 pytestmark = pytest.mark.gpu
 
 
-def _gpu(w, inputs=None):
+def _gpu_with_o(w, inputs=None):
+    """Inputs (CPU), gradients and the forward's stored output O (fp64 numpy)."""
     q, k, v, do = inputs if inputs is not None else make_inputs(w, with_grad=True)
     qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
     o, lse = fa.forward(qd, kd, vd, w.causal, w.scale)
     dq, dk, dv = fa.backward(qd, kd, vd, o, dod, lse, w.causal, w.scale)
     torch.cuda.synchronize()
     assert fa.fa_get_device_status() == 0
-    _gpu.o = f64(o)
-    return (q, k, v, do), (f64(dq), f64(dk), f64(dv))
+    return (q, k, v, do), (f64(dq), f64(dk), f64(dv)), f64(o)
+
+
+def _gpu(w, inputs=None):
+    ins, grads, _ = _gpu_with_o(w, inputs)
+    return ins, grads
 
 
 def _check_heads(w, heads=None, inputs=None, rel_tol=None, term_bound=False, given_o=False):
     """given_o: the oracle's D_i = rowsum(dO o O) is taken from the bf16 O the forward stored
     (the backward's own input) instead of the exact one."""
-    (q, k, v, do), (dq, dk, dv) = _gpu(w, inputs)
+    (q, k, v, do), (dq, dk, dv), o_st = _gpu_with_o(w, inputs)
     if heads is None:
         heads = [(b, h) for b in range(w.B) for h in range(w.H)]
     for b, h in heads:
         args = [to_f64(t[b, h]) for t in (q, k, v, do)]
         gq, gk, gv, _ = oracle.attention_backward_head(*args, w.scale, w.causal,
-                                                       o=_gpu.o[b, h] if given_o else None)
+                                                       o=o_st[b, h] if given_o else None)
         sums = abs_term_sums(*args, w.scale, w.causal) if term_bound else (None, None, None)
         kw = {}
         if rel_tol is not None:
