@@ -239,8 +239,8 @@ def _ok(rc, name):
 # the zig-zag layout the sequence is cut into 2W chunks and rank r holds chunks r and 2W-1-r
 # (one early, one late), so every rank computes 2W+1 pieces (W(2W+1) = the 2W(2W+1)/2 visible
 # chunk pairs spread evenly).  Each rank passes a list of two chunks of q, k, v (and so on) of
-# equal shape [B, H, n, d]; the pieces are the same partial-result, merge and accumulate calls
-# as for contiguous shards.
+# equal shape [B, H, n, d]; the pieces are the same carry and accumulate calls as for
+# contiguous shards.
 
 def zigzag_chunks(r: int, W: int):
     """Sequence chunks (of 2W) held by rank r: (r, 2W-1-r)."""
@@ -273,24 +273,21 @@ def _check_chunks(ts, bwd: bool):
 
 def _zigzag_forward(q2, shard_iter, r, W, causal, scale, out2, lse2):
     """O and LSE of rank r's two query chunks from the key/value chunks of every rank
-    (shard_iter yields (src, [k_a, k_b, v_a, v_b]) of rank src's chunks)."""
+    (shard_iter yields (src, [k_a, k_b, v_a, v_b]) of rank src's chunks).  Each query chunk
+    folds its pieces, as they come, into one running partial result (fa_fwd_carry); its last
+    piece writes the bf16 output and LSE."""
     B, H, n, d = q2[0].shape
     chunks = zigzag_chunks(r, W)
-    parts = []
-    for a in chunks:
-        m = a + 1 if causal else 2 * W  # key chunks visible to query chunk a
-        parts.append((torch.empty((m, B, H, n, d), device=q2[0].device, dtype=torch.float32),
-                      torch.empty((m, B, H, n), device=q2[0].device, dtype=torch.float32)))
+    total = [a + 1 if causal else 2 * W for a in chunks]  # key chunks visible to each query chunk
+    runs = [(torch.empty((B, H, n, d), device=q2[0].device, dtype=torch.float32),
+             torch.empty((B, H, n), device=q2[0].device, dtype=torch.float32)) for _ in chunks]
     used = [0, 0]
     for src, held in shard_iter:
         for iq, ik, masked in zigzag_pieces(r, W, src, causal):
-            po, pl = parts[iq]
-            _ok(fa.fa_fwd_partial(q2[iq], held[ik], held[2 + ik], po[used[iq]], pl[used[iq]], B, H, n, d,
-                                  scale, masked), "fa_fwd_partial")
+            flags = (fa.FA_CARRY_IN if used[iq] else 0) | (fa.FA_CARRY_FINAL if used[iq] == total[iq] - 1 else 0)
+            _ok(fa.fa_fwd_carry(q2[iq], held[ik], held[2 + ik], runs[iq][0], runs[iq][1], out2[iq], lse2[iq],
+                                B, H, n, d, scale, masked, flags), "fa_fwd_carry")
             used[iq] += 1
-    for iq in range(2):
-        _ok(fa.fa_merge_partials(parts[iq][0], parts[iq][1], used[iq], out2[iq], lse2[iq], B, H, n, d),
-            "fa_merge_partials")
     return out2, lse2
 
 
