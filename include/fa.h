@@ -178,7 +178,8 @@ fa_status_t fa_fwd_carry(const void* q, const void* k, const void* v, float* o_p
 /*
  * Bytes of device workspace that fa_bwd needs: per 64-row query tile, the fp32 base-2 LSE and
  * row term D_i of its 64 rows (B*H*ceil(N/64)*128 floats, rounded up to 256 bytes), followed
- * by the fp32 dQ accumulator [B*H*N*d].  Returns 0 for an empty or invalid shape.
+ * by the fp32 dQ accumulator [B*H*N*d] and a 256-byte block holding the work counter of the
+ * persistent key-tile kernel.  Returns 0 for an empty or invalid shape.
  */
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 

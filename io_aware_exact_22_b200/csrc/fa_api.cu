@@ -128,6 +128,13 @@ size_t ld_bytes(long long bh, int N) {
   return ((size_t)tiles * 128 * 4 + 255) & ~(size_t)255;
 }
 
+// The backward workspace: the per-tile statistics (ld_bytes), the fp32 dQ accumulator, then a
+// 256-byte block whose first two ints are the key-tile kernel's work counter.
+constexpr size_t kWorkBytes = 256;
+int* work_counter(void* workspace, long long bh, int N, int d) {
+  return reinterpret_cast<int*>(reinterpret_cast<char*>(workspace) + ld_bytes(bh, N) + (size_t)bh * N * d * 4);
+}
+
 }  // namespace
 
 // Tensor maps depend only on (address, shape, box, element type, swizzle), so encoded maps are
@@ -518,7 +525,7 @@ fa_status_t fa_merge_partials(const float* o_parts, const float* lse_parts, int 
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
   const long long rows = (long long)B * H * N;
-  return ld_bytes((long long)B * H, N) + (size_t)rows * d * 4;
+  return ld_bytes((long long)B * H, N) + (size_t)rows * d * 4 + kWorkBytes;
 }
 
 // The key-tile kernel of fa_bwd on prepared statistics (d = 64 or 128): bf16 dK, dV stored (or,
@@ -553,6 +560,7 @@ static fa_status_t bwd_main_dq(const void* q, const void* k, const void* v, cons
   a.scale = scale;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   a.group = work_group(BH, N, d, 2, causal);
+  a.work = work_counter(workspace, BH, N, d);
   cudaError_t e = launch_bwd_main(d, tq, tk, tv, tdo, tdk, tdv, tdq, a, s);
   if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -584,7 +592,8 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
   float* ld = reinterpret_cast<float*>(workspace);
   float* dq_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + ld_bytes(BH, N));
   cudaStream_t s = (cudaStream_t)stream;
-  if (launch_bwd_pre(o, dO, lse, ld, dq_acc, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (launch_bwd_pre(o, dO, lse, ld, dq_acc, work_counter(workspace, BH, N, d), BH, N, d, s) != cudaSuccess)
+    return FA_ERR_CUDA;
   if ((st = bwd_main_dq(q, k, v, dO, workspace, dk, dv, BH, N, d, scale, causal, s)) != FA_OK) return st;
   if (launch_bwd_post(dq_acc, dq, rows * d, scale, s) != cudaSuccess) return FA_ERR_CUDA;
   return FA_OK;
@@ -627,7 +636,8 @@ fa_status_t fa_bwd_prepare(const void* o, const void* dO, const float* lse, void
   const int BH = B * H;
   float* ld = reinterpret_cast<float*>(workspace);
   float* dq_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + ld_bytes(BH, N));
-  return launch_bwd_pre(o, dO, lse, ld, dq_acc, BH, N, d, (cudaStream_t)stream) == cudaSuccess ? FA_OK
+  return launch_bwd_pre(o, dO, lse, ld, dq_acc, work_counter(workspace, BH, N, d), BH, N, d,
+                        (cudaStream_t)stream) == cudaSuccess ? FA_OK
                                                                                                 : FA_ERR_CUDA;
 }
 
@@ -706,7 +716,8 @@ fa_status_t fa_bwd_deterministic(const void* q, const void* k, const void* v, co
   a.scale = scale;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   a.group = work_group(BH, N, d, 2, causal);
-  if (launch_bwd_pre(o, dO, lse, ld, nullptr, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  a.work = work_counter(workspace, BH, N, d);
+  if (launch_bwd_pre(o, dO, lse, ld, nullptr, a.work, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
   if (launch_bwd_main(d, tq64, tk128, tv128, tdo64, tdk, tdv, tdk, a, s, false) != cudaSuccess) return FA_ERR_CUDA;
   if (launch_bwd_dq(d, tq128, tk64, tv64, tdo128, tdq, a, s) != cudaSuccess) return FA_ERR_CUDA;
   return FA_OK;

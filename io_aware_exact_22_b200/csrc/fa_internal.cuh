@@ -48,6 +48,10 @@ struct BwdArgs {
   float* dk_acc = nullptr;
   float* dv_acc = nullptr;
   int group = 1;  // work order: heads per group, heaviest key tile first within a group
+  // two ints in device memory, zero before each launch of the key-tile kernel (the pre-kernel
+  // zeroes them; the kernel's last CTA zeroes them again on exit): the next unclaimed item
+  // and the number of CTAs done
+  int* work = nullptr;
   // debug build: visit counters of the kernel launched with these arguments (null in release)
   int* visits = nullptr;
   long long visits_cap = 0;
@@ -97,7 +101,7 @@ cudaError_t launch_fwd_fp8(int d, const CUtensorMap& tq, const CUtensorMap& tk, 
 cudaError_t launch_fwd_merge(const float* o_part, const float* lse_part, void* o, float* lse, int nsplit,
                              long long rows, int d, cudaStream_t stream);
 
-cudaError_t launch_bwd_pre(const void* o, const void* dO, const float* lse, float* ld, float* dq_acc,
+cudaError_t launch_bwd_pre(const void* o, const void* dO, const float* lse, float* ld, float* dq_acc, int* work,
                            int BH, int N, int d, cudaStream_t stream);
 // fp32 [BH, N, d] tensor map without swizzle, box = box_inner columns x box_rows rows.
 bool make_tmap_f32(CUtensorMap* m, const void* ptr, int BH, int N, int d, int box_inner, int box_rows,

@@ -48,7 +48,8 @@ def test_workspace_size():
     B, H, N, d = 2, 3, 100, 128
     rows = B * H * N
     tiles = B * H * ((N + 63) // 64)
-    assert fa.fa_bwd_workspace_bytes(B, H, N, d) == ((tiles * 512 + 255) // 256) * 256 + rows * d * 4
+    # per-tile statistics (rounded up to 256 bytes), the fp32 dQ accumulator, the work counter block
+    assert fa.fa_bwd_workspace_bytes(B, H, N, d) == ((tiles * 512 + 255) // 256) * 256 + rows * d * 4 + 256
     assert fa.fa_bwd_workspace_bytes(0, 3, 100, 128) == 0
     assert fa.fa_bwd_workspace_bytes(1, 1, -1, 128) == 0
 
