@@ -53,8 +53,8 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
                                                          float* __restrict__ ld,
                                                          float* __restrict__ dq_acc, int* __restrict__ work,
                                                          int BH, int N, int Tq) {
-  constexpr int PIECES = D / 32;
-  if (blockIdx.x == 0 && threadIdx.x < 2) work[threadIdx.x] = 0;  // the key-tile kernel's work counter  // 16-byte pieces of a bf16 row per thread
+  constexpr int PIECES = D / 32;  // 16-byte pieces of a bf16 row per thread
+  if (blockIdx.x == 0 && threadIdx.x < 2) work[threadIdx.x] = 0;  // the key-tile kernel's work counter
   const int r = threadIdx.x >> 2;  // row within the tile
   const int q = threadIdx.x & 3;
   const long long tiles = (long long)BH * Tq;
