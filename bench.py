@@ -496,7 +496,8 @@ def measure_variants(w, dev, stream, qd, kd, vd, o, lse, dod, dq, dk, dv, ws, ws
                       iters=5)
         tf = w.fwd_flops() / (ms * 1e-3) / 1e12
         out["fwd_ring_sharded_on_one_gpu"] = {
-            "kernels": "fa_fwd_kernel<128, partial> per (rank, visible shard) + fa_fwd_merge_kernel<128>",
+            "kernels": "fa_fwd_kernel<128> per (rank, visible shard), each carrying the rank's running "
+                       "result (fa_fwd_carry); the last visible shard writes bf16",
             "shape": f"{w.name}, {W} shards of {n}", "ms": round(ms, 4), "tflops": round(tf, 1),
             "peak": peak, "frac": round(tf / peak, 4)}
         if d == 128:
