@@ -509,7 +509,8 @@ def measure_variants(w, dev, stream, qd, kd, vd, o, lse, dod, dq, dk, dv, ws, ws
             tf = w.bwd_flops() / (ms * 1e-3) / 1e12
             out["bwd_ring_sharded_on_one_gpu"] = {
                 "kernels": "fa_bwd_pre_kernel per rank + fa_bwd_main_kernel<128> (accumulate) per (rank, "
-                           "visible shard) + fa_bwd_post_kernel x 3 per rank",
+                           "visible shard), into a zeroed local pair and fa_acc_add_kernel x 2 for other "
+                           "ranks' shards + fa_bwd_post_kernel x 3 per rank",
                 "shape": f"{w.name}, {W} shards of {n}", "ms": round(ms, 4), "tflops": round(tf, 1),
                 "peak": peak, "frac": round(tf / peak, 4)}
             del fw, os_, ls_, dos

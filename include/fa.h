@@ -263,6 +263,26 @@ fa_status_t fa_bwd_accumulate(const void* q, const void* k, const void* v, const
 fa_status_t fa_bwd_finish(const void* workspace, size_t workspace_bytes, const float* dk_acc,
                           const float* dv_acc, void* dq, void* dk, void* dv,
                           int B, int H, int N, int d, float scale, void* stream);
+/*
+ * fa_bwd_accumulate with the key set's contribution stored instead of added: dk_out = scale *
+ * dK and dv_out = dV of this key set alone (fp32 [B,H,N,d], 16-byte aligned, every row
+ * written), dQ still added into the workspace's accumulator.  The sequence-sharded backward
+ * computes a passing key set's contribution this way while that key set's accumulators are
+ * on their way, then adds it in with fa_bwd_acc_add.  Same arguments and error rules as
+ * fa_bwd_accumulate.
+ */
+fa_status_t fa_bwd_contribute(const void* q, const void* k, const void* v, const void* dO,
+                              void* workspace, size_t workspace_bytes, float* dk_out,
+                              float* dv_out, int B, int H, int N, int d, float scale, int causal,
+                              void* stream);
+
+/*
+ * acc += x, element by element, for two fp32 [B,H,N,d] accumulators (16-byte aligned, d in
+ * {64, 128}): the sequence-sharded backward computes a key set's contribution into a zeroed
+ * local pair while that key set's dK/dV accumulators are still arriving from the previous
+ * rank, then adds it in with this call.  Same error rules as fa_bwd_finish.
+ */
+fa_status_t fa_bwd_acc_add(float* acc, const float* x, int B, int H, int N, int d, void* stream);
 
 /*
  * fa_bwd taken apart into its three kernels, so that each can be launched, and

@@ -533,7 +533,7 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
 // workspace's fp32 accumulator.  Arguments are checked by the callers.
 static fa_status_t bwd_main_dq(const void* q, const void* k, const void* v, const void* dO, void* workspace,
                                void* dk, void* dv, int BH, int N, int d, float scale, int causal, cudaStream_t s,
-                               float* dk_acc = nullptr, float* dv_acc = nullptr) {
+                               float* dk_acc = nullptr, float* dv_acc = nullptr, bool acc_overwrite = false) {
   float* ld = reinterpret_cast<float*>(workspace);
   float* dq_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + ld_bytes(BH, N));
   CUtensorMap tq, tk, tv, tdo, tdk, tdv, tdq;
@@ -554,6 +554,7 @@ static fa_status_t bwd_main_dq(const void* q, const void* k, const void* v, cons
   a.dq_acc = dq_acc;
   a.dk_acc = dk_acc;
   a.dv_acc = dv_acc;
+  a.acc_overwrite = acc_overwrite ? 1 : 0;
   a.N = N;
   a.BH = BH;
   a.causal = causal;
@@ -657,6 +658,22 @@ fa_status_t fa_bwd_accumulate(const void* q, const void* k, const void* v, const
                        dk_acc, dv_acc);
 }
 
+fa_status_t fa_bwd_contribute(const void* q, const void* k, const void* v, const void* dO, void* workspace,
+                              size_t workspace_bytes, float* dk_out, float* dv_out, int B, int H, int N, int d,
+                              float scale, int causal, void* stream) {
+  bool empty = false;
+  fa_status_t st = check_shape(B, H, N, d, scale, causal, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!q || !k || !v || !dO || !workspace || !dk_out || !dv_out) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dO, 16) || !aligned(workspace, 256) ||
+      !aligned(dk_out, 16) || !aligned(dv_out, 16))
+    return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  if ((st = check_device()) != FA_OK) return st;
+  return bwd_main_dq(q, k, v, dO, workspace, nullptr, nullptr, B * H, N, d, scale, causal, (cudaStream_t)stream,
+                     dk_out, dv_out, true);
+}
+
 fa_status_t fa_bwd_finish(const void* workspace, size_t workspace_bytes, const float* dk_acc, const float* dv_acc,
                           void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, void* stream) {
   bool empty = false;
@@ -676,6 +693,16 @@ fa_status_t fa_bwd_finish(const void* workspace, size_t workspace_bytes, const f
   if (launch_bwd_post(dk_acc, dk, elems, 1.0f, s) != cudaSuccess) return FA_ERR_CUDA;
   if (launch_bwd_post(dv_acc, dv, elems, 1.0f, s) != cudaSuccess) return FA_ERR_CUDA;
   return FA_OK;
+}
+
+fa_status_t fa_bwd_acc_add(float* acc, const float* x, int B, int H, int N, int d, void* stream) {
+  bool empty = false;
+  fa_status_t st = check_shape(B, H, N, d, 1.0f, 0, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!acc || !x || !aligned(acc, 16) || !aligned(x, 16)) return FA_ERR_INVALID_ARG;
+  if ((st = check_device()) != FA_OK) return st;
+  const long long elems = (long long)B * H * N * d;
+  return launch_acc_add(acc, x, elems, (cudaStream_t)stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 fa_status_t fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o, const void* dO,

@@ -115,6 +115,21 @@ __global__ void __launch_bounds__(256) fa_bwd_post_kernel(const float4* __restri
   }
 }
 
+// Accumulator add for the sequence-sharded backward: acc += x, fp32, 16 bytes per thread.
+__global__ void __launch_bounds__(256) fa_acc_add_kernel(float4* __restrict__ acc, const float4* __restrict__ x,
+                                                         long long n4) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (long long)gridDim.x * blockDim.x) {
+    float4 a = acc[i];
+    const float4 b = x[i];
+    a.x += b.x;
+    a.y += b.y;
+    a.z += b.z;
+    a.w += b.w;
+    acc[i] = a;
+  }
+}
+
 // ------------------------------------------------------------------ K3
 template <int D_>
 struct BwdCfg {
@@ -682,8 +697,9 @@ __global__ void __launch_bounds__(480, 1)
       const int r = wq * 32 + lane;
       const int key = 128 * w.j + r;
       if (a.dk_acc != nullptr) {
-        // accumulate mode: add this key row's scale * dK (or dV) into the fp32 accumulator row;
-        // this CTA is the only one touching these rows in this call
+        // accumulate mode: add this key row's scale * dK (or dV) into the fp32 accumulator row
+        // (acc_overwrite: store it there); this CTA is the only one touching these rows in this
+        // call
 #pragma unroll 1
         for (int which = 0; which < 2; ++which) {
           const bool is_dk = which == 1;
@@ -700,7 +716,15 @@ __global__ void __launch_bounds__(480, 1)
               tc_fence_before();
               mbar_arrive(is_dk ? dk_free : dv_free);
             }
-            if (key < a.N && w.count > 0) {
+            if (key < a.N && a.acc_overwrite) {
+#pragma unroll
+              for (int cc = 0; cc < 8; ++cc) {
+                const bool z = w.count == 0;
+                *reinterpret_cast<float4*>(accrow + c32 + 4 * cc) =
+                    make_float4(z ? 0.f : __uint_as_float(o[4 * cc + 0]) * mul, z ? 0.f : __uint_as_float(o[4 * cc + 1]) * mul,
+                                z ? 0.f : __uint_as_float(o[4 * cc + 2]) * mul, z ? 0.f : __uint_as_float(o[4 * cc + 3]) * mul);
+              }
+            } else if (key < a.N && w.count > 0) {
 #pragma unroll
               for (int cc = 0; cc < 8; ++cc) {
                 float4* pa = reinterpret_cast<float4*>(accrow + c32 + 4 * cc);
@@ -849,6 +873,13 @@ cudaError_t launch_bwd_main(int d, const CUtensorMap& tq, const CUtensorMap& tk,
   if (d != 128) return cudaErrorNotSupported;
   return with_dq ? launch_bwd_main_t<128, true>(tq, tk, tv, tdo, tdk, tdv, tdq, a, stream)
                  : launch_bwd_main_t<128, false>(tq, tk, tv, tdo, tdk, tdv, tdq, a, stream);
+}
+
+cudaError_t launch_acc_add(float* acc, const float* x, long long elems, cudaStream_t stream) {
+  const long long n4 = elems / 4;
+  fa_acc_add_kernel<<<grid_for(n4, 256), 256, 0, stream>>>(reinterpret_cast<float4*>(acc),
+                                                          reinterpret_cast<const float4*>(x), n4);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_post(const float* dq_acc, void* dq, long long elems, float scale, cudaStream_t stream) {

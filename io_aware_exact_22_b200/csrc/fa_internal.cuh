@@ -47,6 +47,7 @@ struct BwdArgs {
   // fp32 [BH, N, d] accumulators instead of being stored as bf16 (the sequence-sharded backward)
   float* dk_acc = nullptr;
   float* dv_acc = nullptr;
+  int acc_overwrite = 0;  // with dk_acc: store into the accumulators instead of adding
   int group = 1;  // work order: heads per group, heaviest key tile first within a group
   // two ints in device memory, zero before each launch of the key-tile kernel (the pre-kernel
   // zeroes them; the kernel's last CTA zeroes them again on exit): the next unclaimed item
@@ -118,6 +119,8 @@ cudaError_t launch_bwd_main(int d, const CUtensorMap& tq, const CUtensorMap& tk,
 cudaError_t launch_bwd_dq(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a,
                           cudaStream_t stream);
+// acc += x over elems fp32 values (a multiple of 4, 16-byte aligned).
+cudaError_t launch_acc_add(float* acc, const float* x, long long elems, cudaStream_t stream);
 cudaError_t launch_bwd_post(const float* dq_acc, void* dq, long long elems, float scale,
                             cudaStream_t stream);
 

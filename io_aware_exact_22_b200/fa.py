@@ -26,7 +26,8 @@ EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_device_status",
            "fa_status_string", "fa_version", "fa_bwd_noalloc", "fa_selftest_wait_timeout",
            "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_default_splits",
            "fa_bwd_deterministic", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials", "fa_fwd_carry",
-           "fa_bwd_prepare", "fa_bwd_accumulate", "fa_bwd_finish", "fa_bwd_main", "fa_bwd_dq_post",
+           "fa_bwd_prepare", "fa_bwd_accumulate", "fa_bwd_finish", "fa_bwd_contribute", "fa_bwd_acc_add",
+           "fa_bwd_main", "fa_bwd_dq_post",
            "fa_debug_build", "fa_debug_visits")
 # Size of the library's built-in scratch used by fa_bwd_noalloc (include/fa.h).
 NOALLOC_MAX_SCRATCH_BYTES = 64 << 20
@@ -65,6 +66,10 @@ def lib() -> ctypes.CDLL:
         L.fa_bwd_accumulate.restype = i
         L.fa_bwd_finish.argtypes = [vp, sz, vp, vp, vp, vp, vp, i, i, i, i, f, vp]
         L.fa_bwd_finish.restype = i
+        L.fa_bwd_contribute.argtypes = [vp, vp, vp, vp, vp, sz, vp, vp, i, i, i, i, f, i, vp]
+        L.fa_bwd_contribute.restype = i
+        L.fa_bwd_acc_add.argtypes = [vp, vp, i, i, i, i, vp]
+        L.fa_bwd_acc_add.restype = i
         L.fa_bwd_main.argtypes = [vp, vp, vp, vp, vp, sz, vp, vp, i, i, i, i, f, i, vp]
         L.fa_bwd_main.restype = i
         L.fa_bwd_dq_post.argtypes = [vp, sz, vp, i, i, i, i, f, vp]
@@ -162,6 +167,17 @@ def fa_bwd_finish(workspace, workspace_bytes, dk_acc, dv_acc, dq, dk, dv, B, H, 
                   stream=None) -> int:
     return lib().fa_bwd_finish(_ptr(workspace), int(workspace_bytes), _ptr(dk_acc), _ptr(dv_acc),
                                _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale), _stream(stream))
+
+
+def fa_bwd_contribute(q, k, v, dO, workspace, workspace_bytes, dk_out, dv_out, B, H, N, d, scale, causal,
+                      stream=None) -> int:
+    return lib().fa_bwd_contribute(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(workspace), int(workspace_bytes),
+                                   _ptr(dk_out), _ptr(dv_out), B, H, N, d, float(scale), int(causal),
+                                   _stream(stream))
+
+
+def fa_bwd_acc_add(acc, x, B, H, N, d, stream=None) -> int:
+    return lib().fa_bwd_acc_add(_ptr(acc), _ptr(x), B, H, N, d, _stream(stream))
 
 
 def fa_bwd_main(q, k, v, dO, workspace, workspace_bytes, dk, dv, B, H, N, d, scale, causal,

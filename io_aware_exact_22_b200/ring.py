@@ -11,10 +11,12 @@ Attention" (special-jiahao.github.io, section 增量求解 softmax), done inside
 running result is the starting state of the next shard's block loop, which is what makes the
 pieces add up to exact attention over the whole sequence with one running result per rank.
 
-The backward passes each K/V shard round the ring together with fp32 accumulators for its
-dK and dV: every rank adds its queries' contribution (fa_bwd_accumulate, which also adds into
-the rank's own dQ accumulator) before handing the shard on, and one more hop brings every
-shard's accumulators back to its owner, which rounds them to bf16 (fa_bwd_finish).
+The backward passes each K/V shard round the ring, with fp32 accumulators for its dK and dV
+one hop behind it: every rank computes its queries' contribution (fa_bwd_contribute, which
+also adds into the rank's own dQ accumulator) into a local pair while the shard's
+accumulators are still arriving, adds it in (fa_bwd_acc_add) and hands them on while its next
+contribution is computed; one more hop brings every shard's accumulators back to its owner,
+which rounds them to bf16 (fa_bwd_finish).
 
 The exchange has no multicast and no library kernel touches another GPU's memory: each shard
 is received into this rank's own buffers before it is read.  Causal sharding by contiguous
@@ -130,27 +132,50 @@ def ring_attention_forward_local(q_shards, k_shards, v_shards, causal: bool,
 
 
 # ------------------------------------------------------------------------------ backward
-def ring_round(tensors, group=None):
-    """Passes a list of tensors (a K/V shard and its gradient accumulators) round the ring.
-    Yields (step, src, held) for step 0 .. W-1, held being the list of rank src = r - step (its
-    own first); after each yield, when the caller has added into the held accumulators, the held
-    list is sent on to rank r+1 and the next one received from rank r-1.  After the last step
-    the list held is this rank's own again; it is yielded once more with step == W."""
+def ring_accumulate(kv, acc, contribute, B, H, n, d, group=None):
+    """Passes this rank's key/value tensors `kv` round the ring (as ring_pass does: the next list
+    in flight while one is used) and its fp32 gradient accumulators `acc` (a list of [B, H, n, d]
+    tensors) one hop behind them, and returns `acc` back home with every rank's contribution.
+
+    At step s the rank holds the key/values of rank src = r - s.  contribute(src, kv_src,
+    targets, add) writes this rank's contribution to src's accumulators into `targets` (a list
+    shaped like acc), added into them when `add` is true and stored over them otherwise, and
+    returns the indices it wrote.  Step 0 adds straight into this rank's own accumulators.  From
+    step 1 on the contribution is stored into a local set while src's accumulators are still on
+    their way from rank r-1; once both are done the local set is added in (fa_bwd_acc_add) and
+    the accumulators are sent on to rank r+1, so that each hop of the accumulators overlaps the
+    next step's products instead of following them.  Every rank must take part."""
     W = dist.get_world_size(group)
     r = dist.get_rank(group)
+    if W == 1:
+        contribute(r, list(kv), acc, True)
+        return acc
     nxt, prv = _peer(group, (r + 1) % W), _peer(group, (r - 1) % W)
-    cur = list(tensors)
-    bufs = [[torch.empty_like(t) for t in cur] for _ in range(2)] if W > 1 else []
-    for step in range(W):
-        yield step, (r - step) % W, cur
-        if W > 1:
-            nb = bufs[step % 2]
-            ops = [dist.P2POp(dist.isend, t, nxt, group) for t in cur]
-            ops += [dist.P2POp(dist.irecv, t, prv, group) for t in nb]
-            for rq in dist.batch_isend_irecv(ops):
+    local = [[torch.empty_like(a) for a in acc] for _ in range(2)]
+    rbuf = [[torch.empty_like(a) for a in acc] for _ in range(2)]
+    cur = acc
+    recv_reqs, send_reqs = [], []
+    for step, (src, kv_src) in enumerate(ring_pass(list(kv), group)):
+        if step == 0:
+            contribute(src, kv_src, cur, True)
+        else:
+            loc = local[step % 2]
+            wrote = contribute(src, kv_src, loc, False)
+            for rq in recv_reqs:  # src's accumulators have arrived
                 rq.wait()
-            cur = nb
-    yield W, r, cur
+            cur = rbuf[(step - 1) % 2]
+            for i in wrote:
+                _ok(fa.fa_bwd_acc_add(cur[i], loc[i], B, H, n, d), "fa_bwd_acc_add")
+        for rq in send_reqs:  # the buffers about to receive were sent from one step ago
+            rq.wait()
+        target = rbuf[step % 2]
+        sends = [dist.P2POp(dist.isend, t, nxt, group) for t in cur]
+        recvs = [dist.P2POp(dist.irecv, t, prv, group) for t in target]
+        reqs = dist.batch_isend_irecv(sends + recvs)
+        send_reqs, recv_reqs = reqs[:len(sends)], reqs[len(sends):]
+    for rq in recv_reqs + send_reqs:
+        rq.wait()
+    return rbuf[(W - 1) % 2]
 
 
 def _check_bwd(*ts):
@@ -181,14 +206,16 @@ def ring_attention_backward(q, k, v, o, do, lse, causal: bool, scale: float | No
     _ok(fa.fa_bwd_prepare(o, do, lse, ws, wsb, B, H, n, d), "fa_bwd_prepare")
     acc = [torch.zeros(q.shape, device=q.device, dtype=torch.float32) for _ in range(2)]
     vis = visible_shards(r, W, causal)
-    home = None
-    for step, src, (ks, vs, dka, dva) in ring_round([k, v, acc[0], acc[1]], group):
-        if step == W:
-            home = (dka, dva)
-            break
-        if src in vis:
-            _ok(fa.fa_bwd_accumulate(q, ks, vs, do, ws, wsb, dka, dva, B, H, n, d, scale, vis[src]),
-                "fa_bwd_accumulate")
+
+    def contribute(src, kv_src, targets, add):
+        if src not in vis:
+            return []
+        call = fa.fa_bwd_accumulate if add else fa.fa_bwd_contribute
+        _ok(call(q, kv_src[0], kv_src[1], do, ws, wsb, targets[0], targets[1], B, H, n, d, scale, vis[src]),
+            "fa_bwd_accumulate" if add else "fa_bwd_contribute")
+        return [0, 1]
+
+    home = ring_accumulate([k, v], acc, contribute, B, H, n, d, group)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
@@ -199,8 +226,10 @@ def ring_attention_backward(q, k, v, o, do, lse, causal: bool, scale: float | No
 def ring_attention_backward_local(q_shards, k_shards, v_shards, o_shards, do_shards, lse_shards,
                                   causal: bool, scale: float | None = None):
     """The same computation for all W shards on one device: every rank's contributions in its
-    ring order, each shard's accumulators shared instead of passed on.  Returns
-    [(dQ_r, dK_r, dV_r)]."""
+    ring order, each shard's accumulators shared instead of passed on (a rank's contribution
+    to another shard still goes through a local pair, fa_bwd_contribute and fa_bwd_acc_add, as
+    on the ring).
+    Returns [(dQ_r, dK_r, dV_r)]."""
     W = len(q_shards)
     _check_bwd(*q_shards, *k_shards, *v_shards, *o_shards, *do_shards)
     for lse, q in zip(lse_shards, q_shards):
@@ -214,13 +243,22 @@ def ring_attention_backward_local(q_shards, k_shards, v_shards, o_shards, do_sha
     for r in range(W):
         _ok(fa.fa_bwd_prepare(o_shards[r], do_shards[r], lse_shards[r], wss[r], wsb, B, H, n, d),
             "fa_bwd_prepare")
+    loc = [torch.empty_like(dka[0]), torch.empty_like(dka[0])]
     for r in range(W):
         vis = visible_shards(r, W, causal)
         for step in range(W):
             src = (r - step) % W
-            if src in vis:
-                _ok(fa.fa_bwd_accumulate(q_shards[r], k_shards[src], v_shards[src], do_shards[r], wss[r], wsb,
-                                         dka[src], dva[src], B, H, n, d, scale, vis[src]), "fa_bwd_accumulate")
+            if src not in vis:
+                continue
+            # as ring_accumulate does: the own shard straight into its accumulators, the others
+            # stored into a local pair that is then added in
+            tgt = (dka[src], dva[src]) if step == 0 else loc
+            call = fa.fa_bwd_accumulate if step == 0 else fa.fa_bwd_contribute
+            _ok(call(q_shards[r], k_shards[src], v_shards[src], do_shards[r], wss[r], wsb, tgt[0], tgt[1], B, H, n, d,
+                     scale, vis[src]), "fa_bwd_accumulate" if step == 0 else "fa_bwd_contribute")
+            if step > 0:
+                _ok(fa.fa_bwd_acc_add(dka[src], loc[0], B, H, n, d), "fa_bwd_acc_add")
+                _ok(fa.fa_bwd_acc_add(dva[src], loc[1], B, H, n, d), "fa_bwd_acc_add")
     outs = []
     for r in range(W):
         g = [torch.empty_like(q_shards[r]) for _ in range(3)]
@@ -340,18 +378,23 @@ def ring_attention_forward_zigzag_local(q, k, v, W: int, causal: bool, scale: fl
     return o, lse
 
 
-def _zigzag_backward(q2, do2, ws2, wsb, round_iter, r, W, causal, scale):
-    """Adds rank r's contributions into every key chunk's dK/dV accumulators as they come round
-    (round_iter yields (step, src, [k_a, k_b, v_a, v_b, dk_a, dk_b, dv_a, dv_b]) and, at
-    step W, this rank's own list back); returns this rank's own [dk_a, dk_b, dv_a, dv_b]."""
+def _zigzag_contribute(q2, do2, ws2, wsb, r, W, causal, scale):
+    """contribute() for ring_accumulate in the zig-zag layout: rank r's pieces with rank src's
+    key chunks (kv_src = [k_a, k_b, v_a, v_b]) added into targets = [dk_a, dk_b, dv_a, dv_b]."""
     B, H, n, d = q2[0].shape
-    for step, src, held in round_iter:
-        if step == W:
-            return held[4:]
+
+    def contribute(src, kv_src, targets, add):
+        wrote = set()
         for iq, ik, masked in zigzag_pieces(r, W, src, causal):
-            _ok(fa.fa_bwd_accumulate(q2[iq], held[ik], held[2 + ik], do2[iq], ws2[iq], wsb, held[4 + ik],
-                                     held[6 + ik], B, H, n, d, scale, masked), "fa_bwd_accumulate")
-    raise RuntimeError("the ring ended before the accumulators came home")
+            # a key chunk's first piece of the step stores (unless adding), its second adds
+            first = ik not in wrote
+            call = fa.fa_bwd_contribute if (first and not add) else fa.fa_bwd_accumulate
+            _ok(call(q2[iq], kv_src[ik], kv_src[2 + ik], do2[iq], ws2[iq], wsb, targets[ik], targets[2 + ik],
+                     B, H, n, d, scale, masked), "fa_bwd_contribute" if (first and not add) else "fa_bwd_accumulate")
+            wrote.update((ik, 2 + ik))
+        return sorted(wrote)
+
+    return contribute
 
 
 def ring_attention_backward_zigzag(q2, k2, v2, o2, do2, lse2, causal: bool, scale: float | None = None,
@@ -371,8 +414,8 @@ def ring_attention_backward_zigzag(q2, k2, v2, o2, do2, lse2, causal: bool, scal
     for i in range(2):
         _ok(fa.fa_bwd_prepare(o2[i], do2[i], lse2[i], ws2[i], wsb, B, H, n, d), "fa_bwd_prepare")
     acc = [torch.zeros(q2[0].shape, device=q2[0].device, dtype=torch.float32) for _ in range(4)]
-    home = _zigzag_backward(q2, do2, ws2, wsb, ring_round([k2[0], k2[1], v2[0], v2[1], *acc], group), r, W,
-                            causal, scale)
+    home = ring_accumulate([k2[0], k2[1], v2[0], v2[1]], acc,
+                           _zigzag_contribute(q2, do2, ws2, wsb, r, W, causal, scale), B, H, n, d, group)
     dq2, dk2, dv2 = [], [], []
     for i in range(2):
         g = [torch.empty_like(q2[i]) for _ in range(3)]
@@ -404,14 +447,27 @@ def ring_attention_backward_zigzag_local(q, k, v, o, do, lse, W: int, causal: bo
         _ok(fa.fa_bwd_prepare(co[c], cdo[c], clse[c], ws[c], wsb, B, H, n, d), "fa_bwd_prepare")
     dka = [torch.zeros(cq[0].shape, device=q.device, dtype=torch.float32) for _ in range(2 * W)]
     dva = [torch.zeros_like(t) for t in dka]
+    loc = [torch.empty_like(dka[0]) for _ in range(4)]  # [dk_a, dk_b, dv_a, dv_b] of a step
     for r in range(W):
         a = zigzag_chunks(r, W)
         for step in range(W):
             src = (r - step) % W
             b = zigzag_chunks(src, W)
+            # as ring_accumulate does: the own chunks straight into their accumulators, the others
+            # stored into local ones (a chunk's second piece of the step added) that are then
+            # added in
+            wrote = set()
             for iq, ik, masked in zigzag_pieces(r, W, src, causal):
-                _ok(fa.fa_bwd_accumulate(cq[a[iq]], ck[b[ik]], cv[b[ik]], cdo[a[iq]], ws[a[iq]], wsb, dka[b[ik]],
-                                         dva[b[ik]], B, H, n, d, scale, masked), "fa_bwd_accumulate")
+                tk, tv = (dka[b[ik]], dva[b[ik]]) if step == 0 else (loc[ik], loc[2 + ik])
+                store = step > 0 and ik not in wrote
+                call = fa.fa_bwd_contribute if store else fa.fa_bwd_accumulate
+                _ok(call(cq[a[iq]], ck[b[ik]], cv[b[ik]], cdo[a[iq]], ws[a[iq]], wsb, tk, tv, B, H, n, d, scale,
+                         masked), "fa_bwd_contribute" if store else "fa_bwd_accumulate")
+                wrote.add(ik)
+            if step > 0:
+                for ik in sorted(wrote):
+                    _ok(fa.fa_bwd_acc_add(dka[b[ik]], loc[ik], B, H, n, d), "fa_bwd_acc_add")
+                    _ok(fa.fa_bwd_acc_add(dva[b[ik]], loc[2 + ik], B, H, n, d), "fa_bwd_acc_add")
     dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
     for c in range(2 * W):
         g = [torch.empty_like(cq[c]) for _ in range(3)]

@@ -15,8 +15,8 @@ class FakeFA:
     result into the running one the same way (or starts it), and writes it back or, with
     FA_CARRY_FINAL, to the output; fa_bwd_prepare keeps D = rowsum(dO o O) and
     LSE with a zeroed dQ accumulator in the workspace; fa_bwd_accumulate adds dS K into that
-    accumulator and scale dS^T Q, P^T dO into the dK, dV accumulators; fa_bwd_finish writes
-    scale * dQ and the two accumulators."""
+    accumulator and scale dS^T Q, P^T dO into the dK, dV accumulators (fa_bwd_contribute stores
+    them there instead); fa_bwd_acc_add adds one accumulator into another; fa_bwd_finish writes scale * dQ and the two accumulators."""
 
     def __init__(self):
         self.ws = {}
@@ -80,6 +80,15 @@ class FakeFA:
         ds = p * (dO.double() @ v.double().transpose(-1, -2) - st["D"][..., None])
         dk_acc += (scale * ds.transpose(-1, -2) @ q.double()).to(dk_acc.dtype)
         st["dq"] += ds @ k.double()
+        return 0
+
+    def fa_bwd_contribute(self, q, k, v, dO, ws, wsb, dk_out, dv_out, B, H, n, d, scale, causal, stream=None):
+        dk_out.zero_()
+        dv_out.zero_()
+        return self.fa_bwd_accumulate(q, k, v, dO, ws, wsb, dk_out, dv_out, B, H, n, d, scale, causal)
+
+    def fa_bwd_acc_add(self, acc, x, B, H, n, d, stream=None):
+        acc += x
         return 0
 
     def fa_bwd_finish(self, ws, wsb, dk_acc, dv_acc, dq, dk, dv, B, H, n, d, scale, stream=None):

@@ -134,21 +134,29 @@ def _round_main(rank, world, port, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        own = [torch.full((2, 3), float(rank)), torch.zeros(2, 3)]
-        seen, home = [], None
-        for step, src, held in ring.ring_round(own):
-            if step == world:
-                home = (float(held[0][0, 0]), float(held[1][1, 1]))
-                break
-            seen.append((src, float(held[0][0, 0])))
-            held[1] += rank + 1  # this rank's contribution to shard src's accumulator
-        q.put((rank, seen, home))
+        use_fakes()  # fa_bwd_acc_add on CPU tensors
+        seen = []
+
+        def contribute(src, kv_src, targets, add):
+            seen.append((src, float(kv_src[0][0, 0])))
+            # this rank's contribution to shard src's accumulator, added or stored
+            if add:
+                targets[0] += rank + 1
+            else:
+                targets[0].fill_(rank + 1)
+            return [0]
+
+        home = ring.ring_accumulate([torch.full((2, 3), float(rank))], [torch.zeros(2, 3)], contribute,
+                                    1, 1, 2, 3)
+        q.put((rank, seen, float(home[0][1, 1])))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [2, 3, 4])
 def test_ring_round_trip_on_gloo_ranks(world):
+    # the key/value lists go round ahead, the accumulators one hop behind; each accumulator
+    # comes home with every rank's contribution added once
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
@@ -162,11 +170,10 @@ def test_ring_round_trip_on_gloo_ranks(world):
     for r in range(world):
         seen, home = res[r]
         assert seen == [((r - s) % world, float((r - s) % world)) for s in range(world)]
-        # back home: this rank's own shard, with every rank's contribution added
-        assert home == (float(r), float(world * (world + 1) // 2))
+        assert home == float(world * (world + 1) // 2)
 
 
-@pytest.mark.parametrize("fn", ["prepare", "accumulate", "finish"])
+@pytest.mark.parametrize("fn", ["prepare", "accumulate", "contribute", "finish", "acc_add"])
 def test_backward_pieces_reject_other_d_and_null(fn):
     a = A16
     if fn == "prepare":
@@ -177,9 +184,50 @@ def test_backward_pieces_reject_other_d_and_null(fn):
         assert fa.fa_bwd_accumulate(a, a, a, a, a, 1 << 30, a, a, 1, 2, 256, 96, 0.1, 0, 0) == UNSUPPORTED
         assert fa.fa_bwd_accumulate(a, a, a, a, a, 1 << 30, 0, a, 1, 2, 256, 128, 0.1, 0, 0) == INVALID
         assert fa.fa_bwd_accumulate(a, a, a, a, a, 1 << 30, a + 4, a, 1, 2, 256, 128, 0.1, 0, 0) == INVALID
-    else:
+    elif fn == "contribute":
+        assert fa.fa_bwd_contribute(a, a, a, a, a, 1 << 30, a, a, 1, 2, 256, 96, 0.1, 0, 0) == UNSUPPORTED
+        assert fa.fa_bwd_contribute(a, a, a, a, a, 1 << 30, a, 0, 1, 2, 256, 128, 0.1, 0, 0) == INVALID
+        assert fa.fa_bwd_contribute(a, a, a, a, a, 100, a, a, 1, 2, 256, 128, 0.1, 0, 0) == INVALID
+    elif fn == "finish":
         assert fa.fa_bwd_finish(a, 1 << 30, a, a, a, a, a, 1, 2, 256, 96, 0.1, 0) == UNSUPPORTED
         assert fa.fa_bwd_finish(a, 1 << 30, a, a, 0, a, a, 1, 2, 256, 128, 0.1, 0) == INVALID
+    else:
+        assert fa.fa_bwd_acc_add(a, a, 1, 2, 256, 96, 0) == UNSUPPORTED
+        assert fa.fa_bwd_acc_add(0, a, 1, 2, 256, 128, 0) == INVALID
+        assert fa.fa_bwd_acc_add(a, a + 4, 1, 2, 256, 128, 0) == INVALID
+        assert fa.fa_bwd_acc_add(a, a, 1, 0, 256, 128, 0) == 0  # empty: nothing to do
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("causal", [True, False])
+def test_contribution_is_the_accumulation_into_zeros(cuda_ok, causal):
+    # fa_bwd_contribute stores exactly what fa_bwd_accumulate adds into zeroed accumulators,
+    # over accumulators that hold anything; every row is written
+    w = custom(2, 3, 333, 128, causal, seed=8, backward=True)
+    q, k, v, do = (t.cuda() for t in make_inputs(w))
+    B, H, n, d = w.shape
+    o, lse = fa.forward(q, k, v, causal, w.scale)
+    wsb = fa.fa_bwd_workspace_bytes(B, H, n, d)
+    ws = torch.empty(wsb, device="cuda", dtype=torch.uint8)
+    assert fa.fa_bwd_prepare(o, do, lse, ws, wsb, B, H, n, d) == 0
+    za, zb = (torch.zeros(q.shape, device="cuda", dtype=torch.float32) for _ in range(2))
+    sa, sb = (torch.full(q.shape, float("nan"), device="cuda", dtype=torch.float32) for _ in range(2))
+    assert fa.fa_bwd_accumulate(q, k, v, do, ws, wsb, za, zb, B, H, n, d, w.scale, int(causal)) == 0
+    assert fa.fa_bwd_contribute(q, k, v, do, ws, wsb, sa, sb, B, H, n, d, w.scale, int(causal)) == 0
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status() == 0
+    assert torch.equal(sa, za) and torch.equal(sb, zb)
+
+
+@pytest.mark.gpu
+def test_accumulator_add_is_the_elementwise_sum(cuda_ok):
+    g = torch.Generator().manual_seed(3)
+    acc = torch.randn(2, 3, 129, 64, generator=g).cuda()
+    x = torch.randn(2, 3, 129, 64, generator=g).cuda()
+    want = acc + x
+    assert fa.fa_bwd_acc_add(acc, x, 2, 3, 129, 64) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(acc, want)
 
 
 @pytest.mark.gpu
