@@ -291,7 +291,7 @@ def _sharded_main(rank, world, port, n, causal, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [2, 3, 4])
 @pytest.mark.parametrize("causal", [True, False])
 def test_sharded_forward_and_backward_on_gloo_ranks(world, causal):
     ctx = mp.get_context("spawn")

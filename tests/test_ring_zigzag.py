@@ -105,7 +105,7 @@ def _rank_main(rank, world, port, n, causal, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [2, 3, 4])
 @pytest.mark.parametrize("causal", [True, False])
 def test_zigzag_on_gloo_ranks(world, causal):
     ctx = mp.get_context("spawn")
