@@ -135,7 +135,9 @@ def ring_attention_forward_local(q_shards, k_shards, v_shards, causal: bool,
 def ring_accumulate(kv, acc, contribute, B, H, n, d, group=None):
     """Passes this rank's key/value tensors `kv` round the ring (as ring_pass does: the next list
     in flight while one is used) and its fp32 gradient accumulators `acc` (a list of [B, H, n, d]
-    tensors) one hop behind them, and returns `acc` back home with every rank's contribution.
+    tensors) one hop behind them, and returns this rank's accumulators as they come back home
+    with every rank's contribution (in one of its receive buffers; `acc` itself is the set that
+    left at step 0).
 
     At step s the rank holds the key/values of rank src = r - s.  contribute(src, kv_src,
     targets, add) writes this rank's contribution to src's accumulators into `targets` (a list
