@@ -60,10 +60,12 @@ struct FwdCfg {
   static constexpr int KV_OFF = 2 * TILE;
   static constexpr int P_OFF = KV_OFF + NS * TILE;  // ring and P tiles together stage partial outputs
   static constexpr int BAR_OFF = P_OFF + 2 * PTILE;
-  // O staging, tile t at OST_OFF + t * OST_STRIDE: the dead P tile (bf16; the Q tiles may
-  // already hold the next item's queries) or the idle K/V ring (FP8, one item per CTA)
-  static constexpr int OST_OFF = FP8 ? KV_OFF : P_OFF;
-  static constexpr int OST_STRIDE = FP8 ? OTILE : PTILE;
+  // O staging, tile t at OST_OFF + t * OST_STRIDE: the dead P tile (the Q tiles may already
+  // hold the next item's queries), OST_BOXES 64-column boxes of bf16 output at a time (FP8:
+  // one, its P tile being half a tile's output; the output then goes in two passes)
+  static constexpr int OST_OFF = P_OFF;
+  static constexpr int OST_STRIDE = PTILE;
+  static constexpr int OST_BOXES = PTILE / 16384;
   // barriers: q_full, q_empty, kv_full[NS], kv_empty[NS], s_full[2], s_free[2], p_full[2],
   // pv_done[2], o_full[2], o_free[2], s_done, pv_end
   static constexpr int NBAR = 2 + 2 * NS + 12 + 2;
@@ -102,7 +104,7 @@ __global__ void __launch_bounds__(352, 1)
                   const FwdArgs a) {
   static_assert(!FP8 || (D == 128 && !PARTIAL), "FP8: d = 128, whole key range");
   using C = FwdCfg<D, FP8>;
-  constexpr bool kOutInP = !PARTIAL && !FP8;  // the output is staged in the tile's own P tile
+  constexpr bool kOutInP = !PARTIAL;  // the output is staged in the tile's own P tile
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
@@ -363,9 +365,9 @@ __global__ void __launch_bounds__(352, 1)
               issue_pv(t ? C::T_O1 : C::T_O0, (uint32_t)(t * C::PTILE), stage_addr(itV), j > 0 || carry);
               mma_commit_e(pv_done(t));
               ++cp[t];
-              // bf16, whole key range: O_t of this item is complete once this product is (its
-              // output is staged in P_t, which no other product reads).  Split and FP8 outputs
-              // are staged in the K/V ring, idle only once every product of the item is done.
+              // whole key range: O_t of this item is complete once this product is (its output is
+              // staged in P_t, which no other product reads).  Split outputs are staged in the K/V
+              // ring, idle only once every product of the item is done.
               if (kOutInP && j == nt[t] - 1) {
                 mma_commit_e(o_full(t));
                 ++co[t];
@@ -632,39 +634,51 @@ __global__ void __launch_bounds__(352, 1)
         const float inv = (l > 0.f) ? vmul / l : 0.f;
         const int row0 = wk.q0 + 128 * t + 32 * wq;
         if (!PARTIAL) {
-          // P_t (bf16) or the K/V ring (FP8) is dead once o_full has fired; each warp stages
-          // and stores its own 32 rows, the rows whose P it writes
+          // P_t is dead once o_full has fired; each warp stages and stores its own 32 rows, the
+          // rows whose P it writes, OST_BOXES 64-column boxes per pass (FP8: two passes, the
+          // second after the first store has read the staging)
           uint8_t* stage = gb + C::OST_OFF + t * C::OST_STRIDE;
 #pragma unroll
-          for (int b = 0; b < D / 64; ++b) {
+          for (int b0 = 0; b0 < D / 64; b0 += C::OST_BOXES) {
+            if (b0 > 0) {
+              if (lane == 0) bulk_wait_read0();
+              __syncwarp();
+            }
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              uint32_t o[32];
-              tmem_ld32(tOrow + 64 * b + 32 * h, o);
-              tmem_wait_ld();
-              reg_fence(o);
+            for (int bb = 0; bb < C::OST_BOXES && b0 + bb < D / 64; ++bb) {
+              const int b = b0 + bb;
 #pragma unroll
-              for (int cc = 0; cc < 4; ++cc) {
-                uint4 v;
-                v.x = pack_bf16(__uint_as_float(o[8 * cc + 0]) * inv, __uint_as_float(o[8 * cc + 1]) * inv);
-                v.y = pack_bf16(__uint_as_float(o[8 * cc + 2]) * inv, __uint_as_float(o[8 * cc + 3]) * inv);
-                v.z = pack_bf16(__uint_as_float(o[8 * cc + 4]) * inv, __uint_as_float(o[8 * cc + 5]) * inv);
-                v.w = pack_bf16(__uint_as_float(o[8 * cc + 6]) * inv, __uint_as_float(o[8 * cc + 7]) * inv);
-                const int chunk = h * 4 + cc;  // 16-byte chunk within the 128-byte row
-                *reinterpret_cast<uint4*>(stage + b * 16384 + r * 128 + ((chunk ^ (r & 7)) << 4)) = v;
+              for (int h = 0; h < 2; ++h) {
+                uint32_t o[32];
+                tmem_ld32(tOrow + 64 * b + 32 * h, o);
+                tmem_wait_ld();
+                reg_fence(o);
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                  uint4 v;
+                  v.x = pack_bf16(__uint_as_float(o[8 * cc + 0]) * inv, __uint_as_float(o[8 * cc + 1]) * inv);
+                  v.y = pack_bf16(__uint_as_float(o[8 * cc + 2]) * inv, __uint_as_float(o[8 * cc + 3]) * inv);
+                  v.z = pack_bf16(__uint_as_float(o[8 * cc + 4]) * inv, __uint_as_float(o[8 * cc + 5]) * inv);
+                  v.w = pack_bf16(__uint_as_float(o[8 * cc + 6]) * inv, __uint_as_float(o[8 * cc + 7]) * inv);
+                  const int chunk = h * 4 + cc;  // 16-byte chunk within the 128-byte row
+                  *reinterpret_cast<uint4*>(stage + bb * 16384 + r * 128 + ((chunk ^ (r & 7)) << 4)) = v;
+                }
               }
             }
+            if (b0 + C::OST_BOXES >= D / 64) {
+              tc_fence_before();
+              mbar_arrive(o_free(t));  // O_t is read: the next item's first P V may overwrite it
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && row0 < a.N) {
+              for (int bb = 0; bb < C::OST_BOXES && b0 + bb < D / 64; ++bb)
+                tma_store_3d(&tmO, sb + C::OST_OFF + t * C::OST_STRIDE + bb * 16384 + wq * 4096, 64 * (b0 + bb),
+                             row0, bh);
+              bulk_commit();
+            }
+            __syncwarp();
           }
-          tc_fence_before();
-          mbar_arrive(o_free(t));  // O_t is read: the next item's first P V may overwrite it
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0 && row0 < a.N) {
-            for (int b = 0; b < D / 64; ++b)
-              tma_store_3d(&tmO, sb + C::OST_OFF + t * C::OST_STRIDE + b * 16384 + wq * 4096, 64 * b, row0, bh);
-            bulk_commit();
-          }
-          __syncwarp();
           store_pending = true;  // waited for before this warp next writes P_t, or at exit
           if (qrow < a.N)
             a.lse[(size_t)bh * a.N + qrow] =
@@ -725,7 +739,8 @@ static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, co
   static_assert(C::SMEM <= 232448, "shared memory budget");
   static_assert(C::SMEM > 116 * 1024, "one CTA per SM: each allocates all 512 TMEM columns");
   static_assert(2 * 128 * D * 4 <= C::NS * C::TILE + 2 * C::PTILE, "partial-output staging must fit the ring and P");
-  static_assert(C::OTILE <= C::OST_STRIDE && C::OST_OFF + C::OST_STRIDE + C::OTILE <= C::BAR_OFF,
+  static_assert(C::OST_BOXES >= 1 && C::OST_BOXES * 16384 <= C::OST_STRIDE &&
+                    C::OST_OFF + 2 * C::OST_STRIDE <= C::BAR_OFF,
                 "output staging must fit");
   static bool attr_set[64];  // per device: the attribute outlives the call
   int dev = 0;
@@ -741,8 +756,8 @@ static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, co
   FwdArgs b = a;
   long long grid = items;
   b.persistent = 0;
-  if (!PARTIAL && !FP8) {
-    // The whole key range in bf16: at most one CTA per SM, each walking its pairs of items,
+  if (!PARTIAL) {
+    // The whole key range (bf16 or FP8): at most one CTA per SM, each walking its pairs of items,
     // when the items are of equal length (no mask) or many per SM.  Under the causal mask with
     // few items per SM the hardware's dispatch of one CTA per item (to whichever SM frees up
     // first) balances the uneven items better.  Measured on B200: persistent is 1-3 % faster
